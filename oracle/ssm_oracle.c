@@ -1,0 +1,156 @@
+/*
+ * Selective-scan forward ORACLE: plain, slow, float64, sequential in time.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path may call, link or
+ * load this file; only the test suite, the smoke check and the bench's CPU
+ * baseline leg use it. It shares no code, header, table or helper with the
+ * CUDA library.
+ *
+ * What it computes follows the recurrence spelled out on the page
+ *   "Mamba: Linear-Time Sequence Modeling with Selective State Spaces"
+ *   (www.abhik.ai/papers/mamba), section "Original paper, equations and
+ *   runnable CPU code", row "2. Retain, write and read each channel's state":
+ *       a[t,c,n] = exp(delta[t,c] * A[c,n])
+ *       h[t,c,n] = a[t,c,n] * h[t-1,c,n] + delta[t,c] * B[t,n] * x[t,c]
+ *       y[t,c]   = sum_n C[t,n] * h[t,c,n] + D[c] * x[t,c]
+ *   read AFTER the state update, with an optional incoming state; and row
+ *   "1. Produce coefficients from the locally mixed input":
+ *       delta = softplus(raw + b_delta),  A = -exp(A_log)
+ *   and row "5. Put the selective operator inside the complete mixer":
+ *       the scan result (D*x already included) is multiplied by SiLU(z).
+ * The same loop, without D, is the sequential reference on the page
+ *   "mamba, from scratch | khushi keswani", section "the scan".
+ *
+ * Readings taken where the pages leave a step open:
+ *   - softplus is PyTorch's default F.softplus (beta 1, threshold 20: the
+ *     identity above 20), the function the page's coefficient code calls;
+ *   - the delta bias is added per channel before softplus; with the softplus
+ *     flag off, delta = raw + bias as given;
+ *   - D == NULL means no direct path (the page's d=None), z == NULL means no
+ *     gate, h0 == NULL means a zero incoming state;
+ *   - the write term is evaluated as (delta * B) * x, the page's order;
+ *   - the readout sums n in ascending order.
+ *
+ * Layouts (all contiguous, row-major, float64):
+ *   x, delta, z, y : [batch, seqlen, dim]        (dim = expanded channels E)
+ *   B, C           : [batch, seqlen, dstate]     (shared by every channel)
+ *   A_log          : [dim, dstate]
+ *   D, delta_bias  : [dim]
+ *   h0, h_last     : [batch, dim, dstate]
+ *   states         : [batch, seqlen, dim, dstate]  (optional: every state)
+ *
+ * Parallelism: independent (batch, channel) pairs are spread over OpenMP
+ * threads; each pair's loop over time stays strictly sequential.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* PyTorch F.softplus with its defaults (beta = 1, threshold = 20). */
+static double softplus_default(double v)
+{
+    if (v > 20.0)
+        return v;
+    return log1p(exp(v));
+}
+
+/* SiLU(z) = z * sigmoid(z) = z / (1 + exp(-z)). */
+static double silu(double z)
+{
+    return z / (1.0 + exp(-z));
+}
+
+/* Step size for one (b, t, c): raw + bias, then softplus if enabled. */
+double ssm_oracle_step_size(double raw, double bias, int delta_softplus)
+{
+    double v = raw + bias;
+    return delta_softplus ? softplus_default(v) : v;
+}
+
+/* Retention a = exp(delta * A) with A = -exp(A_log). */
+double ssm_oracle_retention(double step, double a_log)
+{
+    double A = -exp(a_log);
+    return exp(step * A);
+}
+
+/*
+ * Returns 0 on success, -1 on a bad argument (NULL required pointer or a
+ * non-positive size). The output y must not alias any input.
+ */
+int ssm_oracle_scan(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                    const double *x, const double *delta, const double *A_log,
+                    const double *B, const double *C, const double *D,
+                    const double *z, const double *delta_bias,
+                    int delta_softplus, const double *h0,
+                    double *y, double *h_last, double *states, int nthreads)
+{
+    if (!x || !delta || !A_log || !B || !C || !y)
+        return -1;
+    if (batch <= 0 || seqlen <= 0 || dim <= 0 || dstate <= 0)
+        return -1;
+
+    const int64_t pairs = batch * dim;
+#ifdef _OPENMP
+    if (nthreads <= 0)
+        nthreads = omp_get_max_threads();
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+#else
+    (void)nthreads;
+#endif
+    for (int64_t p = 0; p < pairs; ++p) {
+        const int64_t b = p / dim;
+        const int64_t c = p % dim;
+        double *A = (double *)malloc((size_t)dstate * sizeof(double));
+        double *h = (double *)malloc((size_t)dstate * sizeof(double));
+        for (int64_t n = 0; n < dstate; ++n) {
+            A[n] = -exp(A_log[c * dstate + n]);
+            h[n] = h0 ? h0[(b * dim + c) * dstate + n] : 0.0;
+        }
+        const double bias = delta_bias ? delta_bias[c] : 0.0;
+        for (int64_t t = 0; t < seqlen; ++t) {
+            const int64_t i = (b * seqlen + t) * dim + c;   /* [b, t, c] */
+            const int64_t r = (b * seqlen + t) * dstate;    /* row of B, C */
+            const double v = delta[i] + bias;
+            const double step = delta_softplus ? softplus_default(v) : v;
+            const double xv = x[i];
+            for (int64_t n = 0; n < dstate; ++n) {
+                const double retention = exp(step * A[n]);
+                const double write = step * B[r + n] * xv;
+                h[n] = retention * h[n] + write;
+            }
+            if (states) {
+                double *s = states + ((b * seqlen + t) * dim + c) * dstate;
+                for (int64_t n = 0; n < dstate; ++n)
+                    s[n] = h[n];
+            }
+            double out = 0.0;
+            for (int64_t n = 0; n < dstate; ++n)
+                out += C[r + n] * h[n];
+            if (D)
+                out += D[c] * xv;
+            if (z)
+                out *= silu(z[i]);
+            y[i] = out;
+        }
+        if (h_last)
+            for (int64_t n = 0; n < dstate; ++n)
+                h_last[(b * dim + c) * dstate + n] = h[n];
+        free(A);
+        free(h);
+    }
+    return 0;
+}
+
+/* Number of OpenMP threads a parallel region would use (1 without OpenMP). */
+int ssm_oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
