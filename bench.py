@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Benchmark of the fused selective-scan forward pass on B200.
+
+One step = one call of ssm_scan_fwd over the whole workload (every step of the
+scan: softplus step size, retention exp, write, recurrence, readout, D skip,
+SiLU gate, y and h_last stores). Default workload: the Mamba-2.8B-shaped layer
+(b=4, L=8192, E=5120, N=16, bfloat16 activations, float32 state), synthetic
+seeded inputs (selective_state_space_51_b200.workloads, shape 3).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--shape I]
+                    [--impl reference]
+
+Prints ONE JSON line (rank 0). Multi-GPU runs are launched by torchrun with
+one process per GPU; each rank scans its own batch of sequences (weak
+scaling, no collective on the data path); the time is the max over ranks.
+
+The metric: scan elements (b*L*E*N) per second, with the achieved GB/s of
+algorithmic traffic and the fraction of the min(HBM, SFU-exp) roofline:
+T_roof = max(bytes / HBM peak, exps / SFU peak), fraction = T_roof / T.
+`--impl reference` times the float64 CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("selective-scan fwd GB/s and (b·L·E·N)/s; "
+          "% of min(HBM, SFU-exp) roofline")
+UNIT = "scan elements/s"
+SFU_EX2_PER_CLK_PER_SM = 16      # MUFU.EX2 lanes per clock per SM
+HBM_NOMINAL_GBS = 8000.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}
+
+
+# ----------------------------------------------------------------- sharding
+def shard_for_rank(rank: int, world: int, shape: int = 3):
+    """Weak scaling: rank r scans its own batch of sequences, drawn with its
+    own seed (the r-th slice of a global batch of world * b sequences)."""
+    if not 0 <= rank < world:
+        raise ValueError("rank %d outside world %d" % (rank, world))
+    return {"shape": shape, "seed": 51000 + shape + 1000 * rank,
+            "global_batch_offset": rank}
+
+
+def max_over_ranks(value: float, dist=None, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity without a group)."""
+    if dist is None or not dist.is_initialized():
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- workload
+def algorithmic_bytes(wl) -> int:
+    """Each input read once, y written once, h0/h_last once; no [b,L,E,N]."""
+    b, L, E, N = wl.batch, wl.seqlen, wl.dim, wl.dstate
+    act = 4 if wl.dtype == "f32" else 2
+    n = 2 * b * L * E * act            # x, delta
+    if wl.dev["z"] is not None:
+        n += b * L * E * act
+    n += b * L * E * act               # y
+    n += 2 * b * L * N * act           # B, C
+    n += E * N * 4                     # A_log
+    n += E * 4 if wl.dev["D"] is not None else 0
+    n += E * 4 if wl.dev["delta_bias"] is not None else 0
+    n += b * E * N * 4                 # h_last
+    n += b * E * N * 4 if wl.dev["h0"] is not None else 0
+    return n
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]),
+                "sm_max_mhz": float(d.get("sm_max_mhz", 1965.0)),
+                "source": "measured"}
+    return dict(FALLBACK_PEAKS, source="fallback")
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 100 ms while running."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,"
+             "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" +
+                 self.QUERY, "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.thread is not None:
+                self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- CPU leg
+def oracle_inputs(wl):
+    return dict(x=wl.values("x"), delta=wl.values("delta"),
+                A_log=wl.dev["A_log"], B=wl.values("B"), C=wl.values("C"),
+                D=wl.dev["D"], z=wl.values("z"),
+                delta_bias=wl.dev["delta_bias"], h0=wl.dev["h0"])
+
+
+def cpu_oracle_rate(wl, target_s: float = 10.0, inputs=None, k=None):
+    """Time the float64 oracle on a bounded sample of the workload: the first
+    k channels of every sequence, k sized for about target_s seconds (or
+    given). Returns the cpu_baseline record; its "channels" is k."""
+    import oracle
+    inputs = oracle_inputs(wl) if inputs is None else inputs
+    per_channel = wl.batch * wl.seqlen * wl.dstate
+    if k is None:
+        k0 = min(wl.dim, 4)
+        t0 = time.perf_counter()
+        oracle.scan_channels(np.arange(k0), **inputs, delta_softplus=True)
+        dt = time.perf_counter() - t0
+        rate = k0 * per_channel / max(dt, 1e-9)
+        k = int(min(wl.dim, max(k0, target_s * rate / per_channel)))
+    t0 = time.perf_counter()
+    oracle.scan_channels(np.arange(k), **inputs, delta_softplus=True)
+    dt = time.perf_counter() - t0
+    return {"value": k * per_channel / dt, "unit": UNIT,
+            "cores": oracle.max_threads(), "kind": "oracle", "channels": k,
+            "sample": "%d of %d channels x all %d sequences x L=%d (%.2f s)"
+                      % (k, wl.dim, wl.batch, wl.seqlen, dt)}
+
+
+def run_reference(args):
+    """--impl reference: the float64 CPU oracle on the same workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from selective_state_space_51_b200 import workloads as W
+    wl = W.make(args.shape)
+    per_step = []
+    sample = None
+    # the whole run stays within about --reference-budget seconds
+    target = max(0.05, args.reference_budget / (args.warmup + args.steps))
+    inputs = oracle_inputs(wl)
+    k = None
+    for i in range(args.warmup + args.steps):
+        r = cpu_oracle_rate(wl, target_s=target, inputs=inputs, k=k)
+        k = r["channels"]
+        if i >= args.warmup:
+            per_step.append(r["value"])
+            sample = r
+    value = statistics.median(per_step)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * wl.elements / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": W.shape_description(args.shape),
+                   "global_batch": wl.batch, "seq_len": wl.seqlen,
+                   "parallelism": "cpu oracle, rank 0 only"},
+        "cpu_baseline": dict(sample, value=value),
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- GPU leg
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    import selective_state_space_51_b200 as S
+    from selective_state_space_51_b200 import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE %d" % (args.gpus, world))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    plan = shard_for_rank(rank, world, args.shape)
+    wl = W.make(plan["shape"], seed=plan["seed"])
+    t = {}
+    for k, v in wl.dev.items():
+        if v is None:
+            t[k] = None
+        elif v.dtype == np.uint16:
+            t[k] = torch.from_numpy(v.view(np.int16)).to(dev).view(
+                torch.bfloat16)
+        else:
+            t[k] = torch.from_numpy(np.ascontiguousarray(v)).to(dev)
+    scan = S.SelectiveScan(local)
+    y = torch.empty_like(t["x"])
+    h_last = torch.empty((wl.batch, wl.dim, wl.dstate), dtype=torch.float32,
+                         device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        scan(t["x"], t["delta"], t["A_log"], t["B"], t["C"], D=t["D"],
+             z=t["z"], delta_bias=t["delta_bias"], h0=t["h0"], y=y,
+             h_last=h_last, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if scan.sync_status(stream) != S.SSM_OK:
+        raise SystemExit("device status error during warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    with ClockSampler(local) as clocks:
+        time.sleep(0.3)
+        barrier()
+        torch.cuda.synchronize(dev)
+        t_begin = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_begin.record(stream)
+        for i in range(args.steps):
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        time.sleep(0.2)
+    status = scan.sync_status(stream)
+    if status != S.SSM_OK:
+        raise SystemExit("device status %d in the timed region" % status)
+    local_ms = t_begin.elapsed_time(t_end)
+    kernel_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends))
+    total_ms = max_over_ranks(local_ms, dist if world > 1 else None, dev)
+    kernel_ms = max_over_ranks(kernel_ms, dist if world > 1 else None, dev)
+    variant = scan.last_variant()
+
+    # ---- end to end through the public API with pinned host buffers
+    host = {k: (None if v is None else v.cpu().pin_memory())
+            for k, v in t.items()}
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    h_host = torch.empty(h_last.shape, dtype=h_last.dtype).pin_memory()
+    dev_in = {k: (None if v is None else torch.empty_like(v))
+              for k, v in t.items()}
+    per_step_in = ("x", "delta", "z", "B", "C", "h0")
+    h2d = sum(host[k].numel() * host[k].element_size()
+              for k in per_step_in if host[k] is not None)
+    d2h = y_host.numel() * y_host.element_size() + \
+        h_host.numel() * h_host.element_size()
+    for k, v in host.items():
+        if v is not None:
+            dev_in[k].copy_(v)
+
+    def e2e_step():
+        for k in per_step_in:
+            if host[k] is not None:
+                dev_in[k].copy_(host[k], non_blocking=True)
+        scan(dev_in["x"], dev_in["delta"], dev_in["A_log"], dev_in["B"],
+             dev_in["C"], D=dev_in["D"], z=dev_in["z"],
+             delta_bias=dev_in["delta_bias"], h0=dev_in["h0"], y=y,
+             h_last=h_last, stream=stream)
+        y_host.copy_(y, non_blocking=True)
+        h_host.copy_(h_last, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, args.e2e_steps))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps,
+                            dist if world > 1 else None, dev)
+
+    # ---- figures
+    peaks = load_peaks()
+    clk = clocks.summary()
+    nbytes = algorithmic_bytes(wl)
+    exps = wl.elements
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    ms = total_ms / args.steps
+    value = world * exps / (ms * 1e-3)
+    gbps = nbytes / (kernel_ms * 1e-3) / 1e9
+    sfu_peak_max = sms * SFU_EX2_PER_CLK_PER_SM * peaks["sm_max_mhz"] * 1e6
+    sfu_peak_run = (sms * SFU_EX2_PER_CLK_PER_SM * clk["sm_mhz"] * 1e6
+                    if clk["sm_mhz"] else None)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_sfu = exps / sfu_peak_max
+    t_roof = max(t_hbm, t_sfu)
+    achieved_exp = exps / (kernel_ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "io_dtype": wl.dtype, "data": "synthetic",
+        "config": {"workload": W.shape_description(args.shape),
+                   "global_batch": world * wl.batch, "seq_len": wl.seqlen,
+                   "dim": wl.dim, "dstate": wl.dstate,
+                   "parallelism": "dp%d" % world,
+                   "l2": "inputs larger than L2 (%.0f MB read per step)"
+                         % (nbytes / 1e6)},
+        "gb_per_s": gbps,
+        "roofline_min_hbm_sfu": {
+            "t_hbm_us": t_hbm * 1e6, "t_sfu_us_at_max_clock": t_sfu * 1e6,
+            "t_kernel_us": kernel_ms * 1e3,
+            "frac": t_roof / (kernel_ms * 1e-3),
+            "hbm_peak_gbs": peaks["hbm_gbs"], "hbm_source": peaks["source"],
+            "frac_at_8tbs_hbm": max(nbytes / (HBM_NOMINAL_GBS * 1e9), t_sfu)
+            / (kernel_ms * 1e-3)},
+        "roofline": {"bound": "alu", "unit": "Gexp/s",
+                     "achieved": achieved_exp / 1e9,
+                     "peak": sfu_peak_max / 1e9,
+                     "frac": achieved_exp / sfu_peak_max,
+                     "peak_note": "SFU ex2: %d SMs x %d/clk x %.0f MHz (max "
+                                  "SM clock, %s)" % (
+                                      sms, SFU_EX2_PER_CLK_PER_SM,
+                                      peaks["sm_max_mhz"], peaks["source"]),
+                     "frac_at_sampled_clock": (achieved_exp / sfu_peak_run
+                                               if sfu_peak_run else None),
+                     "traffic": None},
+        "e2e": {"value": world * exps / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps,
+        "kernel": {"variant": variant[0], "segments": variant[1]},
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_rate(wl, args.reference_seconds)
+    scan.close()
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--shape", type=int, default=3,
+                    help="workload shape index (default 3: Mamba-2.8B layer)")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--reference-seconds", type=float, default=10.0,
+                    help="CPU seconds of the oracle sample in cpu_baseline")
+    ap.add_argument("--reference-budget", type=float, default=120.0,
+                    help="total CPU seconds of an --impl reference run")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,172 @@
+/*
+ * ssm_scan.h: C ABI of the B200 (sm_100a) selective-scan forward library
+ * (libssmscan.so).
+ *
+ * The operation is the selective state-space recurrence (Mamba-1 / S6) as
+ * the page "Mamba: Linear-Time Sequence Modeling with Selective State Spaces"
+ * (www.abhik.ai/papers/mamba) states it, section "Original paper, equations
+ * and runnable CPU code":
+ *   row "1. Produce coefficients from the locally mixed input":
+ *       delta = softplus(delta_raw + delta_bias),   A = -exp(A_log)
+ *   row "2. Retain, write and read each channel's state":
+ *       a[t,e,n] = exp(delta[t,e] * A[e,n])
+ *       h[t,e,n] = a[t,e,n] * h[t-1,e,n] + delta[t,e] * B[t,n] * x[t,e]
+ *       y[t,e]   = sum_n C[t,n] * h[t,e,n] + D[e] * x[t,e]
+ *     (read after the update; an optional incoming state continues an
+ *     earlier prefix; the write is delta*B*x, not the exact zero-order-hold
+ *     integral)
+ *   row "5. Put the selective operator inside the complete mixer":
+ *       y <- y * SiLU(z)      (after D*x is included)
+ * per batch b, expanded channel e, state coordinate n. B and C are shared by
+ * every channel ("In the pinned mamba_simple block, B and C have shape
+ * [b, T, N] and are shared across the expanded channels", section "The input
+ * changes the coefficients, while A stays learned"). The final state h_L is
+ * returned; the states of the other steps are never written to memory (the
+ * fused, on-chip evaluation the same page describes in "Compose the updates
+ * instead of waiting for every state").
+ *
+ * Conventions for every call:
+ *   - Pointers named x, delta, z, B, C, y point to DEVICE memory of the
+ *     activation dtype (SSM_F32: float, SSM_BF16: bfloat16). A_log, D,
+ *     delta_bias, h0, h_last point to DEVICE memory of float32.
+ *   - All tensors are dense, row-major (C order), with these shapes:
+ *         x, delta, z, y : [batch, seqlen, dim]       dim = E, contiguous
+ *         B, C           : [batch, seqlen, dstate]    dstate = N
+ *         A_log          : [dim, dstate]
+ *         D, delta_bias  : [dim]
+ *         h0, h_last     : [batch, dim, dstate]       (float32)
+ *   - Ownership: the caller owns every buffer. The library keeps no pointer
+ *     after a call returns. Work is ASYNCHRONOUS on `stream` (a cudaStream_t;
+ *     NULL means the legacy default stream): buffers must stay valid and
+ *     unmodified until the stream has passed the call.
+ *   - Errors: every call returns an int status (SSM_OK or a negative code)
+ *     and never aborts or throws. Argument errors are found on the host
+ *     before anything is launched. A failed launch returns SSM_ERR_CUDA.
+ *   - Thread safety: a handle may be used by one host thread at a time, and
+ *     carries at most one in-flight call on any stream at a time when it
+ *     needs workspace (long sequences with few channels). Different
+ *     handles are independent.
+ */
+#ifndef SSM_SCAN_H
+#define SSM_SCAN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SSM_API __attribute__((visibility("default")))
+#else
+#define SSM_API
+#endif
+
+struct CUstream_st; /* cudaStream_t is `struct CUstream_st *` */
+
+typedef struct ssm_scan_s *ssm_scan_t;
+
+typedef struct {
+    int64_t batch;  /* b  > 0 */
+    int64_t seqlen; /* L  > 0 */
+    int64_t dim;    /* E  > 0, expanded channels */
+    int64_t dstate; /* N  in 1..64 */
+} ssm_scan_dims;
+
+/* Activation dtype (x, delta, z, B, C and y). */
+enum { SSM_F32 = 0, SSM_BF16 = 1 };
+
+/* flags: delta = softplus(delta + delta_bias) when set, else delta + bias. */
+enum { SSM_DELTA_SOFTPLUS = 1u << 0 };
+
+/* Status codes. */
+enum {
+    SSM_OK = 0,
+    SSM_ERR_INVALID = -1,     /* NULL required pointer, bad size or flag  */
+    SSM_ERR_UNSUPPORTED = -2, /* dtype or dstate outside what is built   */
+    SSM_ERR_ALIGN = -3,       /* pointer misaligned for its element type */
+    SSM_ERR_ARCH = -4,        /* device is not compute capability 10.0   */
+    SSM_ERR_CUDA = -5,        /* a CUDA runtime call failed              */
+    SSM_ERR_TIMEOUT = -6,     /* a bounded inter-block wait gave up      */
+    SSM_ERR_NOMEM = -7        /* workspace or handle allocation failed   */
+};
+
+/* Kernel variant selection (ssm_scan_set_variant). AUTO picks by shape. */
+enum {
+    SSM_VARIANT_AUTO = 0,
+    SSM_VARIANT_SEQUENTIAL = 1, /* one thread per (b, e), any shape        */
+    SSM_VARIANT_CHUNKED = 2     /* staged tiles, warp-level scan, fused    */
+};
+
+/*
+ * ssm_scan_create: make a handle bound to CUDA device `device`.
+ * Checks that the device has compute capability 10.0 (B200, sm_100a) and
+ * caches its multiprocessor count. Allocates no device memory.
+ * Returns SSM_OK and writes *out; SSM_ERR_INVALID if out is NULL or device is
+ * out of range; SSM_ERR_ARCH on another architecture; SSM_ERR_CUDA if the
+ * runtime cannot be queried; SSM_ERR_NOMEM if the host allocation fails.
+ */
+SSM_API int ssm_scan_create(ssm_scan_t *out, int device);
+
+/*
+ * ssm_scan_destroy: release the handle and any workspace it grew. Waits for
+ * nothing: the caller must ensure no call using the handle is still in
+ * flight. NULL is accepted and ignored (SSM_OK).
+ */
+SSM_API int ssm_scan_destroy(ssm_scan_t h);
+
+/*
+ * ssm_scan_fwd: the fused selective-scan forward pass (see the file header
+ * for the recurrence and layouts).
+ *   x, delta, B, C, A_log, y : required (non-NULL).
+ *   D          : NULL means no direct path (D = 0).
+ *   z          : NULL means no gate.
+ *   delta_bias : NULL means a zero bias.
+ *   h0         : NULL means a zero incoming state.
+ *   h_last     : NULL means the final state is not written.
+ *   flags      : SSM_DELTA_SOFTPLUS or 0; other bits are SSM_ERR_INVALID.
+ *   dtype      : SSM_F32 or SSM_BF16 (activations and y).
+ * y must not overlap any input. Pointers must be aligned to their element
+ * size (SSM_ERR_ALIGN otherwise). Launches on `stream` and returns without
+ * waiting. The handle's device must be current on the calling thread.
+ */
+SSM_API int ssm_scan_fwd(ssm_scan_t h, const void *x, const void *delta,
+                 const float *A_log, const void *B, const void *C,
+                 const float *D, const void *z, const float *delta_bias,
+                 uint32_t flags, const float *h0, void *y, float *h_last,
+                 ssm_scan_dims dims, int dtype, struct CUstream_st *stream);
+
+/*
+ * ssm_scan_set_variant: force a kernel variant for later calls on this
+ * handle (SSM_VARIANT_*), or SSM_VARIANT_AUTO to choose by shape.
+ * `segments` > 1 asks the chunked variant to split every sequence into that
+ * many independent pieces joined by the inter-block carry (0 = automatic,
+ * 1 = never split). A forced variant that cannot run a given shape makes
+ * ssm_scan_fwd return SSM_ERR_UNSUPPORTED. Returns SSM_ERR_INVALID for an
+ * unknown variant or a negative segment count.
+ */
+SSM_API int ssm_scan_set_variant(ssm_scan_t h, int variant, int segments);
+
+/*
+ * ssm_scan_last_variant: the variant (SSM_VARIANT_*) and segment count the
+ * most recent successful ssm_scan_fwd on this handle launched. Either output
+ * pointer may be NULL.
+ */
+SSM_API int ssm_scan_last_variant(ssm_scan_t h, int *variant, int *segments);
+
+/*
+ * ssm_scan_sync_status: wait for `stream`, then report device-side status of
+ * the calls made on this handle since the previous sync: SSM_ERR_TIMEOUT if a
+ * bounded wait between thread blocks gave up (its results are then invalid),
+ * SSM_ERR_CUDA on an asynchronous CUDA error, else SSM_OK. Resets the status.
+ */
+SSM_API int ssm_scan_sync_status(ssm_scan_t h, struct CUstream_st *stream);
+
+/* ssm_scan_status_string: static English text for a status code. */
+SSM_API const char *ssm_scan_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSM_SCAN_H */

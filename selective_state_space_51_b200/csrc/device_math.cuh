@@ -1,0 +1,84 @@
+// Device-side arithmetic shared by the scan kernels: hardware exp2/log2/rcp
+// through the SFU (MUFU) pipe, the step-size softplus, the SiLU gate and
+// activation loads/stores for float32 and bfloat16.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace ssm {
+
+constexpr float kLog2e = 1.4426950408889634f;  // 1 / ln 2
+constexpr float kLn2 = 0.6931471805599453f;
+
+// 2^x on the SFU (one MUFU.EX2). Flushes subnormal results to zero, so a
+// retention exp(delta*A) below 2^-126 becomes exactly 0.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// log2(x) on the SFU (one MUFU.LG2).
+__device__ __forceinline__ float lg2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 1/x on the SFU (one MUFU.RCP); 1/inf = 0.
+__device__ __forceinline__ float rcp(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// log(1 + u) for u in [0, 1]. Below 1/8 the alternating Taylor series
+// u - u^2/2 + u^3/3 - ... truncated after the u^8 term (relative truncation
+// error < u^8 / 9 < 2^-27); from 1/8 up, log2(1 + u) * ln 2, where rounding
+// 1 + u costs at most 2^-24 absolute, i.e. < 5e-7 relative to log(1.125).
+__device__ __forceinline__ float log1p_unit(float u) {
+  float s = fmaf(u, -0.125f, 0.14285714285714285f);
+  s = fmaf(u, s, -0.16666666666666666f);
+  s = fmaf(u, s, 0.2f);
+  s = fmaf(u, s, -0.25f);
+  s = fmaf(u, s, 0.3333333333333333f);
+  s = fmaf(u, s, -0.5f);
+  s = fmaf(u, s, 1.0f);
+  s *= u;
+  const float l = lg2(1.0f + u) * kLn2;
+  return u < 0.125f ? s : l;
+}
+
+// softplus with PyTorch's default threshold: v for v > 20, else
+// log(1 + e^v) = max(v, 0) + log(1 + e^-|v|), which never overflows and keeps
+// relative accuracy for very negative v (where the result is ~e^v).
+__device__ __forceinline__ float softplus(float v) {
+  const float u = ex2(-fabsf(v) * kLog2e);  // e^-|v| in (0, 1]
+  const float r = fmaxf(v, 0.0f) + log1p_unit(u);
+  return v > 20.0f ? v : r;
+}
+
+// SiLU(z) = z * sigmoid(z) = z / (1 + e^-z). For z -> -inf, e^-z = inf and
+// rcp(inf) = 0 gives -0; for z -> +inf it gives z.
+__device__ __forceinline__ float silu(float z) {
+  return z * rcp(1.0f + ex2(-z * kLog2e));
+}
+
+template <typename T> struct Act;
+
+template <> struct Act<float> {
+  static __device__ __forceinline__ float load(const float *p) { return *p; }
+  static __device__ __forceinline__ void store(float *p, float v) { *p = v; }
+};
+
+template <> struct Act<__nv_bfloat16> {
+  static __device__ __forceinline__ float load(const __nv_bfloat16 *p) {
+    return __bfloat162float(*p);
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16 *p, float v) {
+    *p = __float2bfloat16_rn(v);
+  }
+};
+
+}  // namespace ssm

@@ -1,0 +1,75 @@
+// Sequential variant: one thread per (batch, channel) walks the whole
+// sequence, keeping that channel's N states in float32 registers. It runs any
+// shape (any E, any L, N up to 64) and serves as the general path for shapes
+// the chunked variant does not tile.
+//
+// Recurrence (page "Mamba: Linear-Time Sequence Modeling with Selective State
+// Spaces", www.abhik.ai/papers/mamba, section "Original paper, equations and
+// runnable CPU code", rows 1, 2 and 5): delta = softplus(raw + bias);
+// a = exp(delta * A) with A = -exp(A_log); h = a * h + delta * B * x;
+// y = sum_n C * h + D * x, read after the update; y *= SiLU(z).
+#pragma once
+
+#include "device_math.cuh"
+#include "scan_params.cuh"
+
+namespace ssm {
+
+template <typename T, int NMAX>
+__global__ void __launch_bounds__(128)
+scan_sequential_kernel(const ScanParams p) {
+  const int64_t pair = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (pair >= p.batch * p.dim) return;
+  const int64_t b = pair / p.dim;
+  const int64_t e = pair - b * p.dim;
+  const int N = p.dstate;
+  const int64_t L = p.seqlen, E = p.dim;
+
+  float A2[NMAX];  // A * log2(e), so that a = 2^(delta * A2)
+  float h[NMAX];
+#pragma unroll
+  for (int n = 0; n < NMAX; ++n) {
+    A2[n] = 0.0f;
+    h[n] = 0.0f;
+    if (n < N) {
+      A2[n] = -expf(p.A_log[e * N + n]) * kLog2e;
+      if (p.h0) h[n] = p.h0[(b * E + e) * N + n];
+    }
+  }
+  const float bias = p.delta_bias ? p.delta_bias[e] : 0.0f;
+  const float Dv = p.D ? p.D[e] : 0.0f;
+  const T *x = static_cast<const T *>(p.x);
+  const T *dl = static_cast<const T *>(p.delta);
+  const T *z = static_cast<const T *>(p.z);
+  const T *Bm = static_cast<const T *>(p.B);
+  const T *Cm = static_cast<const T *>(p.C);
+  T *y = static_cast<T *>(p.y);
+
+  for (int64_t t = 0; t < L; ++t) {
+    const int64_t i = (b * L + t) * E + e;
+    const int64_t r = (b * L + t) * N;
+    const float v = Act<T>::load(dl + i) + bias;
+    const float step = p.softplus ? softplus(v) : v;
+    const float xv = Act<T>::load(x + i);
+    const float dx = step * xv;
+    float acc = 0.0f;
+#pragma unroll
+    for (int n = 0; n < NMAX; ++n) {
+      if (n < N) {
+        const float a = ex2(step * A2[n]);
+        h[n] = fmaf(a, h[n], dx * Act<T>::load(Bm + r + n));
+        acc = fmaf(Act<T>::load(Cm + r + n), h[n], acc);
+      }
+    }
+    acc = fmaf(Dv, xv, acc);
+    if (z) acc *= silu(Act<T>::load(z + i));
+    Act<T>::store(y + i, acc);
+  }
+  if (p.h_last) {
+#pragma unroll
+    for (int n = 0; n < NMAX; ++n)
+      if (n < N) p.h_last[(b * E + e) * N + n] = h[n];
+  }
+}
+
+}  // namespace ssm

@@ -1,0 +1,208 @@
+// C ABI of libssmscan.so: handle management, host-side validation, variant
+// choice and launches. Declarations and the contract live in
+// include/ssm_scan.h.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <new>
+
+#include "../../include/ssm_scan.h"
+#include "kernel_sequential.cuh"
+
+struct ssm_scan_s {
+  int device = 0;
+  int sm_count = 0;
+  int variant = SSM_VARIANT_AUTO;
+  int segments = 0;
+  int last_variant = 0;
+  int last_segments = 0;
+  unsigned epoch = 0;
+  // device workspace: [status word, ticket][segment carry arrays]
+  void *ws = nullptr;
+  size_t ws_bytes = 0;
+};
+
+namespace {
+
+bool aligned(const void *p, size_t a) {
+  return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+bool mul_ok(int64_t a, int64_t b, int64_t *out) {
+  return !__builtin_mul_overflow(a, b, out);
+}
+
+template <typename T, int NMAX>
+int launch_sequential(const ssm::ScanParams &p, cudaStream_t s) {
+  const int64_t pairs = p.batch * p.dim;
+  const int threads = 128;
+  const int64_t blocks = (pairs + threads - 1) / threads;
+  if (blocks > 0x7fffffff) return SSM_ERR_UNSUPPORTED;
+  ssm::scan_sequential_kernel<T, NMAX><<<(unsigned)blocks, threads, 0, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+template <typename T>
+int dispatch_sequential(const ssm::ScanParams &p, cudaStream_t s) {
+  if (p.dstate <= 4) return launch_sequential<T, 4>(p, s);
+  if (p.dstate <= 8) return launch_sequential<T, 8>(p, s);
+  if (p.dstate <= 16) return launch_sequential<T, 16>(p, s);
+  if (p.dstate <= 32) return launch_sequential<T, 32>(p, s);
+  return launch_sequential<T, 64>(p, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+int ssm_scan_create(ssm_scan_t *out, int device) {
+  if (!out) return SSM_ERR_INVALID;
+  *out = nullptr;
+  int count = 0;
+  if (cudaGetDeviceCount(&count) != cudaSuccess) {
+    cudaGetLastError();
+    return SSM_ERR_CUDA;
+  }
+  if (device < 0 || device >= count) return SSM_ERR_INVALID;
+  int major = 0, minor = 0, sms = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor,
+                             device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor,
+                             device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) !=
+          cudaSuccess) {
+    cudaGetLastError();
+    return SSM_ERR_CUDA;
+  }
+  if (major != 10 || minor != 0) return SSM_ERR_ARCH;
+  ssm_scan_s *h = new (std::nothrow) ssm_scan_s();
+  if (!h) return SSM_ERR_NOMEM;
+  h->device = device;
+  h->sm_count = sms;
+  *out = h;
+  return SSM_OK;
+}
+
+int ssm_scan_destroy(ssm_scan_t h) {
+  if (!h) return SSM_OK;
+  int rc = SSM_OK;
+  if (h->ws) {
+    int prev = 0;
+    cudaGetDevice(&prev);
+    cudaSetDevice(h->device);
+    if (cudaFree(h->ws) != cudaSuccess) rc = SSM_ERR_CUDA;
+    cudaSetDevice(prev);
+  }
+  delete h;
+  return rc;
+}
+
+int ssm_scan_set_variant(ssm_scan_t h, int variant, int segments) {
+  if (!h) return SSM_ERR_INVALID;
+  if (variant < SSM_VARIANT_AUTO || variant > SSM_VARIANT_CHUNKED)
+    return SSM_ERR_INVALID;
+  if (segments < 0) return SSM_ERR_INVALID;
+  h->variant = variant;
+  h->segments = segments;
+  return SSM_OK;
+}
+
+int ssm_scan_last_variant(ssm_scan_t h, int *variant, int *segments) {
+  if (!h) return SSM_ERR_INVALID;
+  if (variant) *variant = h->last_variant;
+  if (segments) *segments = h->last_segments;
+  return SSM_OK;
+}
+
+int ssm_scan_sync_status(ssm_scan_t h, struct CUstream_st *stream) {
+  if (!h) return SSM_ERR_INVALID;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return SSM_ERR_CUDA;
+  }
+  if (!h->ws) return SSM_OK;
+  int status = 0;
+  if (cudaMemcpy(&status, h->ws, sizeof(int), cudaMemcpyDeviceToHost) !=
+      cudaSuccess)
+    return SSM_ERR_CUDA;
+  if (status != ssm::kStatusOk) {
+    const int zero = 0;
+    if (cudaMemcpy(h->ws, &zero, sizeof(int), cudaMemcpyHostToDevice) !=
+        cudaSuccess)
+      return SSM_ERR_CUDA;
+    return SSM_ERR_TIMEOUT;
+  }
+  return SSM_OK;
+}
+
+const char *ssm_scan_status_string(int status) {
+  switch (status) {
+    case SSM_OK: return "ok";
+    case SSM_ERR_INVALID: return "invalid argument";
+    case SSM_ERR_UNSUPPORTED: return "unsupported dtype, state size or shape";
+    case SSM_ERR_ALIGN: return "misaligned pointer";
+    case SSM_ERR_ARCH: return "device is not compute capability 10.0 (sm_100a)";
+    case SSM_ERR_CUDA: return "CUDA runtime error";
+    case SSM_ERR_TIMEOUT: return "bounded wait between thread blocks timed out";
+    case SSM_ERR_NOMEM: return "allocation failed";
+    default: return "unknown status";
+  }
+}
+
+int ssm_scan_fwd(ssm_scan_t h, const void *x, const void *delta,
+                 const float *A_log, const void *B, const void *C,
+                 const float *D, const void *z, const float *delta_bias,
+                 uint32_t flags, const float *h0, void *y, float *h_last,
+                 ssm_scan_dims dims, int dtype, struct CUstream_st *stream) {
+  // ---- host-side validation: nothing touches the GPU before it passes
+  if (!h || !x || !delta || !A_log || !B || !C || !y) return SSM_ERR_INVALID;
+  if (dims.batch <= 0 || dims.seqlen <= 0 || dims.dim <= 0 || dims.dstate <= 0)
+    return SSM_ERR_INVALID;
+  if (flags & ~uint32_t(SSM_DELTA_SOFTPLUS)) return SSM_ERR_INVALID;
+  if (dtype != SSM_F32 && dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
+  if (dims.dstate > 64) return SSM_ERR_UNSUPPORTED;
+  int64_t rows = 0, acts = 0, bc = 0, st = 0;
+  if (!mul_ok(dims.batch, dims.seqlen, &rows) ||
+      !mul_ok(rows, dims.dim, &acts) || !mul_ok(rows, dims.dstate, &bc) ||
+      !mul_ok(dims.batch * dims.dim, dims.dstate, &st) ||
+      acts > (int64_t(1) << 56))
+    return SSM_ERR_INVALID;
+  const size_t esz = dtype == SSM_F32 ? 4 : 2;
+  const void *acts_in[] = {x, delta, B, C, z, y};
+  for (const void *p : acts_in)
+    if (p && !aligned(p, esz)) return SSM_ERR_ALIGN;
+  const float *params[] = {A_log, D, delta_bias, h0, h_last};
+  for (const float *p : params)
+    if (p && !aligned(p, 4)) return SSM_ERR_ALIGN;
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) {
+    cudaGetLastError();
+    return SSM_ERR_CUDA;
+  }
+  if (cur != h->device) return SSM_ERR_INVALID;
+
+  ssm::ScanParams p{};
+  p.x = x; p.delta = delta; p.A_log = A_log; p.B = B; p.C = C;
+  p.D = D; p.z = z; p.delta_bias = delta_bias; p.h0 = h0;
+  p.y = y; p.h_last = h_last;
+  p.batch = dims.batch; p.seqlen = dims.seqlen; p.dim = dims.dim;
+  p.dstate = (int)dims.dstate;
+  p.softplus = (flags & SSM_DELTA_SOFTPLUS) ? 1 : 0;
+  p.segments = 1;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  if (h->variant == SSM_VARIANT_CHUNKED) return SSM_ERR_UNSUPPORTED;
+  int rc;
+  if (dtype == SSM_F32)
+    rc = dispatch_sequential<float>(p, s);
+  else
+    rc = dispatch_sequential<__nv_bfloat16>(p, s);
+  if (rc == SSM_OK) {
+    h->last_variant = SSM_VARIANT_SEQUENTIAL;
+    h->last_segments = 1;
+  }
+  return rc;
+}
+
+}  // extern "C"
