@@ -148,6 +148,16 @@ SSM_API int ssm_scan_fwd(ssm_scan_t h, const void *x, const void *delta,
 SSM_API int ssm_scan_set_variant(ssm_scan_t h, int variant, int segments);
 
 /*
+ * ssm_scan_set_time_blocks: for the chunked variant, how many lanes of a warp
+ * share one channel's time axis (1, 2, 4 or 8: each takes a block of
+ * consecutive steps, and the blocks are joined by a warp-shuffle scan of
+ * their affine maps), or 0 to choose by shape. Returns SSM_ERR_INVALID for
+ * other values. A value a shape cannot use is reported by ssm_scan_fwd as
+ * SSM_ERR_UNSUPPORTED.
+ */
+SSM_API int ssm_scan_set_time_blocks(ssm_scan_t h, int time_blocks);
+
+/*
  * ssm_scan_last_variant: the variant (SSM_VARIANT_*) and segment count the
  * most recent successful ssm_scan_fwd on this handle launched. Either output
  * pointer may be NULL.

@@ -7,6 +7,7 @@
 #include <new>
 
 #include "../../include/ssm_scan.h"
+#include "kernel_chunked.cuh"
 #include "kernel_sequential.cuh"
 
 struct ssm_scan_s {
@@ -14,6 +15,7 @@ struct ssm_scan_s {
   int sm_count = 0;
   int variant = SSM_VARIANT_AUTO;
   int segments = 0;
+  int time_blocks = 0;
   int last_variant = 0;
   int last_segments = 0;
   unsigned epoch = 0;
@@ -49,6 +51,77 @@ int dispatch_sequential(const ssm::ScanParams &p, cudaStream_t s) {
   if (p.dstate <= 16) return launch_sequential<T, 16>(p, s);
   if (p.dstate <= 32) return launch_sequential<T, 32>(p, s);
   return launch_sequential<T, 64>(p, s);
+}
+
+// Chunked-variant shapes. Paddings (bytes: per tile row, per block of rows,
+// per block of float B/C rows) make each lane access pattern bank-conflict
+// free for that lane layout.
+using bf16 = __nv_bfloat16;
+//                          T      NG TB  K  TW NW pad  PB  BFPB
+using C16b1 = ssm::ChunkCfg<bf16,  4, 1, 4, 64, 4, 16,  0,  0>;
+using C16f1 = ssm::ChunkCfg<float, 4, 1, 4, 64, 4, 32,  0,  0>;
+using C16b2 = ssm::ChunkCfg<bf16,  4, 2, 8, 64, 4,  0, 16, 64>;
+using C16f2 = ssm::ChunkCfg<float, 4, 2, 8, 64, 4, 32, 16, 64>;
+using C8b1 = ssm::ChunkCfg<bf16,   2, 1, 2, 64, 4, 32,  0,  0>;
+using C8f1 = ssm::ChunkCfg<float,  2, 1, 2, 64, 4, 64,  0,  0>;
+using C8b2 = ssm::ChunkCfg<bf16,   2, 2, 8, 64, 4,  0, 16, 32>;
+using C8f2 = ssm::ChunkCfg<float,  2, 2, 8, 64, 4, 32, 64, 32>;
+using C4f1 = ssm::ChunkCfg<float,  1, 1, 1, 64, 4,  0,  0,  0>;
+using C4f2 = ssm::ChunkCfg<float,  1, 2, 8, 64, 4,  0, 64, 16>;
+
+template <class Cfg>
+int launch_chunked(const ssm::ScanParams &p, cudaStream_t s) {
+  const int64_t tiles = (p.dim + Cfg::G - 1) / Cfg::G;
+  const int64_t blocks = p.batch * tiles;
+  if (blocks > 0x7fffffff) return SSM_ERR_UNSUPPORTED;
+  auto kern = ssm::scan_chunked_kernel<Cfg>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           Cfg::SMEM_BYTES) != cudaSuccess) {
+    cudaGetLastError();
+    return SSM_ERR_CUDA;
+  }
+  kern<<<(unsigned)blocks, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+// Whether the chunked variant can run these arguments: N of 4, 8 or 16, whole
+// 16-byte chunks per channel tile row and per B/C row, 16-byte aligned tiles.
+bool chunked_supported(const ssm::ScanParams &p, int dtype) {
+  const int esz = dtype == SSM_F32 ? 4 : 2;
+  if (p.dstate != 4 && p.dstate != 8 && p.dstate != 16) return false;
+  if (p.dstate * esz < 16) return false;
+  if ((p.dim * esz) % 16 != 0) return false;
+  const void *tiles[] = {p.x, p.delta, p.z, p.B, p.C};
+  for (const void *t : tiles)
+    if (t && !aligned(t, 16)) return false;
+  return true;
+}
+
+// Time blocks per channel: 1 while the channels alone give every SM
+// sub-partition several warps, else 2.
+int auto_time_blocks(const ssm::ScanParams &p, int sm_count) {
+  const int64_t warps1 = p.batch * p.dim * (p.dstate / 4) / 32;
+  return warps1 >= 4LL * 4 * sm_count ? 1 : 2;
+}
+
+template <typename T, class Cf1, class Cf2>
+int pick(const ssm::ScanParams &p, int tb, cudaStream_t s) {
+  if (tb == 1) return launch_chunked<Cf1>(p, s);
+  if (tb == 2) return launch_chunked<Cf2>(p, s);
+  return SSM_ERR_UNSUPPORTED;
+}
+
+int dispatch_chunked(const ssm::ScanParams &p, int dtype, int tb,
+                     cudaStream_t s) {
+  if (dtype == SSM_BF16) {
+    if (p.dstate == 16) return pick<bf16, C16b1, C16b2>(p, tb, s);
+    if (p.dstate == 8) return pick<bf16, C8b1, C8b2>(p, tb, s);
+    return SSM_ERR_UNSUPPORTED;
+  }
+  if (p.dstate == 16) return pick<float, C16f1, C16f2>(p, tb, s);
+  if (p.dstate == 8) return pick<float, C8f1, C8f2>(p, tb, s);
+  if (p.dstate == 4) return pick<float, C4f1, C4f2>(p, tb, s);
+  return SSM_ERR_UNSUPPORTED;
 }
 
 }  // namespace
@@ -104,6 +177,15 @@ int ssm_scan_set_variant(ssm_scan_t h, int variant, int segments) {
   if (segments < 0) return SSM_ERR_INVALID;
   h->variant = variant;
   h->segments = segments;
+  return SSM_OK;
+}
+
+int ssm_scan_set_time_blocks(ssm_scan_t h, int time_blocks) {
+  if (!h) return SSM_ERR_INVALID;
+  if (time_blocks != 0 && time_blocks != 1 && time_blocks != 2 &&
+      time_blocks != 4 && time_blocks != 8)
+    return SSM_ERR_INVALID;
+  h->time_blocks = time_blocks;
   return SSM_OK;
 }
 
@@ -192,14 +274,23 @@ int ssm_scan_fwd(ssm_scan_t h, const void *x, const void *delta,
   p.segments = 1;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
-  if (h->variant == SSM_VARIANT_CHUNKED) return SSM_ERR_UNSUPPORTED;
+  int variant = h->variant;
+  const bool chunk_ok = chunked_supported(p, dtype);
+  if (variant == SSM_VARIANT_AUTO)
+    variant = chunk_ok ? SSM_VARIANT_CHUNKED : SSM_VARIANT_SEQUENTIAL;
   int rc;
-  if (dtype == SSM_F32)
+  if (variant == SSM_VARIANT_CHUNKED) {
+    if (!chunk_ok) return SSM_ERR_UNSUPPORTED;
+    const int tb = h->time_blocks ? h->time_blocks
+                                  : auto_time_blocks(p, h->sm_count);
+    rc = dispatch_chunked(p, dtype, tb, s);
+  } else if (dtype == SSM_F32) {
     rc = dispatch_sequential<float>(p, s);
-  else
+  } else {
     rc = dispatch_sequential<__nv_bfloat16>(p, s);
+  }
   if (rc == SSM_OK) {
-    h->last_variant = SSM_VARIANT_SEQUENTIAL;
+    h->last_variant = variant;
     h->last_segments = 1;
   }
   return rc;

@@ -15,8 +15,10 @@ from gpu_helpers import TOL, assert_close, oracle_inputs, run, to_device
 
 pytestmark = pytest.mark.gpu
 
-VARIANTS = [S.SSM_VARIANT_AUTO, S.SSM_VARIANT_SEQUENTIAL]
-VARIANT_IDS = ["auto", "sequential"]
+# (variant, time blocks per channel for the chunked variant)
+VARIANTS = [(S.SSM_VARIANT_AUTO, 0), (S.SSM_VARIANT_SEQUENTIAL, 0),
+            (S.SSM_VARIANT_CHUNKED, 1), (S.SSM_VARIANT_CHUNKED, 2)]
+VARIANT_IDS = ["auto", "sequential", "chunked_tb1", "chunked_tb2"]
 
 # Small cases with each workload's distributions: several tiles, ragged
 # sequence ends and ragged channel tiles.
@@ -37,7 +39,12 @@ def scan():
 
 
 def _with_variant(scan, variant, segments=0):
+    if isinstance(variant, tuple):
+        variant, tb = variant
+    else:
+        tb = 0
     scan.set_variant(variant, segments)
+    S.library().ssm_scan_set_time_blocks(scan.handle, tb)
 
 
 @pytest.mark.parametrize("variant", VARIANTS, ids=VARIANT_IDS)
@@ -91,6 +98,23 @@ def test_state_sizes(scan, N):
     assert_close(h, ho, wl.dtype, "h_last")
 
 
+@pytest.mark.parametrize("variant", VARIANTS[2:], ids=VARIANT_IDS[2:])
+@pytest.mark.parametrize("N,dtype", [(4, W.F32), (8, W.F32), (8, W.BF16),
+                                     (16, W.F32), (16, W.BF16)])
+def test_chunked_state_sizes(scan, N, dtype, variant):
+    wl = W.make(2, batch=3, seqlen=333, dim=72, dstate=N, dtype=dtype,
+                with_h0=True)
+    _with_variant(scan, variant)
+    try:
+        y, h = run(scan, wl)
+        assert scan.last_variant()[0] == S.SSM_VARIANT_CHUNKED
+    finally:
+        _with_variant(scan, S.SSM_VARIANT_AUTO)
+    yo, ho = oracle.scan(**oracle_inputs(wl))
+    assert_close(y, yo, wl.dtype, "y")
+    assert_close(h, ho, wl.dtype, "h_last")
+
+
 @pytest.mark.parametrize("variant", VARIANTS, ids=VARIANT_IDS)
 @pytest.mark.parametrize("L", [1, 2, 31, 33, 257])
 def test_short_and_ragged_lengths(scan, L, variant):
@@ -118,9 +142,11 @@ def test_optional_inputs(scan, opts, dtype):
         wl.dev["delta_bias"] = None
     softplus = opts.get("softplus", True)
     if not softplus:
-        # keep the steps positive and moderate without softplus
+        # without softplus the step is raw + bias as given: keep it positive
+        # and moderate (the recipe's bias is negative, made for softplus)
         d = np.abs(wl.values("delta")) * np.float32(0.1)
         wl.dev["delta"] = (W.round_to_bf16_bits(d) if dtype == W.BF16 else d)
+        wl.dev["delta_bias"] = np.full(48, 0.01, dtype=np.float32)
     y, h = run(scan, wl, softplus=softplus)
     yo, ho = oracle.scan(**oracle_inputs(wl), delta_softplus=softplus)
     assert_close(y, yo, dtype, "y")
@@ -192,6 +218,25 @@ def test_channel_permutation(scan):
     yp, hp = run(scan, wl, t=tp)
     pn = perm.cpu().numpy()
     assert np.array_equal(yp, y[..., pn]) and np.array_equal(hp, h[:, pn])
+
+
+def test_chunked_unsupported_shapes(scan):
+    """A forced chunked variant reports shapes it cannot tile; AUTO falls
+    back to the sequential variant for them."""
+    wl = W.make(1, batch=1, seqlen=100, dim=42, dstate=16)   # E*4 % 16 != 0
+    t = to_device(wl)
+    _with_variant(scan, (S.SSM_VARIANT_CHUNKED, 1))
+    try:
+        with pytest.raises(S.SsmScanError) as ei:
+            scan(t["x"], t["delta"], t["A_log"], t["B"], t["C"], D=t["D"],
+                 z=t["z"], delta_bias=t["delta_bias"])
+        assert ei.value.status == S.SSM_ERR_UNSUPPORTED
+    finally:
+        _with_variant(scan, S.SSM_VARIANT_AUTO)
+    y, h = run(scan, wl, t=t)
+    assert scan.last_variant()[0] == S.SSM_VARIANT_SEQUENTIAL
+    yo, ho = oracle.scan(**oracle_inputs(wl))
+    assert_close(y, yo, wl.dtype, "y")
 
 
 def test_argument_errors(scan):
