@@ -302,6 +302,9 @@ def run_gpu(args):
     variant = scan.last_variant()
 
     # ---- end to end through the public API with pinned host buffers
+    if args.no_e2e:
+        return _finish(args, wl, world, rank, local, dev, dist, scan, clocks,
+                       total_ms, kernel_ms, variant, None, 0, 0)
     host = {k: (None if v is None else v.cpu().pin_memory())
             for k, v in t.items()}
     y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
@@ -343,8 +346,14 @@ def run_gpu(args):
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps,
                             dist if world > 1 else None, dev)
+    return _finish(args, wl, world, rank, local, dev, dist, scan, clocks,
+                   total_ms, kernel_ms, variant, e2e_ms, h2d, d2h)
 
-    # ---- figures
+
+def _finish(args, wl, world, rank, local, dev, dist, scan, clocks, total_ms,
+            kernel_ms, variant, e2e_ms, h2d, d2h):
+    import torch
+    from selective_state_space_51_b200 import workloads as W
     peaks = load_peaks()
     clk = clocks.summary()
     nbytes = algorithmic_bytes(wl)
@@ -390,9 +399,10 @@ def run_gpu(args):
                      "frac_at_sampled_clock": (achieved_exp / sfu_peak_run
                                                if sfu_peak_run else None),
                      "traffic": None},
-        "e2e": {"value": world * exps / (e2e_ms * 1e-3), "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_ms},
+        "e2e": (None if e2e_ms is None else
+                {"value": world * exps / (e2e_ms * 1e-3), "unit": UNIT,
+                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                 "ms_per_step": e2e_ms}),
         "gpu_launches": args.steps,
         "kernel": {"variant": variant[0], "segments": variant[1]},
         "clocks": clk,
@@ -422,6 +432,8 @@ def main(argv=None):
     ap.add_argument("--reference-budget", type=float, default=120.0,
                     help="total CPU seconds of an --impl reference run")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end (host buffer) measurement")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
