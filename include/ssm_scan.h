@@ -158,6 +158,17 @@ SSM_API int ssm_scan_set_variant(ssm_scan_t h, int variant, int segments);
 SSM_API int ssm_scan_set_time_blocks(ssm_scan_t h, int time_blocks);
 
 /*
+ * ssm_scan_set_debug: testing hook. `flags` bit 0 makes the first piece of
+ * every split sequence skip its publication, so that the bounded wait of its
+ * successor runs out: that call then reports SSM_ERR_TIMEOUT through
+ * ssm_scan_sync_status and its outputs are invalid. `spin_limit` bounds every
+ * wait between thread blocks (in polls of roughly 1 us each; 0 restores the
+ * default of 10^6 polls, about one second). Returns SSM_ERR_INVALID for a NULL handle.
+ */
+SSM_API int ssm_scan_set_debug(ssm_scan_t h, unsigned flags,
+                               unsigned spin_limit);
+
+/*
  * ssm_scan_last_variant: the variant (SSM_VARIANT_*) and segment count the
  * most recent successful ssm_scan_fwd on this handle launched. Either output
  * pointer may be NULL.

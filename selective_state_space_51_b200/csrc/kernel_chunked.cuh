@@ -9,30 +9,43 @@
 // the updates instead of waiting for every state"].
 //
 // Work decomposition. A thread block owns one batch row b, a tile of G
-// consecutive channels and a contiguous range of steps; it walks that range in
+// consecutive channels and a contiguous piece of the sequence, walked in
 // windows of TW steps. Inside a warp a lane is (c, g, q):
 //   c: one of CW channels of the warp,
 //   g: one of NG groups of 4 state coordinates (N = 4 NG),
-//   q: one of TB time blocks: with TB > 1 the TB lanes of a (c, g) pair own
-//      consecutive K-step blocks of a sub-window, fold their steps into one
-//      affine map, combine the maps with a warp-shuffle scan and then replay
-//      their steps from the true incoming state (time parallelism inside the
-//      warp); with TB == 1 a lane walks every step itself.
-// Each lane keeps its 4 states in float32 registers across windows; states of
-// intermediate steps never leave the chip.
+//   q: one of TB time blocks. With TB > 1 the TB lanes of a (c, g) pair own
+//      consecutive K-step blocks of each sub-window: each folds its steps into
+//      one affine map, the maps are combined by a warp-shuffle scan, and each
+//      lane then replays its steps from the true incoming state. With TB == 1
+//      a lane walks every step itself.
+// Each lane keeps its 4 states in float32 registers (two packed pairs, updated
+// with FFMA2/FMUL2); states of intermediate steps never leave the chip.
 //
 // Per window: x, raw delta, z tiles [TW x G] and B, C tiles [TW x N] are
 // staged in shared memory with cp.async (double buffered, one window ahead;
-// rows padded so the lane access patterns are bank-conflict free); bfloat16
-// B and C are widened once per window to float32. For each block of NG steps
-// the NG lanes of a (c, q) pair each compute softplus for one step (so every
-// (t, e) pays its softplus once) and exchange (delta, delta*x) by shuffles.
-// The readout partial sums over each lane's 4 states are combined over the NG
-// lanes by a transposing butterfly that leaves lane g holding the full y of
-// the block's step g, which then adds D x, applies the SiLU gate, and stores.
+// rows padded so every lane access pattern is bank-conflict free); bfloat16
+// B and C are widened to float32 once per window. In each block of NG steps
+// lane g computes softplus for step g only and publishes (delta, delta,
+// delta*x, delta*x) in a per-warp exchange slot, so every (t, e) pays its
+// softplus once and the state arithmetic reads ready-made pairs. Readout
+// partials over each lane's 4 states are combined over the NG lanes by a
+// transposing butterfly that leaves lane g holding the full y of the block's
+// step g; lane g adds D x, applies the SiLU gate and stores.
+//
+// Split sequences (SPLIT). For few channels and long sequences each sequence
+// is cut into pieces scanned concurrently. A piece starts from a zero state,
+// stores its outputs, and publishes its affine aggregate (end state from
+// zero, product of retentions). It then looks back over its predecessors'
+// publications (bounded waits) to learn its true incoming state, publishes
+// its inclusive end state, and replays its first windows with no write term,
+// adding C h * SiLU(z) to the stored outputs, until the carried-in part of the
+// state has decayed to exactly zero (FTZ underflow). Blocks take pieces in
+// launch-ticket order, so a block only ever waits for blocks already running.
 #pragma once
 
 #include <float.h>
+
+#include <type_traits>
 
 #include "device_math.cuh"
 #include "scan_params.cuh"
@@ -53,6 +66,17 @@ __device__ __forceinline__ void cp_async_commit() {
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(unsigned *p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v)
+               : "memory");
 }
 
 constexpr int round16(int x) { return (x + 15) / 16 * 16; }
@@ -77,12 +101,15 @@ struct ChunkCfg {
   static constexpr int RAW_BYTES = round16(TW * RAW_P + (TW / BLK) * RAW_PB);
   static constexpr int BF_ROW = N * 4;
   static constexpr int BF_PB = TB > 1 ? BF_PB_ : 0;
-  static constexpr int BF_BYTES = round16(TW * BF_ROW + (TW / K) * BF_PB);
+  static constexpr int BF_BYTES =
+      round16(TW * BF_ROW + (TB > 1 ? (TW / K) * BF_PB : 0));
   static constexpr int BCRAW_BYTES = ESZ == 2 ? round16(TW * N * 2) : 0;
   static constexpr int STAGE_BYTES =
       3 * RAW_BYTES + (ESZ == 2 ? 2 * BCRAW_BYTES : 2 * BF_BYTES);
+  // per warp: 2 parities x 32 slots x float4 (delta, delta, dx, dx)
+  static constexpr int XCH_BYTES = NW * 2 * 32 * 16;
   static constexpr int SMEM_BYTES =
-      2 * STAGE_BYTES + (ESZ == 2 ? 2 * BF_BYTES : 0);
+      2 * STAGE_BYTES + (ESZ == 2 ? 2 * BF_BYTES : 0) + XCH_BYTES;
   static constexpr int SUBWIN = TB * K;  // steps per sub-window (TB > 1)
 
   static_assert(NG == 1 || NG == 2 || NG == 4, "N must be 4, 8 or 16");
@@ -94,6 +121,8 @@ struct ChunkCfg {
   static_assert(K % NG == 0, "a time block holds whole NG-step blocks");
   static_assert(RAW_P % 16 == 0 && RAW_PB % 16 == 0 && BF_PB % 16 == 0,
                 "cp.async destinations are 16-byte aligned");
+  static_assert((TB > 1 ? K / NG : TW / NG) % 2 == 0,
+                "exchange slots alternate parity from block to block");
 
   __device__ static __forceinline__ int raw_off(int r) {
     return r * RAW_P + (r / BLK) * RAW_PB;
@@ -128,7 +157,9 @@ __device__ __forceinline__ float transpose_reduce(const float (&p)[NG], int g) {
   }
 }
 
-template <class Cfg>
+enum { kWalkMain = 0, kWalkCorrect = 1 };
+
+template <class Cfg, bool SPLIT>
 __global__ void __launch_bounds__(Cfg::THREADS)
 scan_chunked_kernel(const ScanParams p) {
   using T = typename Cfg::T;
@@ -137,6 +168,7 @@ scan_chunked_kernel(const ScanParams p) {
   constexpr int THREADS = Cfg::THREADS;
   constexpr unsigned FULL = 0xffffffffu;
   extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ unsigned s_word;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q = lane % TB;
@@ -146,10 +178,24 @@ scan_chunked_kernel(const ScanParams p) {
 
   const int64_t L = p.seqlen, E = p.dim;
   const int64_t tiles = (E + G - 1) / G;
-  const int64_t b = blockIdx.x / tiles;
-  const int64_t e0 = (blockIdx.x - b * tiles) * G;
+
+  // ---- which (piece, batch row, channel tile) this block scans
+  int64_t unit = blockIdx.x;
+  if constexpr (SPLIT) {
+    if (tid == 0) s_word = atomicAdd(p.ticket, 1u);
+    __syncthreads();
+    unit = s_word;
+    __syncthreads();
+  }
+  const int64_t seg = unit / (p.batch * tiles);
+  const int64_t rem = unit - seg * p.batch * tiles;
+  const int64_t b = rem / tiles;
+  const int64_t tile = rem - b * tiles;
+  const int64_t e0 = tile * G;
   const int64_t e = e0 + cl;
   const bool ch_ok = e < E;
+  const int64_t t_begin = SPLIT ? seg * p.seg_len : 0;
+  const int64_t t_end = SPLIT ? min(L, t_begin + p.seg_len) : L;
 
   const T *gx = static_cast<const T *>(p.x);
   const T *gdl = static_cast<const T *>(p.delta);
@@ -159,22 +205,29 @@ scan_chunked_kernel(const ScanParams p) {
   T *gy = static_cast<T *>(p.y);
   const bool has_z = gz != nullptr;
 
-  float A2[4];     // A * log2(e) for this lane's 4 states
-  float carry[4];  // state entering the next (sub-)window
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    A2[i] = 0.0f;
-    carry[i] = 0.0f;
-    if (ch_ok) {
-      // clamp so that a zero step never meets -inf (0 * -inf = NaN)
-      A2[i] = fmaxf(-expf(p.A_log[e * N + 4 * g + i]) * kLog2e, -FLT_MAX);
-      if (p.h0) carry[i] = p.h0[(b * E + e) * N + 4 * g + i];
+  float2 A01 = make_float2(0.0f, 0.0f), A23 = A01;  // A * log2(e)
+  float2 h01 = A01, h23 = A01;  // state (TB == 1) or carry (TB > 1)
+  if (ch_ok) {
+    const float *al = p.A_log + e * N + 4 * g;
+    // clamp so that a zero step never meets -inf (0 * -inf = NaN)
+    A01 = make_float2(fmaxf(-expf(al[0]) * kLog2e, -FLT_MAX),
+                      fmaxf(-expf(al[1]) * kLog2e, -FLT_MAX));
+    A23 = make_float2(fmaxf(-expf(al[2]) * kLog2e, -FLT_MAX),
+                      fmaxf(-expf(al[3]) * kLog2e, -FLT_MAX));
+    if (p.h0 && seg == 0) {
+      const float *hp = p.h0 + (b * E + e) * N + 4 * g;
+      h01 = make_float2(hp[0], hp[1]);
+      h23 = make_float2(hp[2], hp[3]);
     }
   }
   const float bias = (ch_ok && p.delta_bias) ? p.delta_bias[e] : 0.0f;
   const float Dv = (ch_ok && p.D) ? p.D[e] : 0.0f;
+  float2 P01 = make_float2(1.0f, 1.0f), P23 = P01;  // product of retentions
 
   float *const bf_conv = reinterpret_cast<float *>(smem + 2 * Cfg::STAGE_BYTES);
+  float4 *const xch = reinterpret_cast<float4 *>(
+      smem + 2 * Cfg::STAGE_BYTES + (ESZ == 2 ? 2 * Cfg::BF_BYTES : 0)) +
+      warp * 64;
 
   // ---- issue the copies of window w into stage s
   auto stage = [&](int64_t w, int s) {
@@ -186,7 +239,7 @@ scan_chunked_kernel(const ScanParams p) {
       const int r = idx / CPR, k = idx - (idx / CPR) * CPR;
       const int64_t t = t0 + r;
       const int64_t ec = e0 + k * EPC;
-      const bool ok = t < L && ec < E;
+      const bool ok = t < t_end && ec < E;
       const int64_t go = ok ? (b * L + t) * E + ec : 0;
       const int so = Cfg::raw_off(r) + k * 16;
       cp_async16(base + so, gx + go, ok);
@@ -199,7 +252,7 @@ scan_chunked_kernel(const ScanParams p) {
       constexpr int CH = TW * N * 2 / 16;
       for (int idx = tid; idx < CH; idx += THREADS) {
         const int r = idx * 16 / (N * 2);
-        const bool ok = t0 + r < L;
+        const bool ok = t0 + r < t_end;
         const int64_t go = ok ? (b * L + t0) * N + (int64_t)idx * 8 : 0;
         cp_async16(bc + idx * 16, gB + go, ok);
         cp_async16(bc + Cfg::BCRAW_BYTES + idx * 16, gC + go, ok);
@@ -209,7 +262,7 @@ scan_chunked_kernel(const ScanParams p) {
       constexpr int CPRB = N * 4 / 16;
       for (int idx = tid; idx < TW * CPRB; idx += THREADS) {
         const int r = idx / CPRB, k = idx - (idx / CPRB) * CPRB;
-        const bool ok = t0 + r < L;
+        const bool ok = t0 + r < t_end;
         const int64_t go = ok ? (b * L + t0 + r) * N + k * 4 : 0;
         const int so = Cfg::bf_off(r) + k * 16;
         cp_async16(bc + so, gB + go, ok);
@@ -218,202 +271,333 @@ scan_chunked_kernel(const ScanParams p) {
     }
   };
 
-  const int64_t nwin = (L + TW - 1) / TW;
-  stage(0, 0);
-  cp_async_commit();
-
-  float h[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) h[i] = carry[i];
-
-  for (int64_t w = 0; w < nwin; ++w) {
-    if (w + 1 < nwin) stage(w + 1, (w + 1) & 1);
+  // ---- walk windows [w_begin, w_end): MAIN stores y; CORRECT adds the
+  // response of the carried-in state (no write term, no D x) to stored y and
+  // stops as soon as that state is exactly zero everywhere in the block.
+  auto walk = [&](auto mode_c, int64_t w_begin, int64_t w_end) {
+    constexpr int MODE = decltype(mode_c)::value;
+    stage(w_begin, 0);
     cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-
-    const unsigned char *base = smem + (w & 1) * Cfg::STAGE_BYTES;
-    const unsigned char *sX = base;
-    const unsigned char *sDL = base + Cfg::RAW_BYTES;
-    const unsigned char *sZ = base + 2 * Cfg::RAW_BYTES;
-    const float *sB;
-    const float *sC;
-    if constexpr (ESZ == 2) {
-      const __nv_bfloat162 *rb = reinterpret_cast<const __nv_bfloat162 *>(
-          base + 3 * Cfg::RAW_BYTES);
-      const __nv_bfloat162 *rc = reinterpret_cast<const __nv_bfloat162 *>(
-          base + 3 * Cfg::RAW_BYTES + Cfg::BCRAW_BYTES);
-      float *fb = bf_conv;
-      float *fc = reinterpret_cast<float *>(
-          reinterpret_cast<unsigned char *>(bf_conv) + Cfg::BF_BYTES);
-      for (int idx = tid; idx < TW * N / 2; idx += THREADS) {
-        const int r = idx * 2 / N, n = idx * 2 - r * N;
-        const int o = (Cfg::bf_off(r) >> 2) + n;
-        const float2 vb = __bfloat1622float2(rb[idx]);
-        const float2 vc = __bfloat1622float2(rc[idx]);
-        *reinterpret_cast<float2 *>(fb + o) = vb;
-        *reinterpret_cast<float2 *>(fc + o) = vc;
-      }
+    for (int64_t w = w_begin; w < w_end; ++w) {
+      const int par = int((w - w_begin) & 1);
+      if (w + 1 < w_end) stage(w + 1, par ^ 1);
+      cp_async_commit();
+      cp_async_wait<1>();
       __syncthreads();
-      sB = fb;
-      sC = fc;
-    } else {
-      sB = reinterpret_cast<const float *>(base + 3 * Cfg::RAW_BYTES);
-      sC = reinterpret_cast<const float *>(base + 3 * Cfg::RAW_BYTES +
-                                           Cfg::BF_BYTES);
-    }
-    const int64_t t0 = w * TW;
 
-    // the raw (x, delta, z) of row r for this lane's channel
-    auto load_raw = [&](int r, float &xv, float &dv, float &zv) {
-      const int o = Cfg::raw_off(r) + cl * ESZ;
-      xv = Act<T>::load(reinterpret_cast<const T *>(sX + o));
-      dv = Act<T>::load(reinterpret_cast<const T *>(sDL + o));
-      zv = has_z ? Act<T>::load(reinterpret_cast<const T *>(sZ + o)) : 0.0f;
-    };
-    // step size and step * x for row r (zero past the end of the sequence)
-    auto step_of = [&](int r, float xv, float dv, float &dm, float &dxm) {
-      const float v = dv + bias;
-      dm = p.softplus ? softplus(v) : v;
-      if (t0 + r >= L) dm = 0.0f;
-      dxm = dm * xv;
-    };
-    auto finish = [&](int r, float yv, float xv, float zv) {
-      yv = fmaf(Dv, xv, yv);
-      if (has_z) yv *= silu(zv);
-      const int64_t t = t0 + r;
-      if (ch_ok && t < L) Act<T>::store(gy + (b * L + t) * E + e, yv);
-    };
-
-    if constexpr (TB == 1) {
-#pragma unroll 2
-      for (int jb = 0; jb < TW / NG; ++jb) {
-        const int rm = jb * NG + g;
-        float xm, dv, zm, dm, dxm;
-        load_raw(rm, xm, dv, zm);
-        step_of(rm, xm, dv, dm, dxm);
-        float ps[NG];
-#pragma unroll
-        for (int s = 0; s < NG; ++s) {
-          const int src = c * NG + s;
-          const float ds = __shfl_sync(FULL, dm, src);
-          const float dxs = __shfl_sync(FULL, dxm, src);
-          const int r = jb * NG + s;
-          const float4 Bq =
-              *reinterpret_cast<const float4 *>(sB + (Cfg::bf_off(r) >> 2) + 4 * g);
-          const float4 Cq =
-              *reinterpret_cast<const float4 *>(sC + (Cfg::bf_off(r) >> 2) + 4 * g);
-          const float bq[4] = {Bq.x, Bq.y, Bq.z, Bq.w};
-          const float cq[4] = {Cq.x, Cq.y, Cq.z, Cq.w};
-          float acc = 0.0f;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float a = ex2(ds * A2[i]);
-            h[i] = fmaf(a, h[i], dxs * bq[i]);
-            acc = fmaf(cq[i], h[i], acc);
-          }
-          ps[s] = acc;
+      const unsigned char *base = smem + par * Cfg::STAGE_BYTES;
+      const unsigned char *sX = base;
+      const unsigned char *sDL = base + Cfg::RAW_BYTES;
+      const unsigned char *sZ = base + 2 * Cfg::RAW_BYTES;
+      const float *sB;
+      const float *sC;
+      if constexpr (ESZ == 2) {
+        const __nv_bfloat162 *rb = reinterpret_cast<const __nv_bfloat162 *>(
+            base + 3 * Cfg::RAW_BYTES);
+        const __nv_bfloat162 *rc = reinterpret_cast<const __nv_bfloat162 *>(
+            base + 3 * Cfg::RAW_BYTES + Cfg::BCRAW_BYTES);
+        float *fb = bf_conv;
+        float *fc = reinterpret_cast<float *>(
+            reinterpret_cast<unsigned char *>(bf_conv) + Cfg::BF_BYTES);
+        for (int idx = tid; idx < TW * N / 2; idx += THREADS) {
+          const int r = idx * 2 / N, n = idx * 2 - r * N;
+          const int o = (Cfg::bf_off(r) >> 2) + n;
+          *reinterpret_cast<float2 *>(fb + o) = __bfloat1622float2(rb[idx]);
+          *reinterpret_cast<float2 *>(fc + o) = __bfloat1622float2(rc[idx]);
         }
-        const float yv = transpose_reduce<NG, TB>(ps, g);
-        finish(rm, yv, xm, zm);
+        __syncthreads();
+        sB = fb;
+        sC = fc;
+      } else {
+        sB = reinterpret_cast<const float *>(base + 3 * Cfg::RAW_BYTES);
+        sC = reinterpret_cast<const float *>(base + 3 * Cfg::RAW_BYTES +
+                                             Cfg::BF_BYTES);
       }
-    } else {
-      constexpr int M = TW / Cfg::SUBWIN;
-      constexpr int NB = K / NG;  // NG-step blocks per time block
-#pragma unroll 1
-      for (int m = 0; m < M; ++m) {
-        const int r0 = m * Cfg::SUBWIN + q * K;  // first row of my time block
-        float a[K][4], wr[K][4];
-        float xs[NB], zs[NB];
-        float Aa[4] = {1.0f, 1.0f, 1.0f, 1.0f};
-        float Bb[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        // pass 1: per-step maps, folded into one map per time block
-#pragma unroll
-        for (int jb = 0; jb < NB; ++jb) {
-          const int rm = r0 + jb * NG + g;
-          float xm, dv, zm, dm, dxm;
-          load_raw(rm, xm, dv, zm);
-          step_of(rm, xm, dv, dm, dxm);
-          xs[jb] = xm;
-          zs[jb] = zm;
-#pragma unroll
-          for (int s = 0; s < NG; ++s) {
-            const int src = (c * NG + s) * TB + q;
-            const float ds = __shfl_sync(FULL, dm, src);
-            const float dxs = __shfl_sync(FULL, dxm, src);
-            const int j = jb * NG + s;
-            const float4 Bq = *reinterpret_cast<const float4 *>(
-                sB + (Cfg::bf_off(r0 + j) >> 2) + 4 * g);
-            const float bq[4] = {Bq.x, Bq.y, Bq.z, Bq.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              a[j][i] = ex2(ds * A2[i]);
-              wr[j][i] = dxs * bq[i];
-              Bb[i] = fmaf(a[j][i], Bb[i], wr[j][i]);
-              Aa[i] *= a[j][i];
-            }
-          }
+      const int64_t t0 = w * TW;
+      const int64_t ybase = (b * L + t0) * E + e;
+
+      // this lane's step of a block: load its inputs, compute its step size,
+      // publish (d, d, d x, d x) for the lanes of its channel and time block
+      auto produce = [&](int r, int slot_par, float &xm, float &zm) {
+        const int o = Cfg::raw_off(r) + cl * ESZ;
+        xm = Act<T>::load(reinterpret_cast<const T *>(sX + o));
+        const float dv = Act<T>::load(reinterpret_cast<const T *>(sDL + o));
+        zm = has_z ? Act<T>::load(reinterpret_cast<const T *>(sZ + o)) : 0.0f;
+        const float v = dv + bias;
+        float dm = p.softplus ? softplus(v) : v;
+        if (t0 + r >= t_end) dm = 0.0f;
+        const float dxm = MODE == kWalkMain ? dm * xm : 0.0f;
+        xch[slot_par * 32 + (c * TB + q) * NG + g] =
+            make_float4(dm, dm, dxm, dxm);
+      };
+      auto finish = [&](int r, float yv, float xm, float zm) {
+        const int64_t t = t0 + r;
+        if (MODE == kWalkMain) yv = fmaf(Dv, xm, yv);
+        if (has_z) yv *= silu(zm);
+        if (ch_ok && t < t_end) {
+          T *yp = gy + ybase + int64_t(r) * E;
+          if (MODE == kWalkCorrect) yv += Act<T>::load(yp);
+          Act<T>::store(yp, yv);
         }
-        // the incoming state enters at the first time block
-        if (q == 0) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) Bb[i] = fmaf(Aa[i], carry[i], Bb[i]);
-        }
-        // inclusive warp-shuffle scan of the block maps over the TB lanes
-#pragma unroll
-        for (int d = 1; d < TB; d <<= 1) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float Ap = __shfl_up_sync(FULL, Aa[i], d, TB);
-            const float Bp = __shfl_up_sync(FULL, Bb[i], d, TB);
-            if (q >= d) {
-              Bb[i] = fmaf(Aa[i], Bp, Bb[i]);
-              Aa[i] *= Ap;
-            }
-          }
-        }
-        // Bb = state at the end of my block; the previous lane's is mine to
-        // start from, the last lane's goes to the next sub-window
-        float hs[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float prev = __shfl_up_sync(FULL, Bb[i], 1, TB);
-          hs[i] = q == 0 ? carry[i] : prev;
-          carry[i] = __shfl_sync(FULL, Bb[i], TB - 1, TB);
-        }
-        // pass 2: replay the block from the true incoming state, read out
-#pragma unroll
-        for (int jb = 0; jb < NB; ++jb) {
+      };
+      // one step of the 4 states: a = 2^(d A'), h = a h + d x B, partial C.h
+      auto bc_row = [&](int r, float4 &Bq, float4 &Cq) {
+        const int o = (Cfg::bf_off(r) >> 2) + 4 * g;
+        Bq = *reinterpret_cast<const float4 *>(sB + o);
+        Cq = *reinterpret_cast<const float4 *>(sC + o);
+      };
+
+      if constexpr (TB == 1) {
+#pragma unroll 2
+        for (int jb = 0; jb < TW / NG; ++jb) {
+          const int rm = jb * NG + g;
+          const int sp = jb & 1;
+          float xm, zm;
+          produce(rm, sp, xm, zm);
+          __syncwarp();
           float ps[NG];
 #pragma unroll
           for (int s = 0; s < NG; ++s) {
-            const int j = jb * NG + s;
-            const float4 Cq = *reinterpret_cast<const float4 *>(
-                sC + (Cfg::bf_off(r0 + j) >> 2) + 4 * g);
-            const float cq[4] = {Cq.x, Cq.y, Cq.z, Cq.w};
-            float acc = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              hs[i] = fmaf(a[j][i], hs[i], wr[j][i]);
-              acc = fmaf(cq[i], hs[i], acc);
+            const float4 dd = xch[sp * 32 + c * NG + s];
+            float4 Bq, Cq;
+            bc_row(jb * NG + s, Bq, Cq);
+            const float2 dA = make_float2(dd.x, dd.y);
+            const float2 a01 = ex2x2(mul2(dA, A01));
+            const float2 a23 = ex2x2(mul2(dA, A23));
+            if (MODE == kWalkMain) {
+              const float2 dx = make_float2(dd.z, dd.w);
+              h01 = fma2(a01, h01, mul2(dx, make_float2(Bq.x, Bq.y)));
+              h23 = fma2(a23, h23, mul2(dx, make_float2(Bq.z, Bq.w)));
+              if constexpr (SPLIT) {
+                P01 = mul2(P01, a01);
+                P23 = mul2(P23, a23);
+              }
+            } else {
+              h01 = mul2(a01, h01);
+              h23 = mul2(a23, h23);
             }
-            ps[s] = acc;
+            const float2 acc =
+                fma2(make_float2(Cq.z, Cq.w), h23,
+                     mul2(make_float2(Cq.x, Cq.y), h01));
+            ps[s] = acc.x + acc.y;
           }
-          const float yv = transpose_reduce<NG, TB>(ps, g);
-          finish(r0 + jb * NG + g, yv, xs[jb], zs[jb]);
+          finish(rm, transpose_reduce<NG, TB>(ps, g), xm, zm);
+        }
+      } else {
+        constexpr int M = TW / Cfg::SUBWIN;
+        constexpr int NB = K / NG;  // NG-step blocks per time block
+#pragma unroll 1
+        for (int m = 0; m < M; ++m) {
+          const int r0 = m * Cfg::SUBWIN + q * K;  // first row of my block
+          float2 a01[K], a23[K], w01[K], w23[K];
+          float xs[NB], zs[NB];
+          float2 Aa01 = make_float2(1.0f, 1.0f), Aa23 = Aa01;
+          float2 Bb01 = make_float2(0.0f, 0.0f), Bb23 = Bb01;
+          // pass 1: per-step maps, folded into one map per time block
+#pragma unroll
+          for (int jb = 0; jb < NB; ++jb) {
+            const int sp = jb & 1;
+            produce(r0 + jb * NG + g, sp, xs[jb], zs[jb]);
+            __syncwarp();
+#pragma unroll
+            for (int s = 0; s < NG; ++s) {
+              const int j = jb * NG + s;
+              const float4 dd = xch[sp * 32 + (c * TB + q) * NG + s];
+              float4 Bq, Cq;
+              bc_row(r0 + j, Bq, Cq);
+              const float2 dA = make_float2(dd.x, dd.y);
+              const float2 dx = make_float2(dd.z, dd.w);
+              a01[j] = ex2x2(mul2(dA, A01));
+              a23[j] = ex2x2(mul2(dA, A23));
+              w01[j] = mul2(dx, make_float2(Bq.x, Bq.y));
+              w23[j] = mul2(dx, make_float2(Bq.z, Bq.w));
+              Bb01 = fma2(a01[j], Bb01, w01[j]);
+              Bb23 = fma2(a23[j], Bb23, w23[j]);
+              Aa01 = mul2(Aa01, a01[j]);
+              Aa23 = mul2(Aa23, a23[j]);
+            }
+          }
+          // the incoming state enters at the first time block
+          if (q == 0) {
+            Bb01 = fma2(Aa01, h01, Bb01);
+            Bb23 = fma2(Aa23, h23, Bb23);
+          }
+          // inclusive warp-shuffle scan of the block maps over the TB lanes
+#pragma unroll
+          for (int d = 1; d < TB; d <<= 1) {
+            float2 Ap01, Ap23, Bp01, Bp23;
+            Ap01.x = __shfl_up_sync(FULL, Aa01.x, d, TB);
+            Ap01.y = __shfl_up_sync(FULL, Aa01.y, d, TB);
+            Ap23.x = __shfl_up_sync(FULL, Aa23.x, d, TB);
+            Ap23.y = __shfl_up_sync(FULL, Aa23.y, d, TB);
+            Bp01.x = __shfl_up_sync(FULL, Bb01.x, d, TB);
+            Bp01.y = __shfl_up_sync(FULL, Bb01.y, d, TB);
+            Bp23.x = __shfl_up_sync(FULL, Bb23.x, d, TB);
+            Bp23.y = __shfl_up_sync(FULL, Bb23.y, d, TB);
+            if (q >= d) {
+              Bb01 = fma2(Aa01, Bp01, Bb01);
+              Bb23 = fma2(Aa23, Bp23, Bb23);
+              Aa01 = mul2(Aa01, Ap01);
+              Aa23 = mul2(Aa23, Ap23);
+            }
+          }
+          if constexpr (SPLIT) {
+            if (MODE == kWalkMain) {
+              // the whole sub-window's retention product sits in the last lane
+              float2 S01, S23;
+              S01.x = __shfl_sync(FULL, Aa01.x, TB - 1, TB);
+              S01.y = __shfl_sync(FULL, Aa01.y, TB - 1, TB);
+              S23.x = __shfl_sync(FULL, Aa23.x, TB - 1, TB);
+              S23.y = __shfl_sync(FULL, Aa23.y, TB - 1, TB);
+              P01 = mul2(P01, S01);
+              P23 = mul2(P23, S23);
+            }
+          }
+          // Bb = state at the end of my block. The previous lane's is mine to
+          // start from; the last lane's carries to the next sub-window.
+          float2 hs01, hs23;
+          hs01.x = __shfl_up_sync(FULL, Bb01.x, 1, TB);
+          hs01.y = __shfl_up_sync(FULL, Bb01.y, 1, TB);
+          hs23.x = __shfl_up_sync(FULL, Bb23.x, 1, TB);
+          hs23.y = __shfl_up_sync(FULL, Bb23.y, 1, TB);
+          if (q == 0) {
+            hs01 = h01;
+            hs23 = h23;
+          }
+          h01.x = __shfl_sync(FULL, Bb01.x, TB - 1, TB);
+          h01.y = __shfl_sync(FULL, Bb01.y, TB - 1, TB);
+          h23.x = __shfl_sync(FULL, Bb23.x, TB - 1, TB);
+          h23.y = __shfl_sync(FULL, Bb23.y, TB - 1, TB);
+          // pass 2: replay the block from the true incoming state, read out
+#pragma unroll
+          for (int jb = 0; jb < NB; ++jb) {
+            float ps[NG];
+#pragma unroll
+            for (int s = 0; s < NG; ++s) {
+              const int j = jb * NG + s;
+              float4 Bq, Cq;
+              bc_row(r0 + j, Bq, Cq);
+              hs01 = fma2(a01[j], hs01, w01[j]);
+              hs23 = fma2(a23[j], hs23, w23[j]);
+              const float2 acc =
+                  fma2(make_float2(Cq.z, Cq.w), hs23,
+                       mul2(make_float2(Cq.x, Cq.y), hs01));
+              ps[s] = acc.x + acc.y;
+            }
+            finish(r0 + jb * NG + g, transpose_reduce<NG, TB>(ps, g), xs[jb],
+                   zs[jb]);
+          }
         }
       }
+      if (MODE == kWalkCorrect) {
+        const int alive = (h01.x != 0.0f) | (h01.y != 0.0f) |
+                          (h23.x != 0.0f) | (h23.y != 0.0f);
+        if (!__syncthreads_or(alive)) break;
+      } else {
+        __syncthreads();
+      }
     }
+    cp_async_wait<0>();
     __syncthreads();
+  };
+
+  const int64_t w_begin = t_begin / TW;
+  const int64_t w_end = (t_end + TW - 1) / TW;
+  walk(std::integral_constant<int, kWalkMain>(), w_begin, w_end);
+
+  float2 H01 = h01, H23 = h23;  // true end state of this piece
+  if constexpr (SPLIT) {
+    const int64_t S = p.segments;
+    const int64_t slot = ((b * S + seg) * E + e) * N + 4 * g;
+    unsigned *flag_of = p.flags + (b * S) * tiles + tile;  // + j * tiles
+    const unsigned tag = p.epoch << 2;
+    // publish the aggregate (the first piece's is already inclusive)
+    if (ch_ok && q == 0) {
+      if (seg == 0) {
+        __stcg(reinterpret_cast<float4 *>(p.incl_state + slot),
+               make_float4(h01.x, h01.y, h23.x, h23.y));
+      } else {
+        __stcg(reinterpret_cast<float4 *>(p.agg_state + slot),
+               make_float4(h01.x, h01.y, h23.x, h23.y));
+        __stcg(reinterpret_cast<float4 *>(p.agg_decay + slot),
+               make_float4(P01.x, P01.y, P23.x, P23.y));
+      }
+    }
+    __threadfence();
+    __syncthreads();
+    const bool suppress = (p.debug & kDebugNoPublish) && seg == 0;
+    if (tid == 0 && !suppress)
+      st_release(flag_of + seg * tiles,
+                 tag | (seg == 0 ? kFlagInclusive : kFlagAggregate));
+
+    if (seg > 0) {
+      // look back: compose predecessors' aggregates until an inclusive one
+      float2 cP01 = make_float2(1.0f, 1.0f), cP23 = cP01;  // map from there
+      float2 cS01 = make_float2(0.0f, 0.0f), cS23 = cS01;  // to this start
+      float2 hin01, hin23;
+      for (int64_t j = seg - 1;; --j) {
+        if (tid == 0) {
+          unsigned f = 0, st = kFlagNone;
+          for (unsigned spin = 0; spin < p.spin_limit; ++spin) {
+            f = ld_acquire(flag_of + j * tiles);
+            if ((f & ~3u) == tag && (f & 3u) != kFlagNone) {
+              st = f & 3u;
+              break;
+            }
+            __nanosleep(64);
+          }
+          s_word = st;
+        }
+        __syncthreads();
+        const unsigned st = s_word;
+        __syncthreads();
+        const int64_t js = ((b * S + j) * E + e) * N + 4 * g;
+        if (st == kFlagNone || j == 0 && st != kFlagInclusive) {
+          if (tid == 0) atomicExch(p.status, kStatusTimeout);
+          hin01 = cS01;
+          hin23 = cS23;
+          break;
+        }
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (st == kFlagInclusive) {
+          if (ch_ok) v = __ldcg(reinterpret_cast<const float4 *>(p.incl_state + js));
+          hin01 = fma2(cP01, make_float2(v.x, v.y), cS01);
+          hin23 = fma2(cP23, make_float2(v.z, v.w), cS23);
+          break;
+        }
+        float4 u = v;
+        if (ch_ok) {
+          v = __ldcg(reinterpret_cast<const float4 *>(p.agg_state + js));
+          u = __ldcg(reinterpret_cast<const float4 *>(p.agg_decay + js));
+        }
+        cS01 = fma2(cP01, make_float2(v.x, v.y), cS01);
+        cS23 = fma2(cP23, make_float2(v.z, v.w), cS23);
+        cP01 = mul2(cP01, make_float2(u.x, u.y));
+        cP23 = mul2(cP23, make_float2(u.z, u.w));
+      }
+      // inclusive end state: own aggregate applied after the incoming state
+      H01 = fma2(P01, hin01, h01);
+      H23 = fma2(P23, hin23, h23);
+      if (ch_ok && q == 0)
+        __stcg(reinterpret_cast<float4 *>(p.incl_state + slot),
+               make_float4(H01.x, H01.y, H23.x, H23.y));
+      __threadfence();
+      __syncthreads();
+      if (tid == 0) st_release(flag_of + seg * tiles, tag | kFlagInclusive);
+      // replay the start of the piece for the carried-in state's response
+      h01 = hin01;
+      h23 = hin23;
+      if (!ch_ok) h01 = h23 = make_float2(0.0f, 0.0f);
+      walk(std::integral_constant<int, kWalkCorrect>(), w_begin, w_end);
+    }
   }
 
-  if (TB == 1) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) carry[i] = h[i];
-  }
-  if (p.h_last && ch_ok && q == 0) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) p.h_last[(b * E + e) * N + 4 * g + i] = carry[i];
+  if (p.h_last && ch_ok && q == 0 && t_end == L) {
+    float *hp = p.h_last + (b * E + e) * N + 4 * g;
+    hp[0] = H01.x;
+    hp[1] = H01.y;
+    hp[2] = H23.x;
+    hp[3] = H23.y;
   }
 }
 

@@ -20,18 +20,31 @@ struct ScanParams {
   int64_t batch, seqlen, dim;
   int dstate;
   int softplus;              // apply softplus to delta + bias
-  // split-sequence workspace (chunked variant with segments > 1)
+  // Split sequences (chunked variant): each sequence is cut into `segments`
+  // pieces of seg_len steps (a multiple of the window), scanned concurrently
+  // from a zero state and joined by a decoupled look-back over per-piece
+  // affine aggregates in the workspace below.
   int segments;              // pieces per sequence (1 = no split)
-  int64_t seg_len;           // steps per piece (multiple of the window)
-  float *seg_state;          // [b, segments, E, N] end state from a zero start
-  float *seg_decay;          // [b, segments, E, N] product of retentions
-  unsigned *seg_flag;        // [b, segments, E / tile] publication flags
-  unsigned *ticket;          // [1] launch-order ticket counter
-  int *status;               // [1] device status word (0 = ok)
-  unsigned epoch;            // value written to flags by this call
+  int64_t seg_len;           // steps per piece
+  unsigned *flags;           // [b, segments, tiles] publication words
+  float *agg_state;          // [b, segments, E, N] end state from zero
+  float *agg_decay;          // [b, segments, E, N] product of retentions
+  float *incl_state;         // [b, segments, E, N] true end state
+  unsigned *ticket;          // launch-order counter, zero before the launch
+  int *status;               // device status word (kStatus*)
+  unsigned epoch;            // tag of this call in the publication words
+  unsigned spin_limit;       // bounded wait: polls before giving up
+  unsigned debug;            // kDebug* bits (tests only)
 };
 
 // Device status codes written to ScanParams::status.
 enum { kStatusOk = 0, kStatusTimeout = 1 };
+
+// Publication states (low 2 bits of a flag word; the rest is the epoch).
+enum { kFlagNone = 0, kFlagAggregate = 1, kFlagInclusive = 2 };
+
+// Test hook: the first piece of every sequence never publishes, so its
+// successor's bounded wait must run out and report kStatusTimeout.
+enum { kDebugNoPublish = 1u << 0 };
 
 }  // namespace ssm

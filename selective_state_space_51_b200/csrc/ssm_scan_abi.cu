@@ -10,6 +10,8 @@
 #include "kernel_chunked.cuh"
 #include "kernel_sequential.cuh"
 
+constexpr unsigned kDefaultSpinLimit = 1000u * 1000u;  // ~1 s of polls
+
 struct ssm_scan_s {
   int device = 0;
   int sm_count = 0;
@@ -19,7 +21,11 @@ struct ssm_scan_s {
   int last_variant = 0;
   int last_segments = 0;
   unsigned epoch = 0;
-  // device workspace: [status word, ticket][segment carry arrays]
+  unsigned debug = 0;
+  unsigned spin_limit = kDefaultSpinLimit;
+  // control block: [0] status word, [1] launch ticket (device, 256 bytes)
+  int *ctl = nullptr;
+  // split-sequence workspace: flags, then three state arrays
   void *ws = nullptr;
   size_t ws_bytes = 0;
 };
@@ -58,23 +64,97 @@ int dispatch_sequential(const ssm::ScanParams &p, cudaStream_t s) {
 // free for that lane layout.
 using bf16 = __nv_bfloat16;
 //                          T      NG TB  K  TW NW pad  PB  BFPB
-using C16b1 = ssm::ChunkCfg<bf16,  4, 1, 4, 64, 4, 16,  0,  0>;
-using C16f1 = ssm::ChunkCfg<float, 4, 1, 4, 64, 4, 32,  0,  0>;
-using C16b2 = ssm::ChunkCfg<bf16,  4, 2, 8, 64, 4,  0, 16, 64>;
-using C16f2 = ssm::ChunkCfg<float, 4, 2, 8, 64, 4, 32, 16, 64>;
-using C8b1 = ssm::ChunkCfg<bf16,   2, 1, 2, 64, 4, 32,  0,  0>;
-using C8f1 = ssm::ChunkCfg<float,  2, 1, 2, 64, 4, 64,  0,  0>;
-using C8b2 = ssm::ChunkCfg<bf16,   2, 2, 8, 64, 4,  0, 16, 32>;
-using C8f2 = ssm::ChunkCfg<float,  2, 2, 8, 64, 4, 32, 64, 32>;
-using C4f1 = ssm::ChunkCfg<float,  1, 1, 1, 64, 4,  0,  0,  0>;
-using C4f2 = ssm::ChunkCfg<float,  1, 2, 8, 64, 4,  0, 64, 16>;
+using C16b1 = ssm::ChunkCfg<bf16,  4, 1, 4, 32, 4, 16,  0,  0>;
+using C16f1 = ssm::ChunkCfg<float, 4, 1, 4, 16, 4, 32,  0,  0>;
+using C16b2 = ssm::ChunkCfg<bf16,  4, 2, 8, 32, 4,  0, 16, 64>;
+using C16f2 = ssm::ChunkCfg<float, 4, 2, 8, 16, 4, 32, 16, 64>;
+using C8b1 = ssm::ChunkCfg<bf16,   2, 1, 2, 32, 4, 32,  0,  0>;
+using C8f1 = ssm::ChunkCfg<float,  2, 1, 2, 16, 4, 64,  0,  0>;
+using C8b2 = ssm::ChunkCfg<bf16,   2, 2, 8, 32, 4,  0, 16, 32>;
+using C8f2 = ssm::ChunkCfg<float,  2, 2, 8, 16, 4, 32, 64, 32>;
+using C4f1 = ssm::ChunkCfg<float,  1, 1, 1, 16, 4,  0,  0,  0>;
+using C4f2 = ssm::ChunkCfg<float,  1, 2, 8, 16, 4,  0, 64, 16>;
 
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Grow the split workspace for `segs` pieces; fills the ScanParams pointers.
+int ensure_workspace(ssm_scan_s *h, ssm::ScanParams &p, int64_t tiles,
+                     int64_t segs, cudaStream_t s) {
+  const size_t nflags = size_t(p.batch) * segs * tiles;
+  const size_t nstate = size_t(p.batch) * segs * p.dim * p.dstate;
+  const size_t off_state = align256(nflags * sizeof(unsigned));
+  const size_t bytes = off_state + 3 * align256(nstate * sizeof(float));
+  if (!h->ctl) {
+    if (cudaMallocAsync(reinterpret_cast<void **>(&h->ctl), 256, s) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return SSM_ERR_NOMEM;
+    }
+    if (cudaMemsetAsync(h->ctl, 0, 256, s) != cudaSuccess) return SSM_ERR_CUDA;
+  }
+  if (bytes > h->ws_bytes) {
+    if (h->ws) cudaFreeAsync(h->ws, s);
+    h->ws = nullptr;
+    h->ws_bytes = 0;
+    if (cudaMallocAsync(&h->ws, bytes, s) != cudaSuccess) {
+      cudaGetLastError();
+      return SSM_ERR_NOMEM;
+    }
+    if (cudaMemsetAsync(h->ws, 0, bytes, s) != cudaSuccess) return SSM_ERR_CUDA;
+    h->ws_bytes = bytes;
+    h->epoch = 0;
+  }
+  if (++h->epoch >= (1u << 30)) {  // tags wrap: clear the flags first
+    if (cudaMemsetAsync(h->ws, 0, off_state, s) != cudaSuccess)
+      return SSM_ERR_CUDA;
+    h->epoch = 1;
+  }
+  unsigned char *base = static_cast<unsigned char *>(h->ws);
+  const size_t sz = align256(nstate * sizeof(float));
+  p.flags = reinterpret_cast<unsigned *>(base);
+  p.agg_state = reinterpret_cast<float *>(base + off_state);
+  p.agg_decay = reinterpret_cast<float *>(base + off_state + sz);
+  p.incl_state = reinterpret_cast<float *>(base + off_state + 2 * sz);
+  p.status = h->ctl;
+  p.ticket = reinterpret_cast<unsigned *>(h->ctl + 1);
+  p.epoch = h->epoch;
+  p.spin_limit = h->spin_limit;
+  p.debug = h->debug;
+  return cudaMemsetAsync(p.ticket, 0, sizeof(unsigned), s) == cudaSuccess
+             ? SSM_OK
+             : SSM_ERR_CUDA;
+}
+
+// Pieces per sequence: enough that the blocks fill every resident slot once,
+// each piece at least 64 windows long (so the start-up replay after the
+// look-back stays a small fraction), and 1 when channels alone fill the GPU.
 template <class Cfg>
-int launch_chunked(const ssm::ScanParams &p, cudaStream_t s) {
+int64_t auto_segments(const ssm::ScanParams &p, int sm_count) {
+  static int per_sm = 0;  // resident blocks per SM for this shape
+  if (!per_sm) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &n, ssm::scan_chunked_kernel<Cfg, true>, Cfg::THREADS,
+            Cfg::SMEM_BYTES) != cudaSuccess) {
+      cudaGetLastError();
+      n = 1;
+    }
+    per_sm = n > 0 ? n : 1;
+  }
   const int64_t tiles = (p.dim + Cfg::G - 1) / Cfg::G;
-  const int64_t blocks = p.batch * tiles;
+  const int64_t base = p.batch * tiles;
+  const int64_t slots = int64_t(per_sm) * sm_count;
+  if (base * 2 > slots) return 1;
+  const int64_t max_segs = p.seqlen / (64 * Cfg::TW);
+  int64_t segs = slots / base;
+  if (segs > max_segs) segs = max_segs;
+  return segs < 2 ? 1 : segs;
+}
+
+template <class Cfg, bool SPLIT>
+int launch_kernel(const ssm::ScanParams &p, int64_t blocks, cudaStream_t s) {
   if (blocks > 0x7fffffff) return SSM_ERR_UNSUPPORTED;
-  auto kern = ssm::scan_chunked_kernel<Cfg>;
+  auto kern = ssm::scan_chunked_kernel<Cfg, SPLIT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Cfg::SMEM_BYTES) != cudaSuccess) {
     cudaGetLastError();
@@ -82,6 +162,27 @@ int launch_chunked(const ssm::ScanParams &p, cudaStream_t s) {
   }
   kern<<<(unsigned)blocks, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+template <class Cfg>
+int launch_chunked(ssm_scan_s *h, ssm::ScanParams &p, int64_t segs_req,
+                   cudaStream_t s) {
+  const int64_t tiles = (p.dim + Cfg::G - 1) / Cfg::G;
+  int64_t segs = segs_req > 0 ? segs_req : auto_segments<Cfg>(p, h->sm_count);
+  int64_t seg_len = p.seqlen;
+  if (segs > 1) {
+    const int64_t wins = (p.seqlen + Cfg::TW - 1) / Cfg::TW;
+    const int64_t per = (wins + segs - 1) / segs;
+    seg_len = per * Cfg::TW;
+    segs = (p.seqlen + seg_len - 1) / seg_len;
+  }
+  p.segments = int(segs);
+  p.seg_len = seg_len;
+  h->last_segments = int(segs);
+  if (segs <= 1) return launch_kernel<Cfg, false>(p, p.batch * tiles, s);
+  const int rc = ensure_workspace(h, p, tiles, segs, s);
+  if (rc != SSM_OK) return rc;
+  return launch_kernel<Cfg, true>(p, segs * p.batch * tiles, s);
 }
 
 // Whether the chunked variant can run these arguments: N of 4, 8 or 16, whole
@@ -97,30 +198,29 @@ bool chunked_supported(const ssm::ScanParams &p, int dtype) {
   return true;
 }
 
-// Time blocks per channel: 1 while the channels alone give every SM
-// sub-partition several warps, else 2.
-int auto_time_blocks(const ssm::ScanParams &p, int sm_count) {
-  const int64_t warps1 = p.batch * p.dim * (p.dstate / 4) / 32;
-  return warps1 >= 4LL * 4 * sm_count ? 1 : 2;
-}
+// Time blocks per channel: 1. Where channels are few, sequences are split
+// into pieces instead (see auto_segments), which keeps the cheaper
+// one-lane-per-step arithmetic; 2 is available on request.
+int auto_time_blocks(const ssm::ScanParams &, int) { return 1; }
 
-template <typename T, class Cf1, class Cf2>
-int pick(const ssm::ScanParams &p, int tb, cudaStream_t s) {
-  if (tb == 1) return launch_chunked<Cf1>(p, s);
-  if (tb == 2) return launch_chunked<Cf2>(p, s);
+template <class Cf1, class Cf2>
+int pick(ssm_scan_s *h, ssm::ScanParams &p, int tb, int64_t segs,
+         cudaStream_t s) {
+  if (tb == 1) return launch_chunked<Cf1>(h, p, segs, s);
+  if (tb == 2) return launch_chunked<Cf2>(h, p, segs, s);
   return SSM_ERR_UNSUPPORTED;
 }
 
-int dispatch_chunked(const ssm::ScanParams &p, int dtype, int tb,
-                     cudaStream_t s) {
+int dispatch_chunked(ssm_scan_s *h, ssm::ScanParams &p, int dtype, int tb,
+                     int64_t segs, cudaStream_t s) {
   if (dtype == SSM_BF16) {
-    if (p.dstate == 16) return pick<bf16, C16b1, C16b2>(p, tb, s);
-    if (p.dstate == 8) return pick<bf16, C8b1, C8b2>(p, tb, s);
+    if (p.dstate == 16) return pick<C16b1, C16b2>(h, p, tb, segs, s);
+    if (p.dstate == 8) return pick<C8b1, C8b2>(h, p, tb, segs, s);
     return SSM_ERR_UNSUPPORTED;
   }
-  if (p.dstate == 16) return pick<float, C16f1, C16f2>(p, tb, s);
-  if (p.dstate == 8) return pick<float, C8f1, C8f2>(p, tb, s);
-  if (p.dstate == 4) return pick<float, C4f1, C4f2>(p, tb, s);
+  if (p.dstate == 16) return pick<C16f1, C16f2>(h, p, tb, segs, s);
+  if (p.dstate == 8) return pick<C8f1, C8f2>(h, p, tb, segs, s);
+  if (p.dstate == 4) return pick<C4f1, C4f2>(h, p, tb, segs, s);
   return SSM_ERR_UNSUPPORTED;
 }
 
@@ -159,11 +259,12 @@ int ssm_scan_create(ssm_scan_t *out, int device) {
 int ssm_scan_destroy(ssm_scan_t h) {
   if (!h) return SSM_OK;
   int rc = SSM_OK;
-  if (h->ws) {
+  if (h->ws || h->ctl) {
     int prev = 0;
     cudaGetDevice(&prev);
     cudaSetDevice(h->device);
-    if (cudaFree(h->ws) != cudaSuccess) rc = SSM_ERR_CUDA;
+    if (h->ws && cudaFree(h->ws) != cudaSuccess) rc = SSM_ERR_CUDA;
+    if (h->ctl && cudaFree(h->ctl) != cudaSuccess) rc = SSM_ERR_CUDA;
     cudaSetDevice(prev);
   }
   delete h;
@@ -177,6 +278,13 @@ int ssm_scan_set_variant(ssm_scan_t h, int variant, int segments) {
   if (segments < 0) return SSM_ERR_INVALID;
   h->variant = variant;
   h->segments = segments;
+  return SSM_OK;
+}
+
+int ssm_scan_set_debug(ssm_scan_t h, unsigned flags, unsigned spin_limit) {
+  if (!h) return SSM_ERR_INVALID;
+  h->debug = flags;
+  h->spin_limit = spin_limit ? spin_limit : kDefaultSpinLimit;
   return SSM_OK;
 }
 
@@ -203,14 +311,14 @@ int ssm_scan_sync_status(ssm_scan_t h, struct CUstream_st *stream) {
     cudaGetLastError();
     return SSM_ERR_CUDA;
   }
-  if (!h->ws) return SSM_OK;
+  if (!h->ctl) return SSM_OK;
   int status = 0;
-  if (cudaMemcpy(&status, h->ws, sizeof(int), cudaMemcpyDeviceToHost) !=
+  if (cudaMemcpy(&status, h->ctl, sizeof(int), cudaMemcpyDeviceToHost) !=
       cudaSuccess)
     return SSM_ERR_CUDA;
   if (status != ssm::kStatusOk) {
     const int zero = 0;
-    if (cudaMemcpy(h->ws, &zero, sizeof(int), cudaMemcpyHostToDevice) !=
+    if (cudaMemcpy(h->ctl, &zero, sizeof(int), cudaMemcpyHostToDevice) !=
         cudaSuccess)
       return SSM_ERR_CUDA;
     return SSM_ERR_TIMEOUT;
@@ -283,7 +391,7 @@ int ssm_scan_fwd(ssm_scan_t h, const void *x, const void *delta,
     if (!chunk_ok) return SSM_ERR_UNSUPPORTED;
     const int tb = h->time_blocks ? h->time_blocks
                                   : auto_time_blocks(p, h->sm_count);
-    rc = dispatch_chunked(p, dtype, tb, s);
+    rc = dispatch_chunked(h, p, dtype, tb, h->segments, s);
   } else if (dtype == SSM_F32) {
     rc = dispatch_sequential<float>(p, s);
   } else {
@@ -291,7 +399,7 @@ int ssm_scan_fwd(ssm_scan_t h, const void *x, const void *delta,
   }
   if (rc == SSM_OK) {
     h->last_variant = variant;
-    h->last_segments = 1;
+    if (variant != SSM_VARIANT_CHUNKED) h->last_segments = 1;
   }
   return rc;
 }
