@@ -10,7 +10,7 @@ import torch
 import oracle
 import selective_state_space_51_b200 as S
 from selective_state_space_51_b200 import workloads as W
-from gpu_helpers import assert_close, oracle_inputs, run, to_device
+from gpu_helpers import assert_close, oracle_inputs, rel_err, run, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -55,17 +55,25 @@ def test_split_parity(scan, idx, size, segments, tb):
 
 def test_split_slow_decay_replays_whole_piece(scan):
     """Tiny steps keep the carried-in state alive through a whole piece, so
-    the replay cannot stop early; the result must still match."""
+    the replay cannot stop early. Split and unsplit must agree at the float32
+    bar. Against the float64 oracle this input is the float32 worst case:
+    the same retention argument repeats for 4000 steps, so each step's
+    rounding of a ~ 1 - 6e-6 (about one unit in the last place) adds up
+    linearly, about 4000 x 6e-8. A looser, stated bound applies there."""
     wl = W.make(4, seqlen=4000, dim=16)
     wl.dev["delta"] = np.full_like(wl.dev["delta"], -12.0)   # delta ~ 6e-6
-    _set(scan, 4, 1)
+    t = to_device(wl)
     try:
-        y, h = run(scan, wl)
+        _set(scan, 4, 1)
+        y, h = run(scan, wl, t=t)
+        _set(scan, 1, 1)
+        y1, h1 = run(scan, wl, t=t)
     finally:
         _reset(scan)
+    assert_close(y, y1, wl.dtype, "y split vs unsplit")
+    assert_close(h, h1, wl.dtype, "h_last split vs unsplit")
     yo, ho = oracle.scan(**oracle_inputs(wl))
-    assert_close(y, yo, wl.dtype, "y")
-    assert_close(h, ho, wl.dtype, "h_last")
+    assert rel_err(y, yo) <= 1e-3 and rel_err(h, ho) <= 1e-3
 
 
 def test_split_matches_unsplit(scan):
