@@ -183,6 +183,44 @@ SSM_API int ssm_scan_last_variant(ssm_scan_t h, int *variant, int *segments);
  */
 SSM_API int ssm_scan_sync_status(ssm_scan_t h, struct CUstream_st *stream);
 
+/*
+ * ssm_scan_fwd_static_scratch: the forward pass of ssm_scan_fwd for callers
+ * that cannot allocate device memory. The source pages have no counterpart:
+ * this entry exists for users of the library, not for the method.
+ * Examples are a serving loop whose memory pool already holds the whole
+ * device, or a plug-in whose host fixes its memory budget up front. For
+ * such callers a cudaMalloc either fails or synchronizes the device at a bad
+ * moment, and ssm_scan_fwd may grow a workspace when it splits sequences.
+ *
+ * This call allocates nothing. The split-sequence workspace is a fixed 8 MiB
+ * device array inside the library, held by every GPU that loads the library
+ * until the process exits.
+ *   device   : CUDA device of every pointer; it must be current.
+ *   segments : pieces per sequence: 0 chooses by shape, 1 never splits, and
+ *              a larger value forces that count.
+ *   status   : NULL, or a device int the caller has zeroed. It is set to 1
+ *              if a bounded wait between thread blocks gave up, and the
+ *              outputs are then invalid.
+ *   the rest : as for ssm_scan_fwd. Additionally dstate is 4, 8 or 16,
+ *              dim * element size is a multiple of 16 bytes, and x, delta,
+ *              z, B, C are 16-byte aligned (else SSM_ERR_UNSUPPORTED or
+ *              SSM_ERR_ALIGN).
+ * A split workspace that does not fit in the array returns
+ * SSM_ERR_UNSUPPORTED before anything is launched. It needs
+ * batch x pieces x dim x dstate x 12 bytes plus flags.
+ * The first call on a device looks up the array's device address and clears
+ * it, which synchronizes that device: make that first call before any stream
+ * capture. Every call shares the one array, which keeps the last call's
+ * contents. Calls that overlap on the GPU race, so callers on several
+ * streams or host threads must serialize them.
+ */
+SSM_API int ssm_scan_fwd_static_scratch(
+    int device, const void *x, const void *delta, const float *A_log,
+    const void *B, const void *C, const float *D, const void *z,
+    const float *delta_bias, uint32_t flags, const float *h0, void *y,
+    float *h_last, ssm_scan_dims dims, int dtype, int segments, int *status,
+    struct CUstream_st *stream);
+
 /* ssm_scan_status_string: static English text for a status code. */
 SSM_API const char *ssm_scan_status_string(int status);
 

@@ -80,6 +80,10 @@ def library() -> ctypes.CDLL:
             lib.ssm_scan_last_variant.restype = i32
             lib.ssm_scan_sync_status.argtypes = [vp, vp]
             lib.ssm_scan_sync_status.restype = i32
+            lib.ssm_scan_fwd_static_scratch.argtypes = [
+                i32, vp, vp, vp, vp, vp, vp, vp, vp, u32, vp, vp, vp,
+                ssm_scan_dims, i32, i32, vp, vp]
+            lib.ssm_scan_fwd_static_scratch.restype = i32
             lib.ssm_scan_status_string.argtypes = [i32]
             lib.ssm_scan_status_string.restype = ctypes.c_char_p
             _lib = lib
@@ -155,6 +159,23 @@ def ssm_scan_fwd(h, x, delta, A_log, B, C, D, z, delta_bias, flags, h0, y,
                                 int(flags), _ptr(h0), _ptr(y), _ptr(h_last),
                                 dims, int(dtype), _stream(stream))
     return _check(rc, "ssm_scan_fwd") if check else rc
+
+
+def ssm_scan_fwd_static_scratch(device, x, delta, A_log, B, C, D, z,
+                                delta_bias, flags, h0, y, h_last, dims, dtype,
+                                segments=0, status=None, stream=None,
+                                check=True) -> int:
+    """Call ssm_scan_fwd_static_scratch (no handle, allocates nothing; see
+    include/ssm_scan.h). Returns the status; raises unless ``check`` is
+    False."""
+    if not isinstance(dims, ssm_scan_dims):
+        dims = ssm_scan_dims(*[int(d) for d in dims])
+    rc = library().ssm_scan_fwd_static_scratch(
+        int(device), _ptr(x), _ptr(delta), _ptr(A_log), _ptr(B), _ptr(C),
+        _ptr(D), _ptr(z), _ptr(delta_bias), int(flags), _ptr(h0), _ptr(y),
+        _ptr(h_last), dims, int(dtype), int(segments), _ptr(status),
+        _stream(stream))
+    return _check(rc, "ssm_scan_fwd_static_scratch") if check else rc
 
 
 class SelectiveScan:
