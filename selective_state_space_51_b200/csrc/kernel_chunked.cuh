@@ -348,24 +348,32 @@ scan_chunked_kernel(const ScanParams p) {
       };
 
       if constexpr (TB == 1) {
+        // Software pipeline: block jb's state updates run in the same
+        // iteration as block jb+1's step sizes (its softplus), so the two
+        // dependency chains overlap. Exchange slots alternate parity; every
+        // read of a slot precedes the __syncwarp that ends its iteration.
+        constexpr int NBW = TW / NG;  // NG-step blocks per window
+        float xm, zm;                 // this lane's step of the current block
+        produce(g, 0, xm, zm);
+        __syncwarp();
 #pragma unroll 2
-        for (int jb = 0; jb < TW / NG; ++jb) {
-          const int rm = jb * NG + g;
+        for (int jb = 0; jb < NBW; ++jb) {
           const int sp = jb & 1;
-          float xm, zm;
-          produce(rm, sp, xm, zm);
-          __syncwarp();
+          float4 dd[NG];
+#pragma unroll
+          for (int s = 0; s < NG; ++s) dd[s] = xch[sp * 32 + c * NG + s];
+          float xn = 0.0f, zn = 0.0f;
+          if (jb + 1 < NBW) produce((jb + 1) * NG + g, sp ^ 1, xn, zn);
           float ps[NG];
 #pragma unroll
           for (int s = 0; s < NG; ++s) {
-            const float4 dd = xch[sp * 32 + c * NG + s];
             float4 Bq, Cq;
             bc_row(jb * NG + s, Bq, Cq);
-            const float2 dA = make_float2(dd.x, dd.y);
+            const float2 dA = make_float2(dd[s].x, dd[s].y);
             const float2 a01 = ex2x2(mul2(dA, A01));
             const float2 a23 = ex2x2(mul2(dA, A23));
             if (MODE == kWalkMain) {
-              const float2 dx = make_float2(dd.z, dd.w);
+              const float2 dx = make_float2(dd[s].z, dd[s].w);
               h01 = fma2(a01, h01, mul2(dx, make_float2(Bq.x, Bq.y)));
               h23 = fma2(a23, h23, mul2(dx, make_float2(Bq.z, Bq.w)));
               if constexpr (SPLIT) {
@@ -381,7 +389,10 @@ scan_chunked_kernel(const ScanParams p) {
                      mul2(make_float2(Cq.x, Cq.y), h01));
             ps[s] = acc.x + acc.y;
           }
-          finish(rm, transpose_reduce<NG, TB>(ps, g), xm, zm);
+          finish(jb * NG + g, transpose_reduce<NG, TB>(ps, g), xm, zm);
+          xm = xn;
+          zm = zn;
+          __syncwarp();
         }
       } else {
         constexpr int M = TW / Cfg::SUBWIN;
