@@ -25,9 +25,8 @@
 // staged in shared memory with cp.async (double buffered, one window ahead;
 // rows padded so every lane access pattern is bank-conflict free); bfloat16
 // B and C are widened to float32 once per window. In each block of NG steps
-// lane g computes softplus for step g only and publishes (delta, delta,
-// delta*x, delta*x) in a per-warp exchange slot, so every (t, e) pays its
-// softplus once and the state arithmetic reads ready-made pairs. Readout
+// lane g computes softplus for step g only and publishes (delta, delta*x) in
+// a per-warp exchange slot, so every (t, e) pays its softplus once. Readout
 // partials over each lane's 4 states are combined over the NG lanes by a
 // transposing butterfly that leaves lane g holding the full y of the block's
 // step g; lane g adds D x, applies the SiLU gate and stores.
@@ -106,8 +105,8 @@ struct ChunkCfg {
   static constexpr int BCRAW_BYTES = ESZ == 2 ? round16(TW * N * 2) : 0;
   static constexpr int STAGE_BYTES =
       3 * RAW_BYTES + (ESZ == 2 ? 2 * BCRAW_BYTES : 2 * BF_BYTES);
-  // per warp: 2 parities x 32 slots x float4 (delta, delta, dx, dx)
-  static constexpr int XCH_BYTES = NW * 2 * 32 * 16;
+  // per warp: 2 parities x 32 slots x float2 (delta, delta * x)
+  static constexpr int XCH_BYTES = NW * 2 * 32 * 8;
   static constexpr int SMEM_BYTES =
       2 * STAGE_BYTES + (ESZ == 2 ? 2 * BF_BYTES : 0) + XCH_BYTES;
   static constexpr int SUBWIN = TB * K;  // steps per sub-window (TB > 1)
@@ -225,9 +224,9 @@ scan_chunked_kernel(const ScanParams p) {
   float2 P01 = make_float2(1.0f, 1.0f), P23 = P01;  // product of retentions
 
   float *const bf_conv = reinterpret_cast<float *>(smem + 2 * Cfg::STAGE_BYTES);
-  float4 *const xch = reinterpret_cast<float4 *>(
+  float2 *const xch = reinterpret_cast<float2 *>(
       smem + 2 * Cfg::STAGE_BYTES + (ESZ == 2 ? 2 * Cfg::BF_BYTES : 0)) +
-      warp * 64;
+      warp * 64;  // 2 parities x 32 slots of (delta, delta * x)
 
   // ---- issue the copies of window w into stage s
   auto stage = [&](int64_t w, int s) {
@@ -327,8 +326,7 @@ scan_chunked_kernel(const ScanParams p) {
         float dm = p.softplus ? softplus(v) : v;
         if (t0 + r >= t_end) dm = 0.0f;
         const float dxm = MODE == kWalkMain ? dm * xm : 0.0f;
-        xch[slot_par * 32 + (c * TB + q) * NG + g] =
-            make_float4(dm, dm, dxm, dxm);
+        xch[slot_par * 32 + (c * TB + q) * NG + g] = make_float2(dm, dxm);
       };
       auto finish = [&](int r, float yv, float xm, float zm) {
         const int64_t t = t0 + r;
@@ -359,7 +357,7 @@ scan_chunked_kernel(const ScanParams p) {
 #pragma unroll 2
         for (int jb = 0; jb < NBW; ++jb) {
           const int sp = jb & 1;
-          float4 dd[NG];
+          float2 dd[NG];
 #pragma unroll
           for (int s = 0; s < NG; ++s) dd[s] = xch[sp * 32 + c * NG + s];
           float xn = 0.0f, zn = 0.0f;
@@ -369,11 +367,11 @@ scan_chunked_kernel(const ScanParams p) {
           for (int s = 0; s < NG; ++s) {
             float4 Bq, Cq;
             bc_row(jb * NG + s, Bq, Cq);
-            const float2 dA = make_float2(dd[s].x, dd[s].y);
+            const float2 dA = make_float2(dd[s].x, dd[s].x);
             const float2 a01 = ex2x2(mul2(dA, A01));
             const float2 a23 = ex2x2(mul2(dA, A23));
             if (MODE == kWalkMain) {
-              const float2 dx = make_float2(dd[s].z, dd[s].w);
+              const float2 dx = make_float2(dd[s].y, dd[s].y);
               h01 = fma2(a01, h01, mul2(dx, make_float2(Bq.x, Bq.y)));
               h23 = fma2(a23, h23, mul2(dx, make_float2(Bq.z, Bq.w)));
               if constexpr (SPLIT) {
@@ -413,11 +411,11 @@ scan_chunked_kernel(const ScanParams p) {
 #pragma unroll
             for (int s = 0; s < NG; ++s) {
               const int j = jb * NG + s;
-              const float4 dd = xch[sp * 32 + (c * TB + q) * NG + s];
+              const float2 dd = xch[sp * 32 + (c * TB + q) * NG + s];
               float4 Bq, Cq;
               bc_row(r0 + j, Bq, Cq);
-              const float2 dA = make_float2(dd.x, dd.y);
-              const float2 dx = make_float2(dd.z, dd.w);
+              const float2 dA = make_float2(dd.x, dd.x);
+              const float2 dx = make_float2(dd.y, dd.y);
               a01[j] = ex2x2(mul2(dA, A01));
               a23[j] = ex2x2(mul2(dA, A23));
               w01[j] = mul2(dx, make_float2(Bq.x, Bq.y));
