@@ -77,6 +77,10 @@ class OracleLib:
         lib.ssm_oracle_scan.argtypes = [i64, i64, i64, i64, d, d, d, d, d, d,
                                         d, d, ctypes.c_int, d, d, d, d,
                                         ctypes.c_int]
+        lib.ssm_oracle_scan_ex.restype = ctypes.c_int
+        lib.ssm_oracle_scan_ex.argtypes = [i64, i64, i64, i64, d, d, d, d, d,
+                                           d, d, d, ctypes.c_int, ctypes.c_int,
+                                           d, d, d, d, ctypes.c_int]
         lib.ssm_oracle_step_size.restype = ctypes.c_double
         lib.ssm_oracle_step_size.argtypes = [ctypes.c_double, ctypes.c_double,
                                              ctypes.c_int]
@@ -98,7 +102,8 @@ class OracleLib:
         return float(self.lib.ssm_oracle_retention(step, a_log))
 
     def scan(self, x, delta, A_log, B, C, D=None, z=None, delta_bias=None,
-             delta_softplus=True, h0=None, return_states=False, nthreads=0):
+             delta_softplus=True, h0=None, return_states=False, nthreads=0,
+             write_zoh=False):
         xa = np.asarray(x)
         if xa.ndim != 3:
             raise ValueError("x must be [batch, seqlen, dim]")
@@ -117,12 +122,13 @@ class OracleLib:
         h_last = np.empty((b, E, N), dtype=np.float64)
         states = (np.empty((b, L, E, N), dtype=np.float64)
                   if return_states else None)
-        rc = self.lib.ssm_oracle_scan(b, L, E, N, _ptr(x64), _ptr(dt64),
-                                      _ptr(al64), _ptr(B64), _ptr(C64),
-                                      _ptr(D64), _ptr(z64), _ptr(bias64),
-                                      int(bool(delta_softplus)), _ptr(h064),
-                                      _ptr(y), _ptr(h_last), _ptr(states),
-                                      int(nthreads))
+        rc = self.lib.ssm_oracle_scan_ex(b, L, E, N, _ptr(x64), _ptr(dt64),
+                                         _ptr(al64), _ptr(B64), _ptr(C64),
+                                         _ptr(D64), _ptr(z64), _ptr(bias64),
+                                         int(bool(delta_softplus)),
+                                         int(bool(write_zoh)), _ptr(h064),
+                                         _ptr(y), _ptr(h_last), _ptr(states),
+                                         int(nthreads))
         if rc != 0:
             raise ValueError("oracle rejected its arguments (rc=%d)" % rc)
         if return_states:
@@ -154,8 +160,9 @@ def retention(step: float, a_log: float) -> float:
 
 
 def scan(x, delta, A_log, B, C, D=None, z=None, delta_bias=None,
-         delta_softplus=True, h0=None, return_states=False, nthreads=0):
-    """Run the float64 oracle.
+         delta_softplus=True, h0=None, return_states=False, nthreads=0,
+         write_zoh=False):
+    """Run the float64 oracle (write_zoh: exact zero-order-hold write).
 
     Shapes: x, delta, z: [b, L, E]; B, C: [b, L, N]; A_log: [E, N];
     D, delta_bias: [E]; h0: [b, E, N]. Returns (y [b,L,E], h_last [b,E,N])
@@ -163,11 +170,13 @@ def scan(x, delta, A_log, B, C, D=None, z=None, delta_bias=None,
     """
     return _load().scan(x, delta, A_log, B, C, D=D, z=z,
                         delta_bias=delta_bias, delta_softplus=delta_softplus,
-                        h0=h0, return_states=return_states, nthreads=nthreads)
+                        h0=h0, return_states=return_states, nthreads=nthreads,
+                        write_zoh=write_zoh)
 
 
 def scan_channels(channels, x, delta, A_log, B, C, D=None, z=None,
-                  delta_bias=None, delta_softplus=True, h0=None, nthreads=0):
+                  delta_bias=None, delta_softplus=True, h0=None, nthreads=0,
+                  write_zoh=False):
     """Oracle on a subset of channels (every batch, the full length).
 
     Channels never interact (A, D and the bias are per channel; B and C are
@@ -181,4 +190,5 @@ def scan_channels(channels, x, delta, A_log, B, C, D=None, z=None,
                 D=None if D is None else np.asarray(D)[ch], z=sel(z),
                 delta_bias=None if delta_bias is None
                 else np.asarray(delta_bias)[ch],
-                delta_softplus=delta_softplus, h0=h0s, nthreads=nthreads)
+                delta_softplus=delta_softplus, h0=h0s, nthreads=nthreads,
+                write_zoh=write_zoh)

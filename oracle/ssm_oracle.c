@@ -29,6 +29,12 @@
  *   - D == NULL means no direct path (the page's d=None), z == NULL means no
  *     gate, h0 == NULL means a zero incoming state;
  *   - the write term is evaluated as (delta * B) * x, the page's order;
+ *   - with write_zoh set, the write is the exact zero-order-hold input map
+ *     instead: Bbar = (delta A)^-1 (exp(delta A) - 1) delta B, which for a
+ *     diagonal A is expm1(delta A) / A * B per state ("Mamba: Linear-Time
+ *     Sequence Modeling with Selective State Spaces", nadeemcite summary,
+ *     section "Core Idea"; the abhik page's "There is a discretization detail
+ *     worth keeping explicit"), and delta * B when A = 0 (its limit);
  *   - the readout sums n in ascending order.
  *
  * Layouts (all contiguous, row-major, float64):
@@ -81,12 +87,41 @@ double ssm_oracle_retention(double step, double a_log)
  * Returns 0 on success, -1 on a bad argument (NULL required pointer or a
  * non-positive size). The output y must not alias any input.
  */
+int ssm_oracle_scan_ex(int64_t batch, int64_t seqlen, int64_t dim,
+                       int64_t dstate, const double *x, const double *delta,
+                       const double *A_log, const double *B, const double *C,
+                       const double *D, const double *z,
+                       const double *delta_bias, int delta_softplus,
+                       int write_zoh, const double *h0, double *y,
+                       double *h_last, double *states, int nthreads);
+
+/* Exact zero-order-hold input factor expm1(step A) / A (step when A = 0). */
+static double zoh_factor(double step, double A)
+{
+    if (A == 0.0)
+        return step;
+    return expm1(step * A) / A;
+}
+
 int ssm_oracle_scan(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
                     const double *x, const double *delta, const double *A_log,
                     const double *B, const double *C, const double *D,
                     const double *z, const double *delta_bias,
                     int delta_softplus, const double *h0,
                     double *y, double *h_last, double *states, int nthreads)
+{
+    return ssm_oracle_scan_ex(batch, seqlen, dim, dstate, x, delta, A_log, B,
+                              C, D, z, delta_bias, delta_softplus, 0, h0, y,
+                              h_last, states, nthreads);
+}
+
+int ssm_oracle_scan_ex(int64_t batch, int64_t seqlen, int64_t dim,
+                       int64_t dstate, const double *x, const double *delta,
+                       const double *A_log, const double *B, const double *C,
+                       const double *D, const double *z,
+                       const double *delta_bias, int delta_softplus,
+                       int write_zoh, const double *h0, double *y,
+                       double *h_last, double *states, int nthreads)
 {
     if (!x || !delta || !A_log || !B || !C || !y)
         return -1;
@@ -119,7 +154,8 @@ int ssm_oracle_scan(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
             const double xv = x[i];
             for (int64_t n = 0; n < dstate; ++n) {
                 const double retention = exp(step * A[n]);
-                const double write = step * B[r + n] * xv;
+                const double write =
+                    (write_zoh ? zoh_factor(step, A[n]) : step) * B[r + n] * xv;
                 h[n] = retention * h[n] + write;
             }
             if (states) {

@@ -435,6 +435,91 @@ def pin_degenerate(o):
     _close(yl, yu * 40.0, 0.0, 1e-14, "gate at z = 40")
 
 
+# ---------------------------------------------------------------- zero-order hold
+def pin_zoh_lti(o):
+    """Exact zero-order hold: constant step and B, C give a convolution with
+    Bbar_n = expm1(delta A_n) / A_n * B_n.
+
+    "Mamba: Linear-Time Sequence Modeling with Selective State Spaces"
+    (nadeemcite summary), section "Core Idea": Abar = exp(delta A) and
+    Bbar = (delta A)^-1 (exp(delta A) - I) delta B; with A diagonal, each
+    state's input map is expm1(delta A_n) / A_n * B_n. With those fixed, the
+    recurrence unrolls into y_k = sum_j K_j x_{k-j} (+ D x_k + the decayed h0),
+    K_j = sum_n C_n Abar_n^j Bbar_n.
+    """
+    rng = np.random.default_rng(23)
+    b, L, E, N = 1, 30, 2, 4
+    raw_e = rng.normal(0.0, 0.5, E)
+    Bc = rng.standard_normal((b, N))
+    Cc = rng.standard_normal((b, N))
+    case = dict(
+        x=rng.standard_normal((b, L, E)),
+        delta=np.broadcast_to(raw_e, (b, L, E)).copy(),
+        A_log=rng.normal(0.0, 0.6, (E, N)),
+        B=np.repeat(Bc[:, None, :], L, axis=1),
+        C=np.repeat(Cc[:, None, :], L, axis=1),
+        D=rng.standard_normal(E), h0=rng.standard_normal((b, E, N)))
+    y, h_last = o.scan(**case, delta_softplus=True, write_zoh=True)
+    step = _softplus(raw_e)
+    A = -np.exp(case["A_log"])
+    abar = np.exp(step[:, None] * A)
+    bbar = np.expm1(step[:, None] * A) / A * Bc[0][None, :]     # [E, N]
+    x, D, h0 = case["x"], case["D"], case["h0"]
+    for e in range(E):
+        powers = abar[e][None, :] ** np.arange(L + 1)[:, None]
+        K = (powers[:L] * Cc[0] * bbar[e]).sum(1)
+        scale = (powers[:L] * np.abs(Cc[0] * bbar[e])).sum(1)
+        for k in range(L):
+            want = np.dot(K[:k + 1], x[0, k::-1, e]) + D[e] * x[0, k, e] \
+                + np.dot(Cc[0] * powers[k + 1], h0[0, e])
+            tol = 1e-12 * (np.dot(scale[:k + 1], np.abs(x[0, k::-1, e]))
+                           + abs(D[e] * x[0, k, e])
+                           + np.dot(np.abs(Cc[0]) * powers[k + 1],
+                                    np.abs(h0[0, e]))) + 1e-300
+            assert abs(y[0, k, e] - want) <= tol, (e, k, y[0, k, e], want)
+
+
+def pin_zoh_fixed_point(o):
+    """Exact zero-order hold keeps the continuous system's equilibrium.
+
+    Same page and section: the discretization is exact for inputs held
+    constant over each step, so with constant x and B the state settles at
+    the fixed point of h' = A h + B x, that is h = -B x / A, whatever the
+    step size. (The delta * B write instead settles at delta B x / (1 - Abar),
+    which depends on delta.)
+    """
+    for raw in (-1.0, 0.8):
+        b, L, E, N = 1, 4000, 2, 3
+        rng = np.random.default_rng(29)
+        xv = rng.standard_normal(E)
+        Bv = rng.standard_normal(N)
+        case = dict(x=np.broadcast_to(xv, (b, L, E)).copy(),
+                    delta=np.full((b, L, E), raw),
+                    A_log=rng.normal(0.0, 0.3, (E, N)),
+                    B=np.broadcast_to(Bv, (b, L, N)).copy(),
+                    C=rng.standard_normal((b, L, N)))
+        _, h_last = o.scan(**case, delta_softplus=True, write_zoh=True)
+        A = -np.exp(case["A_log"])
+        want = -Bv[None, :] * xv[:, None] / A
+        _close(h_last[0], want, 1e-12, 1e-10, "ZOH fixed point")
+
+
+def pin_zoh_small_step(o):
+    """Zero-order hold tends to the delta * B write as delta -> 0.
+
+    expm1(delta A) / A = delta (1 + delta A / 2 + ...), so for delta ~ 1e-9
+    the two writes agree to about 1e-9 relative ("There is a discretization
+    detail worth keeping explicit" on the abhik page contrasts the two).
+    """
+    case = random_case(37, 2, 20, 3, 4, gate=False, bias=False)
+    case["delta"] = np.full_like(case["delta"], 1e-9)
+    yz, hz = o.scan(**case, delta_softplus=False, write_zoh=True)
+    yd, hd = o.scan(**case, delta_softplus=False, write_zoh=False)
+    _scaled_close(yz, yd, np.abs(yd) + 1e-6, 1e-7, "ZOH small step y")
+    _scaled_close(hz, hd, np.abs(hd) + 1e-9, 1e-7, "ZOH small step h")
+    assert not np.array_equal(yz, yd)
+
+
 # ---------------------------------------------------------------- softplus
 def pin_step_size(o):
     """delta = softplus(raw + bias), PyTorch default softplus.
@@ -465,4 +550,4 @@ def pin_step_size(o):
 ALL_PINS = (pin_associative_prefix, pin_lti_convolution, pin_forgetting,
             pin_freezing, pin_retention_bounds, pin_continuation,
             pin_decode_step, pin_linearity, pin_independence, pin_degenerate,
-            pin_step_size)
+            pin_step_size, pin_zoh_lti, pin_zoh_fixed_point, pin_zoh_small_step)

@@ -23,12 +23,17 @@ MUTANTS = [
     ("retention exp(step)*A", [("exp(step * A[n])", "(exp(step) * A[n])")]),
     ("retention without step", [("exp(step * A[n])", "exp(A[n])")]),
     ("D term dropped", [("out += D[c] * xv;", "out += 0.0 * xv;")]),
-    ("B and C transposed", [("step * B[r + n] * xv", "step * C[r + n] * xv"),
+    ("B and C transposed", [(": step) * B[r + n] * xv", ": step) * C[r + n] * xv"),
                             ("out += C[r + n] * h[n];",
                              "out += B[r + n] * h[n];")]),
     ("write uses previous B row",
-     [("step * B[r + n] * xv", "step * B[(t ? r - dstate : r) + n] * xv")]),
-    ("write without x", [("step * B[r + n] * xv", "step * B[r + n]")]),
+     [(": step) * B[r + n] * xv",
+       ": step) * B[(t ? r - dstate : r) + n] * xv")]),
+    ("write without x", [(": step) * B[r + n] * xv;", ": step) * B[r + n];")]),
+    ("zero-order hold without dividing by A",
+     [("return expm1(step * A) / A;", "return expm1(step * A);")]),
+    ("zero-order hold with exp instead of expm1",
+     [("return expm1(step * A) / A;", "return exp(step * A) / A;")]),
     ("x from the wrong channel",
      [("const double xv = x[i];",
        "const double xv = x[(b * seqlen + t) * dim + (dim - 1 - c)];")]),
