@@ -96,6 +96,47 @@ __device__ __forceinline__ float2 ex2x2(float2 v) {
   return make_float2(ex2(v.x), ex2(v.y));
 }
 
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n .reg .b64 ra, rb, rd;\n"
+      " mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+      " add.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// softplus of two values at once: the same formula as softplus(), with the
+// series and the bookkeeping on packed pairs.
+__device__ __forceinline__ float2 softplus2(float2 v) {
+  const float2 u = make_float2(ex2(-fabsf(v.x) * kLog2e),
+                               ex2(-fabsf(v.y) * kLog2e));
+  const float2 u2 = mul2(u, u);
+  const float2 u4 = mul2(u2, u2);
+  const float2 p0 = fma2(u, make_float2(-0.5f, -0.5f), make_float2(1.0f, 1.0f));
+  const float2 p1 = fma2(u, make_float2(-0.25f, -0.25f),
+                         make_float2(0.3333333333333333f, 0.3333333333333333f));
+  const float2 p2 = fma2(u, make_float2(-0.16666666666666666f,
+                                        -0.16666666666666666f),
+                         make_float2(0.2f, 0.2f));
+  const float2 p3 = fma2(u, make_float2(-0.125f, -0.125f),
+                         make_float2(0.14285714285714285f, 0.14285714285714285f));
+  const float2 s = mul2(fma2(u4, fma2(u2, p3, p2), fma2(u2, p1, p0)), u);
+  const float2 w = add2(u, make_float2(1.0f, 1.0f));
+  const float2 l = mul2(make_float2(lg2(w.x), lg2(w.y)), make_float2(kLn2, kLn2));
+  const float2 lp = make_float2(u.x < 0.125f ? s.x : l.x,
+                                u.y < 0.125f ? s.y : l.y);
+  const float2 r = add2(make_float2(fmaxf(v.x, 0.0f), fmaxf(v.y, 0.0f)), lp);
+  return make_float2(v.x > 20.0f ? v.x : r.x, v.y > 20.0f ? v.y : r.y);
+}
+
+// SiLU of two values at once.
+__device__ __forceinline__ float2 silu2(float2 z) {
+  const float2 e = mul2(z, make_float2(-kLog2e, -kLog2e));
+  const float2 d = add2(make_float2(ex2(e.x), ex2(e.y)), make_float2(1.0f, 1.0f));
+  return mul2(z, make_float2(rcp(d.x), rcp(d.y)));
+}
+
 template <typename T> struct Act;
 
 template <> struct Act<float> {

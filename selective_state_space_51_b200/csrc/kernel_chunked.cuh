@@ -105,8 +105,14 @@ struct ChunkCfg {
   static constexpr int BCRAW_BYTES = ESZ == 2 ? round16(TW * N * 2) : 0;
   static constexpr int STAGE_BYTES =
       3 * RAW_BYTES + (ESZ == 2 ? 2 * BCRAW_BYTES : 2 * BF_BYTES);
-  // per warp: 2 parities x 32 slots x float2 (delta, delta * x)
-  static constexpr int XCH_BYTES = NW * 2 * 32 * 8;
+  // time-block-1 blocks: BS = 2 NG steps, 2 per lane; exchange rows of the
+  // (delta, delta * x) pairs of a block, padded by 2 pairs per channel
+  static constexpr int BS = 2 * NG;
+  static constexpr int SLOT = BS + 2;
+  // per warp, 2 parities of: CW rows of SLOT pairs (time blocks 1) or 32
+  // single slots (time blocks > 1)
+  static constexpr int XCH_PER_WARP = TB == 1 ? CW * SLOT : 32;
+  static constexpr int XCH_BYTES = NW * 2 * XCH_PER_WARP * 8;
   static constexpr int SMEM_BYTES =
       2 * STAGE_BYTES + (ESZ == 2 ? 2 * BF_BYTES : 0) + XCH_BYTES;
   static constexpr int SUBWIN = TB * K;  // steps per sub-window (TB > 1)
@@ -120,7 +126,7 @@ struct ChunkCfg {
   static_assert(K % NG == 0, "a time block holds whole NG-step blocks");
   static_assert(RAW_P % 16 == 0 && RAW_PB % 16 == 0 && BF_PB % 16 == 0,
                 "cp.async destinations are 16-byte aligned");
-  static_assert((TB > 1 ? K / NG : TW / NG) % 2 == 0,
+  static_assert((TB > 1 ? K / NG : TW / (2 * NG)) % 2 == 0,
                 "exchange slots alternate parity from block to block");
 
   __device__ static __forceinline__ int raw_off(int r) {
@@ -153,6 +159,33 @@ __device__ __forceinline__ float transpose_reduce(const float (&p)[NG], int g) {
     const float s = lo ? k0 : k1;
     const float k = lo ? k1 : k0;
     return k + __shfl_xor_sync(FULL, s, TB);
+  }
+}
+
+// Sum over the NG lanes of a (c, q) pair of 2 NG per-step partials, leaving
+// lane g the totals of steps 2g and 2g+1 (a pair).
+template <int NG, int TB>
+__device__ __forceinline__ float2 transpose_reduce2(const float (&p)[2 * NG],
+                                                    int g) {
+  constexpr unsigned FULL = 0xffffffffu;
+  auto shfl2 = [](float2 v, int m) {
+    return make_float2(__shfl_xor_sync(FULL, v.x, m),
+                       __shfl_xor_sync(FULL, v.y, m));
+  };
+  if constexpr (NG == 1) {
+    return make_float2(p[0], p[1]);
+  } else if constexpr (NG == 2) {
+    const float2 P0 = make_float2(p[0], p[1]), P1 = make_float2(p[2], p[3]);
+    const bool lo = g & 1;
+    return add2(lo ? P1 : P0, shfl2(lo ? P0 : P1, TB));
+  } else {
+    const float2 P0 = make_float2(p[0], p[1]), P1 = make_float2(p[2], p[3]);
+    const float2 P2 = make_float2(p[4], p[5]), P3 = make_float2(p[6], p[7]);
+    const bool hi = g & 2;
+    const float2 k0 = add2(hi ? P2 : P0, shfl2(hi ? P0 : P2, 2 * TB));
+    const float2 k1 = add2(hi ? P3 : P1, shfl2(hi ? P1 : P3, 2 * TB));
+    const bool lo = g & 1;
+    return add2(lo ? k1 : k0, shfl2(lo ? k0 : k1, TB));
   }
 }
 
@@ -226,7 +259,7 @@ scan_chunked_kernel(const ScanParams p) {
   float *const bf_conv = reinterpret_cast<float *>(smem + 2 * Cfg::STAGE_BYTES);
   float2 *const xch = reinterpret_cast<float2 *>(
       smem + 2 * Cfg::STAGE_BYTES + (ESZ == 2 ? 2 * Cfg::BF_BYTES : 0)) +
-      warp * 64;  // 2 parities x 32 slots of (delta, delta * x)
+      warp * 2 * Cfg::XCH_PER_WARP;
 
   // ---- issue the copies of window w into stage s
   auto stage = [&](int64_t w, int s) {
@@ -346,27 +379,86 @@ scan_chunked_kernel(const ScanParams p) {
       };
 
       if constexpr (TB == 1) {
-        // Software pipeline: block jb's state updates run in the same
-        // iteration as block jb+1's step sizes (its softplus), so the two
-        // dependency chains overlap. Exchange slots alternate parity; every
-        // read of a slot precedes the __syncwarp that ends its iteration.
-        constexpr int NBW = TW / NG;  // NG-step blocks per window
-        float xm, zm;                 // this lane's step of the current block
-        produce(g, 0, xm, zm);
+        // Blocks of BS = 2 NG steps. Lane g owns steps 2g and 2g+1 of a block:
+        // it computes their step sizes (softplus on packed pairs) and
+        // publishes them in its channel's exchange row, and after the
+        // transposing reduction it finishes their outputs. Block jb's state
+        // updates share an iteration with block jb+1's step sizes, so the two
+        // dependency chains overlap. Exchange rows alternate parity; every
+        // read of a row precedes the __syncwarp that ends its iteration.
+        constexpr int BS = Cfg::BS, NBW = TW / BS, SLOT = Cfg::SLOT;
+        (void)SLOT;
+        const bool full = t0 + TW <= t_end;  // no step of the window is past
+        T *const yw = gy + ybase;
+
+        auto produce2 = [&](int jb, int par, float2 &x2, float2 &z2,
+                            float2 &dd0, float2 &dd1) {
+          const int r0 = jb * BS + 2 * g;
+          const int o0 = Cfg::raw_off(r0) + cl * ESZ;
+          const int o1 = Cfg::raw_off(r0 + 1) + cl * ESZ;
+          x2 = make_float2(Act<T>::load(reinterpret_cast<const T *>(sX + o0)),
+                           Act<T>::load(reinterpret_cast<const T *>(sX + o1)));
+          const float2 v2 = add2(
+              make_float2(Act<T>::load(reinterpret_cast<const T *>(sDL + o0)),
+                          Act<T>::load(reinterpret_cast<const T *>(sDL + o1))),
+              make_float2(bias, bias));
+          z2 = has_z ? make_float2(
+                           Act<T>::load(reinterpret_cast<const T *>(sZ + o0)),
+                           Act<T>::load(reinterpret_cast<const T *>(sZ + o1)))
+                     : make_float2(0.0f, 0.0f);
+          float2 d2 = p.softplus ? softplus2(v2) : v2;
+          if (!full) {
+            if (t0 + r0 >= t_end) d2.x = 0.0f;
+            if (t0 + r0 + 1 >= t_end) d2.y = 0.0f;
+          }
+          const float2 dx2 =
+              MODE == kWalkMain ? mul2(d2, x2) : make_float2(0.0f, 0.0f);
+          dd0 = make_float2(d2.x, dx2.x);
+          dd1 = make_float2(d2.y, dx2.y);
+          if constexpr (NG > 1)
+            *reinterpret_cast<float4 *>(xch + par * CW * SLOT + c * SLOT +
+                                        2 * g) =
+                make_float4(d2.x, dx2.x, d2.y, dx2.y);
+        };
+        auto finish2 = [&](int jb, float2 y2, float2 x2, float2 z2) {
+          const int r0 = jb * BS + 2 * g;
+          if (MODE == kWalkMain) y2 = fma2(make_float2(Dv, Dv), x2, y2);
+          if (has_z) y2 = mul2(y2, silu2(z2));
+          if (ch_ok) {
+            T *yp = yw + int64_t(r0) * E;
+            if (full || t0 + r0 < t_end) {
+              if (MODE == kWalkCorrect) y2.x += Act<T>::load(yp);
+              Act<T>::store(yp, y2.x);
+            }
+            if (full || t0 + r0 + 1 < t_end) {
+              if (MODE == kWalkCorrect) y2.y += Act<T>::load(yp + E);
+              Act<T>::store(yp + E, y2.y);
+            }
+          }
+        };
+
+        float2 x2, z2, e0, e1;
+        produce2(0, 0, x2, z2, e0, e1);
         __syncwarp();
 #pragma unroll 2
         for (int jb = 0; jb < NBW; ++jb) {
-          const int sp = jb & 1;
-          float2 dd[NG];
+          const int par = jb & 1;
+          float2 dd[BS];
+          if constexpr (NG > 1) {
 #pragma unroll
-          for (int s = 0; s < NG; ++s) dd[s] = xch[sp * 32 + c * NG + s];
-          float xn = 0.0f, zn = 0.0f;
-          if (jb + 1 < NBW) produce((jb + 1) * NG + g, sp ^ 1, xn, zn);
-          float ps[NG];
+            for (int s = 0; s < BS; ++s)
+              dd[s] = xch[par * CW * SLOT + c * SLOT + s];
+          } else {
+            dd[0] = e0;
+            dd[1] = e1;
+          }
+          float2 xn = make_float2(0.f, 0.f), zn = xn, n0 = xn, n1 = xn;
+          if (jb + 1 < NBW) produce2(jb + 1, par ^ 1, xn, zn, n0, n1);
+          float ps[BS];
 #pragma unroll
-          for (int s = 0; s < NG; ++s) {
+          for (int s = 0; s < BS; ++s) {
             float4 Bq, Cq;
-            bc_row(jb * NG + s, Bq, Cq);
+            bc_row(jb * BS + s, Bq, Cq);
             const float2 dA = make_float2(dd[s].x, dd[s].x);
             const float2 a01 = ex2x2(mul2(dA, A01));
             const float2 a23 = ex2x2(mul2(dA, A23));
@@ -387,9 +479,11 @@ scan_chunked_kernel(const ScanParams p) {
                      mul2(make_float2(Cq.x, Cq.y), h01));
             ps[s] = acc.x + acc.y;
           }
-          finish(jb * NG + g, transpose_reduce<NG, TB>(ps, g), xm, zm);
-          xm = xn;
-          zm = zn;
+          finish2(jb, transpose_reduce2<NG, TB>(ps, g), x2, z2);
+          x2 = xn;
+          z2 = zn;
+          e0 = n0;
+          e1 = n1;
           __syncwarp();
         }
       } else {

@@ -65,11 +65,11 @@ int dispatch_sequential(const ssm::ScanParams &p, cudaStream_t s) {
 using bf16 = __nv_bfloat16;
 //                          T      NG TB  K  TW NW pad  PB  BFPB
 using C16b1 = ssm::ChunkCfg<bf16,  4, 1, 4, 32, 4, 16,  0,  0>;
-using C16f1 = ssm::ChunkCfg<float, 4, 1, 4, 16, 4, 32,  0,  0>;
+using C16f1 = ssm::ChunkCfg<float, 4, 1, 4, 16, 4, 16,  0,  0>;
 using C16b2 = ssm::ChunkCfg<bf16,  4, 2, 8, 32, 4,  0, 16, 64>;
 using C16f2 = ssm::ChunkCfg<float, 4, 2, 8, 16, 4, 32, 16, 64>;
 using C8b1 = ssm::ChunkCfg<bf16,   2, 1, 2, 32, 4, 32,  0,  0>;
-using C8f1 = ssm::ChunkCfg<float,  2, 1, 2, 16, 4, 64,  0,  0>;
+using C8f1 = ssm::ChunkCfg<float,  2, 1, 2, 16, 4, 32,  0,  0>;
 using C8b2 = ssm::ChunkCfg<bf16,   2, 2, 8, 32, 4,  0, 16, 32>;
 using C8f2 = ssm::ChunkCfg<float,  2, 2, 8, 16, 4, 32, 64, 32>;
 using C4f1 = ssm::ChunkCfg<float,  1, 1, 1, 16, 4,  0,  0,  0>;

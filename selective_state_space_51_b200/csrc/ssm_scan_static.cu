@@ -47,9 +47,9 @@ bool aligned(const void *p, size_t a) {
 using bf16 = __nv_bfloat16;
 //                          T      NG TB  K  TW NW pad PB BFPB
 using S16b = ssm::ChunkCfg<bf16,  4, 1, 4, 32, 4, 16, 0, 0>;
-using S16f = ssm::ChunkCfg<float, 4, 1, 4, 16, 4, 32, 0, 0>;
+using S16f = ssm::ChunkCfg<float, 4, 1, 4, 16, 4, 16, 0, 0>;
 using S8b = ssm::ChunkCfg<bf16,   2, 1, 2, 32, 4, 32, 0, 0>;
-using S8f = ssm::ChunkCfg<float,  2, 1, 2, 16, 4, 64, 0, 0>;
+using S8f = ssm::ChunkCfg<float,  2, 1, 2, 16, 4, 32, 0, 0>;
 using S4f = ssm::ChunkCfg<float,  1, 1, 1, 16, 4,  0, 0, 0>;
 
 template <class Cfg>
