@@ -76,8 +76,18 @@ typedef struct {
 /* Activation dtype (x, delta, z, B, C and y). */
 enum { SSM_F32 = 0, SSM_BF16 = 1 };
 
-/* flags: delta = softplus(delta + delta_bias) when set, else delta + bias. */
-enum { SSM_DELTA_SOFTPLUS = 1u << 0 };
+/*
+ * flags:
+ *   SSM_DELTA_SOFTPLUS: delta = softplus(delta + delta_bias), else delta + bias.
+ *   SSM_WRITE_ZOH: the write is the exact zero-order-hold input map
+ *     Bbar = (delta A)^-1 (exp(delta A) - 1) delta B, i.e. per state
+ *     expm1(delta A[e,n]) / A[e,n] * B[t,n] * x[t,e] (delta * B * x when
+ *     A = 0), instead of the default delta * B * x ("Mamba: Linear-Time
+ *     Sequence Modeling with Selective State Spaces", nadeemcite summary,
+ *     section "Core Idea"; the abhik page, "There is a discretization detail
+ *     worth keeping explicit").
+ */
+enum { SSM_DELTA_SOFTPLUS = 1u << 0, SSM_WRITE_ZOH = 1u << 1 };
 
 /* Status codes. */
 enum {
@@ -124,7 +134,8 @@ SSM_API int ssm_scan_destroy(ssm_scan_t h);
  *   delta_bias : NULL means a zero bias.
  *   h0         : NULL means a zero incoming state.
  *   h_last     : NULL means the final state is not written.
- *   flags      : SSM_DELTA_SOFTPLUS or 0; other bits are SSM_ERR_INVALID.
+ *   flags      : SSM_DELTA_SOFTPLUS and/or SSM_WRITE_ZOH; other bits are
+ *                SSM_ERR_INVALID.
  *   dtype      : SSM_F32 or SSM_BF16 (activations and y).
  * y must not overlap any input. Pointers must be aligned to their element
  * size (SSM_ERR_ALIGN otherwise). Launches on `stream` and returns without

@@ -22,6 +22,7 @@ LIBRARY_PATH = os.path.join(_HERE, "libssmscan.so")
 SSM_F32 = 0
 SSM_BF16 = 1
 SSM_DELTA_SOFTPLUS = 1
+SSM_WRITE_ZOH = 2
 
 SSM_OK = 0
 SSM_ERR_INVALID = -1
@@ -218,7 +219,7 @@ class SelectiveScan:
 
     def __call__(self, x, delta, A_log, B, C, D=None, z=None, delta_bias=None,
                  delta_softplus=True, h0=None, y=None, h_last=None,
-                 return_last_state=True, stream=None):
+                 return_last_state=True, stream=None, write_zoh=False):
         import torch
         if x.dtype == torch.float32:
             dtype = SSM_F32
@@ -248,7 +249,8 @@ class SelectiveScan:
                                  device=self.device)
         if stream is None:
             stream = torch.cuda.current_stream(self.device)
-        flags = SSM_DELTA_SOFTPLUS if delta_softplus else 0
+        flags = (SSM_DELTA_SOFTPLUS if delta_softplus else 0) | \
+            (SSM_WRITE_ZOH if write_zoh else 0)
         ssm_scan_fwd(self.handle, x, delta, A_log, B, C, D, z, delta_bias,
                      flags, h0, y, h_last, (b, L, E, N), dtype, stream)
         return (y, h_last) if return_last_state else y

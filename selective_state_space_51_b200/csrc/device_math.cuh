@@ -137,6 +137,38 @@ __device__ __forceinline__ float2 silu2(float2 z) {
   return mul2(z, make_float2(rcp(d.x), rcp(d.y)));
 }
 
+// Exact zero-order-hold write factor expm1(z) / A, z = d A, for one state:
+// given zl = z log2(e) (so a = 2^zl) and invA = 1/A. For |z| < 1/8 it is
+// d phi(z) with phi(z) = (e^z - 1)/z = 1 + z/2 + z^2/6 + z^3/24 + z^4/120 +
+// z^5/720 (truncation below z^6/5040 < 8e-10 relative); otherwise (a - 1)/A,
+// where |a - 1| >= 1 - e^(-1/8) = 0.1175 keeps the subtraction accurate.
+__device__ __forceinline__ float zoh_factor(float d, float zl, float a,
+                                            float invA) {
+  const float z = zl * kLn2;
+  float ph = fmaf(z, 1.0f / 720.0f, 1.0f / 120.0f);
+  ph = fmaf(z, ph, 1.0f / 24.0f);
+  ph = fmaf(z, ph, 1.0f / 6.0f);
+  ph = fmaf(z, ph, 0.5f);
+  ph = fmaf(z, ph, 1.0f);
+  return fabsf(z) < 0.125f ? d * ph : (a - 1.0f) * invA;
+}
+
+// The same for two states at once (packed pairs).
+__device__ __forceinline__ float2 zoh_factor2(float2 d, float2 zl, float2 a,
+                                              float2 invA) {
+  const float2 z = mul2(zl, make_float2(kLn2, kLn2));
+  float2 ph = fma2(z, make_float2(1.0f / 720.0f, 1.0f / 720.0f),
+                   make_float2(1.0f / 120.0f, 1.0f / 120.0f));
+  ph = fma2(z, ph, make_float2(1.0f / 24.0f, 1.0f / 24.0f));
+  ph = fma2(z, ph, make_float2(1.0f / 6.0f, 1.0f / 6.0f));
+  ph = fma2(z, ph, make_float2(0.5f, 0.5f));
+  ph = fma2(z, ph, make_float2(1.0f, 1.0f));
+  const float2 sm = mul2(d, ph);
+  const float2 lg = mul2(add2(a, make_float2(-1.0f, -1.0f)), invA);
+  return make_float2(fabsf(z.x) < 0.125f ? sm.x : lg.x,
+                     fabsf(z.y) < 0.125f ? sm.y : lg.y);
+}
+
 template <typename T> struct Act;
 
 template <> struct Act<float> {

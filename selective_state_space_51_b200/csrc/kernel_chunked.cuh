@@ -191,9 +191,11 @@ __device__ __forceinline__ float2 transpose_reduce2(const float (&p)[2 * NG],
 
 enum { kWalkMain = 0, kWalkCorrect = 1 };
 
-template <class Cfg, bool SPLIT>
+template <class Cfg, bool SPLIT, bool ZOH = false>
 __global__ void __launch_bounds__(Cfg::THREADS)
 scan_chunked_kernel(const ScanParams p) {
+  static_assert(!ZOH || Cfg::TB == 1,
+                "the zero-order-hold write runs with one time block");
   using T = typename Cfg::T;
   constexpr int NG = Cfg::NG, TB = Cfg::TB, K = Cfg::K, TW = Cfg::TW;
   constexpr int CW = Cfg::CW, G = Cfg::G, N = Cfg::N, ESZ = Cfg::ESZ;
@@ -238,9 +240,14 @@ scan_chunked_kernel(const ScanParams p) {
   const bool has_z = gz != nullptr;
 
   float2 A01 = make_float2(0.0f, 0.0f), A23 = A01;  // A * log2(e)
+  float2 iA01 = A01, iA23 = A01;  // 1 / A (zero-order-hold write only)
   float2 h01 = A01, h23 = A01;  // state (TB == 1) or carry (TB > 1)
   if (ch_ok) {
     const float *al = p.A_log + e * N + 4 * g;
+    if constexpr (ZOH) {
+      iA01 = make_float2(-expf(-al[0]), -expf(-al[1]));
+      iA23 = make_float2(-expf(-al[2]), -expf(-al[3]));
+    }
     // clamp so that a zero step never meets -inf (0 * -inf = NaN)
     A01 = make_float2(fmaxf(-expf(al[0]) * kLog2e, -FLT_MAX),
                       fmaxf(-expf(al[1]) * kLog2e, -FLT_MAX));
@@ -411,8 +418,11 @@ scan_chunked_kernel(const ScanParams p) {
             if (t0 + r0 >= t_end) d2.x = 0.0f;
             if (t0 + r0 + 1 >= t_end) d2.y = 0.0f;
           }
-          const float2 dx2 =
-              MODE == kWalkMain ? mul2(d2, x2) : make_float2(0.0f, 0.0f);
+          // the second member is d x, or x itself for the zero-order-hold
+          // write (its factor depends on the state)
+          const float2 dx2 = MODE != kWalkMain ? make_float2(0.0f, 0.0f)
+                             : ZOH          ? x2
+                                            : mul2(d2, x2);
           dd0 = make_float2(d2.x, dx2.x);
           dd1 = make_float2(d2.y, dx2.y);
           if constexpr (NG > 1)
@@ -460,12 +470,19 @@ scan_chunked_kernel(const ScanParams p) {
             float4 Bq, Cq;
             bc_row(jb * BS + s, Bq, Cq);
             const float2 dA = make_float2(dd[s].x, dd[s].x);
-            const float2 a01 = ex2x2(mul2(dA, A01));
-            const float2 a23 = ex2x2(mul2(dA, A23));
+            const float2 zl01 = mul2(dA, A01), zl23 = mul2(dA, A23);
+            const float2 a01 = ex2x2(zl01);
+            const float2 a23 = ex2x2(zl23);
             if (MODE == kWalkMain) {
               const float2 dx = make_float2(dd[s].y, dd[s].y);
-              h01 = fma2(a01, h01, mul2(dx, make_float2(Bq.x, Bq.y)));
-              h23 = fma2(a23, h23, mul2(dx, make_float2(Bq.z, Bq.w)));
+              float2 w01 = mul2(dx, make_float2(Bq.x, Bq.y));
+              float2 w23 = mul2(dx, make_float2(Bq.z, Bq.w));
+              if constexpr (ZOH) {  // dx holds x: scale by expm1(dA)/A
+                w01 = mul2(w01, zoh_factor2(dA, zl01, a01, iA01));
+                w23 = mul2(w23, zoh_factor2(dA, zl23, a23, iA23));
+              }
+              h01 = fma2(a01, h01, w01);
+              h23 = fma2(a23, h23, w23);
               if constexpr (SPLIT) {
                 P01 = mul2(P01, a01);
                 P23 = mul2(P23, a23);

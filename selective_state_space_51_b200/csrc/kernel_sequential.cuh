@@ -7,7 +7,8 @@
 // Spaces", www.abhik.ai/papers/mamba, section "Original paper, equations and
 // runnable CPU code", rows 1, 2 and 5): delta = softplus(raw + bias);
 // a = exp(delta * A) with A = -exp(A_log); h = a * h + delta * B * x;
-// y = sum_n C * h + D * x, read after the update; y *= SiLU(z).
+// y = sum_n C * h + D * x, read after the update; y *= SiLU(z). With the
+// exact zero-order-hold flag the write is expm1(delta A) / A * B * x.
 #pragma once
 
 #include "device_math.cuh"
@@ -26,13 +27,16 @@ scan_sequential_kernel(const ScanParams p) {
   const int64_t L = p.seqlen, E = p.dim;
 
   float A2[NMAX];  // A * log2(e), so that a = 2^(delta * A2)
+  float iA[NMAX];  // 1 / A (exact zero-order-hold write only)
   float h[NMAX];
 #pragma unroll
   for (int n = 0; n < NMAX; ++n) {
     A2[n] = 0.0f;
+    iA[n] = 0.0f;
     h[n] = 0.0f;
     if (n < N) {
       A2[n] = -expf(p.A_log[e * N + n]) * kLog2e;
+      iA[n] = -expf(-p.A_log[e * N + n]);
       if (p.h0) h[n] = p.h0[(b * E + e) * N + n];
     }
   }
@@ -56,8 +60,10 @@ scan_sequential_kernel(const ScanParams p) {
 #pragma unroll
     for (int n = 0; n < NMAX; ++n) {
       if (n < N) {
-        const float a = ex2(step * A2[n]);
-        h[n] = fmaf(a, h[n], dx * Act<T>::load(Bm + r + n));
+        const float zl = step * A2[n];
+        const float a = ex2(zl);
+        const float wf = p.write_zoh ? zoh_factor(step, zl, a, iA[n]) * xv : dx;
+        h[n] = fmaf(a, h[n], wf * Act<T>::load(Bm + r + n));
         acc = fmaf(Act<T>::load(Cm + r + n), h[n], acc);
       }
     }

@@ -20,6 +20,7 @@ struct ScanParams {
   int64_t batch, seqlen, dim;
   int dstate;
   int softplus;              // apply softplus to delta + bias
+  int write_zoh;             // exact zero-order-hold write (see ssm_scan.h)
   // Split sequences (chunked variant): each sequence is cut into `segments`
   // pieces of seg_len steps (a multiple of the window), scanned concurrently
   // from a zero state and joined by a decoupled look-back over per-piece

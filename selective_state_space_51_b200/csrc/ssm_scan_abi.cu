@@ -128,13 +128,13 @@ int ensure_workspace(ssm_scan_s *h, ssm::ScanParams &p, int64_t tiles,
 // Pieces per sequence: enough that the blocks fill every resident slot once,
 // each piece at least 64 windows long (so the start-up replay after the
 // look-back stays a small fraction), and 1 when channels alone fill the GPU.
-template <class Cfg>
+template <class Cfg, bool ZOH>
 int64_t auto_segments(const ssm::ScanParams &p, int sm_count) {
   static int per_sm = 0;  // resident blocks per SM for this shape
   if (!per_sm) {
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-            &n, ssm::scan_chunked_kernel<Cfg, true>, Cfg::THREADS,
+            &n, ssm::scan_chunked_kernel<Cfg, true, ZOH>, Cfg::THREADS,
             Cfg::SMEM_BYTES) != cudaSuccess) {
       cudaGetLastError();
       n = 1;
@@ -151,10 +151,10 @@ int64_t auto_segments(const ssm::ScanParams &p, int sm_count) {
   return segs < 2 ? 1 : segs;
 }
 
-template <class Cfg, bool SPLIT>
+template <class Cfg, bool SPLIT, bool ZOH>
 int launch_kernel(const ssm::ScanParams &p, int64_t blocks, cudaStream_t s) {
   if (blocks > 0x7fffffff) return SSM_ERR_UNSUPPORTED;
-  auto kern = ssm::scan_chunked_kernel<Cfg, SPLIT>;
+  auto kern = ssm::scan_chunked_kernel<Cfg, SPLIT, ZOH>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Cfg::SMEM_BYTES) != cudaSuccess) {
     cudaGetLastError();
@@ -164,11 +164,12 @@ int launch_kernel(const ssm::ScanParams &p, int64_t blocks, cudaStream_t s) {
   return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
-template <class Cfg>
+template <class Cfg, bool ZOH = false>
 int launch_chunked(ssm_scan_s *h, ssm::ScanParams &p, int64_t segs_req,
                    cudaStream_t s) {
   const int64_t tiles = (p.dim + Cfg::G - 1) / Cfg::G;
-  int64_t segs = segs_req > 0 ? segs_req : auto_segments<Cfg>(p, h->sm_count);
+  int64_t segs =
+      segs_req > 0 ? segs_req : auto_segments<Cfg, ZOH>(p, h->sm_count);
   int64_t seg_len = p.seqlen;
   if (segs > 1) {
     const int64_t wins = (p.seqlen + Cfg::TW - 1) / Cfg::TW;
@@ -179,10 +180,10 @@ int launch_chunked(ssm_scan_s *h, ssm::ScanParams &p, int64_t segs_req,
   p.segments = int(segs);
   p.seg_len = seg_len;
   h->last_segments = int(segs);
-  if (segs <= 1) return launch_kernel<Cfg, false>(p, p.batch * tiles, s);
+  if (segs <= 1) return launch_kernel<Cfg, false, ZOH>(p, p.batch * tiles, s);
   const int rc = ensure_workspace(h, p, tiles, segs, s);
   if (rc != SSM_OK) return rc;
-  return launch_kernel<Cfg, true>(p, segs * p.batch * tiles, s);
+  return launch_kernel<Cfg, true, ZOH>(p, segs * p.batch * tiles, s);
 }
 
 // Whether the chunked variant can run these arguments: N of 4, 8 or 16, whole
@@ -206,6 +207,9 @@ int auto_time_blocks(const ssm::ScanParams &, int) { return 1; }
 template <class Cf1, class Cf2>
 int pick(ssm_scan_s *h, ssm::ScanParams &p, int tb, int64_t segs,
          cudaStream_t s) {
+  if (p.write_zoh)  // the zero-order-hold write runs with one time block
+    return tb == 1 ? launch_chunked<Cf1, true>(h, p, segs, s)
+                   : SSM_ERR_UNSUPPORTED;
   if (tb == 1) return launch_chunked<Cf1>(h, p, segs, s);
   if (tb == 2) return launch_chunked<Cf2>(h, p, segs, s);
   return SSM_ERR_UNSUPPORTED;
@@ -349,7 +353,8 @@ int ssm_scan_fwd(ssm_scan_t h, const void *x, const void *delta,
   if (!h || !x || !delta || !A_log || !B || !C || !y) return SSM_ERR_INVALID;
   if (dims.batch <= 0 || dims.seqlen <= 0 || dims.dim <= 0 || dims.dstate <= 0)
     return SSM_ERR_INVALID;
-  if (flags & ~uint32_t(SSM_DELTA_SOFTPLUS)) return SSM_ERR_INVALID;
+  if (flags & ~uint32_t(SSM_DELTA_SOFTPLUS | SSM_WRITE_ZOH))
+    return SSM_ERR_INVALID;
   if (dtype != SSM_F32 && dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
   if (dims.dstate > 64) return SSM_ERR_UNSUPPORTED;
   int64_t rows = 0, acts = 0, bc = 0, st = 0;
@@ -379,6 +384,7 @@ int ssm_scan_fwd(ssm_scan_t h, const void *x, const void *delta,
   p.batch = dims.batch; p.seqlen = dims.seqlen; p.dim = dims.dim;
   p.dstate = (int)dims.dstate;
   p.softplus = (flags & SSM_DELTA_SOFTPLUS) ? 1 : 0;
+  p.write_zoh = (flags & SSM_WRITE_ZOH) ? 1 : 0;
   p.segments = 1;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 

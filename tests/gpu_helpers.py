@@ -25,13 +25,13 @@ def to_device(wl, device="cuda"):
     return out
 
 
-def run(scan, wl, t=None, softplus=None, with_h_last=True):
+def run(scan, wl, t=None, softplus=None, with_h_last=True, write_zoh=False):
     t = to_device(wl) if t is None else t
     y, h_last = scan(t["x"], t["delta"], t["A_log"], t["B"], t["C"],
                      D=t["D"], z=t["z"], delta_bias=t["delta_bias"],
                      delta_softplus=wl.delta_softplus if softplus is None
                      else softplus,
-                     h0=t["h0"], return_last_state=True)
+                     h0=t["h0"], return_last_state=True, write_zoh=write_zoh)
     torch.cuda.synchronize()
     assert scan.sync_status() == S.SSM_OK
     yf = y.float().cpu().numpy().astype(np.float64)
