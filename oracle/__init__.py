@@ -81,6 +81,10 @@ class OracleLib:
         lib.ssm_oracle_scan_ex.argtypes = [i64, i64, i64, i64, d, d, d, d, d,
                                            d, d, d, ctypes.c_int, ctypes.c_int,
                                            d, d, d, d, ctypes.c_int]
+        lib.ssm_oracle_step.restype = ctypes.c_int
+        lib.ssm_oracle_step.argtypes = [i64, i64, i64, i64, d, d, d, d, d, d,
+                                        ctypes.c_int, ctypes.c_int, d, d, d, d,
+                                        d, d, d]
         lib.ssm_oracle_step_size.restype = ctypes.c_double
         lib.ssm_oracle_step_size.argtypes = [ctypes.c_double, ctypes.c_double,
                                              ctypes.c_int]
@@ -136,6 +140,34 @@ class OracleLib:
         return y, h_last
 
 
+    def step(self, x_new, delta, A_log, B, C, state, conv_state=None,
+             conv_weight=None, conv_bias=None, D=None, z=None,
+             delta_bias=None, delta_softplus=True, write_zoh=False):
+        """One decode step. Returns (y [b, E], new state [b, E, N], new
+        conv_state [b, E, K] or None); the inputs are not modified."""
+        xa = np.asarray(x_new)
+        b, E = xa.shape
+        N = np.asarray(A_log).shape[-1]
+        K = 0 if conv_state is None else np.asarray(conv_state).shape[-1]
+        st = _f64(state, (b, E, N), "state").copy()
+        cs = None if conv_state is None else \
+            _f64(conv_state, (b, E, K), "conv_state").copy()
+        cw = _f64(conv_weight, (E, K), "conv_weight") if K else None
+        cb = _f64(conv_bias, (E,), "conv_bias") if K else None
+        y = np.empty((b, E), dtype=np.float64)
+        rc = self.lib.ssm_oracle_step(
+            b, E, N, K, _ptr(_f64(xa, (b, E), "x_new")), _ptr(cs), _ptr(cw),
+            _ptr(cb), _ptr(_f64(delta, (b, E), "delta")),
+            _ptr(_f64(delta_bias, (E,), "delta_bias")),
+            int(bool(delta_softplus)), int(bool(write_zoh)),
+            _ptr(_f64(A_log, (E, N), "A_log")), _ptr(_f64(B, (b, N), "B")),
+            _ptr(_f64(C, (b, N), "C")), _ptr(_f64(D, (E,), "D")),
+            _ptr(_f64(z, (b, E), "z")), _ptr(st), _ptr(y))
+        if rc != 0:
+            raise ValueError("oracle rejected its arguments (rc=%d)" % rc)
+        return y, st, cs
+
+
 def _load() -> OracleLib:
     global _default
     with _lock:
@@ -172,6 +204,16 @@ def scan(x, delta, A_log, B, C, D=None, z=None, delta_bias=None,
                         delta_bias=delta_bias, delta_softplus=delta_softplus,
                         h0=h0, return_states=return_states, nthreads=nthreads,
                         write_zoh=write_zoh)
+
+
+def step(x_new, delta, A_log, B, C, state, conv_state=None, conv_weight=None,
+         conv_bias=None, D=None, z=None, delta_bias=None, delta_softplus=True,
+         write_zoh=False):
+    """One batched decode step (see OracleLib.step)."""
+    return _load().step(x_new, delta, A_log, B, C, state,
+                        conv_state=conv_state, conv_weight=conv_weight,
+                        conv_bias=conv_bias, D=D, z=z, delta_bias=delta_bias,
+                        delta_softplus=delta_softplus, write_zoh=write_zoh)
 
 
 def scan_channels(channels, x, delta, A_log, B, C, D=None, z=None,

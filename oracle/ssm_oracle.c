@@ -190,3 +190,73 @@ int ssm_oracle_max_threads(void)
     return 1;
 #endif
 }
+
+/*
+ * One decode step for a batch of sequences, float64 ("Mamba: Linear-Time
+ * Sequence Modeling with Selective State Spaces", www.abhik.ai/papers/mamba,
+ * section "Original paper, equations and runnable CPU code", row "6. Carry
+ * both buffers to the next token", and row "4. Add causal local context
+ * before selecting coefficients"):
+ *   conv_state <- shift left by one, append x_new     (K samples, the last
+ *                                                      one is the newest)
+ *   x  = SiLU(sum_k conv_state[k] * w[c, k] + conv_bias[c])
+ *   delta = softplus(raw + delta_bias)  (or raw + bias), A = -exp(A_log)
+ *   state <- exp(delta A) * state + delta * B * x  (or the zero-order-hold
+ *            write, as in ssm_oracle_scan_ex)
+ *   y  = sum_n C[n] * state[n] + D[c] * x, then y *= SiLU(z)
+ * With conv_state == NULL the convolution is skipped and x = x_new.
+ * Layouts: x_new, delta, z, y: [batch, dim]; conv_state: [batch, dim, K];
+ * conv_weight: [dim, K]; conv_bias, D, delta_bias: [dim]; B, C: [batch,
+ * dstate]; A_log: [dim, dstate]; state: [batch, dim, dstate]. conv_state and
+ * state are updated in place. Returns 0, or -1 on a bad argument.
+ */
+int ssm_oracle_step(int64_t batch, int64_t dim, int64_t dstate, int64_t width,
+                    const double *x_new, double *conv_state,
+                    const double *conv_weight, const double *conv_bias,
+                    const double *delta, const double *delta_bias,
+                    int delta_softplus, int write_zoh, const double *A_log,
+                    const double *B, const double *C, const double *D,
+                    const double *z, double *state, double *y)
+{
+    if (!x_new || !delta || !A_log || !B || !C || !state || !y)
+        return -1;
+    if (batch <= 0 || dim <= 0 || dstate <= 0)
+        return -1;
+    if (conv_state && (!conv_weight || width <= 0))
+        return -1;
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t c = 0; c < dim; ++c) {
+            const int64_t i = b * dim + c;
+            double xv = x_new[i];
+            if (conv_state) {
+                double *buf = conv_state + i * width;
+                for (int64_t k = 0; k + 1 < width; ++k)
+                    buf[k] = buf[k + 1];
+                buf[width - 1] = x_new[i];
+                double acc = conv_bias ? conv_bias[c] : 0.0;
+                for (int64_t k = 0; k < width; ++k)
+                    acc += buf[k] * conv_weight[c * width + k];
+                xv = silu(acc);
+            }
+            const double v = delta[i] + (delta_bias ? delta_bias[c] : 0.0);
+            const double step = delta_softplus ? softplus_default(v) : v;
+            double out = 0.0;
+            for (int64_t n = 0; n < dstate; ++n) {
+                const double A = -exp(A_log[c * dstate + n]);
+                const double retention = exp(step * A);
+                const double write =
+                    (write_zoh ? zoh_factor(step, A) : step) * B[b * dstate + n]
+                    * xv;
+                double *h = state + i * dstate + n;
+                *h = retention * *h + write;
+                out += C[b * dstate + n] * *h;
+            }
+            if (D)
+                out += D[c] * xv;
+            if (z)
+                out *= silu(z[i]);
+            y[i] = out;
+        }
+    }
+    return 0;
+}

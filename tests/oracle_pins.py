@@ -520,6 +520,102 @@ def pin_zoh_small_step(o):
     assert not np.array_equal(yz, yd)
 
 
+# ---------------------------------------------------------------- decode step
+def pin_step_matches_scan(o):
+    """Decoding one token at a time reproduces the full scan, bitwise.
+
+    [abhik] "6. Carry both buffers to the next token" updates the [b, E, N]
+    state exactly as the scan does for one step, and "The selective operator
+    is one part of the Mamba block" asks the full sequence and token-by-token
+    results to agree. Checked without the convolution, for both writes.
+    """
+    for zoh in (False, True):
+        case = random_case(43, 2, 17, 3, 4)
+        y, h_last = o.scan(**case, delta_softplus=True, write_zoh=zoh)
+        state = case["h0"].copy()
+        for t in range(17):
+            yt, state, _ = o.step(case["x"][:, t], case["delta"][:, t],
+                                  case["A_log"], case["B"][:, t],
+                                  case["C"][:, t], state, D=case["D"],
+                                  z=case["z"][:, t],
+                                  delta_bias=case["delta_bias"],
+                                  delta_softplus=True, write_zoh=zoh)
+            assert np.array_equal(yt, y[:, t]), (zoh, t)
+        assert np.array_equal(state, h_last), zoh
+
+
+def pin_step_causal_convolution(o):
+    """The step's convolution is the causal depthwise convolution + SiLU.
+
+    [abhik] "4. Add causal local context before selecting coefficients":
+    x_t = SiLU(b + sum_k q_k v_{t-K+1+k}) with zeros before the start, and
+    "6. Carry both buffers" keeps K samples including the newest. With B = 0,
+    D = 1 and no gate the step outputs that x, which must equal numpy's full
+    convolution with the reversed kernel, cut to the causal part.
+    """
+    rng = np.random.default_rng(47)
+    b, E, N, K, L = 2, 3, 2, 4, 12
+    v = rng.standard_normal((b, L, E))
+    w = rng.standard_normal((E, K))
+    bias = rng.standard_normal(E)
+    conv = np.zeros((b, E, K))
+    state = np.zeros((b, E, N))
+    for t in range(L):
+        yt, state, conv = o.step(v[:, t], np.zeros((b, E)),
+                                 np.zeros((E, N)), np.zeros((b, N)),
+                                 rng.standard_normal((b, N)), state,
+                                 conv_state=conv, conv_weight=w,
+                                 conv_bias=bias, D=np.ones(E),
+                                 delta_softplus=False)
+        for bb in range(b):
+            for e in range(E):
+                full = np.convolve(v[bb, :t + 1, e], w[e, ::-1])[:t + 1]
+                pre = full[t] + bias[e]
+                want = pre / (1.0 + math.exp(-pre))
+                assert abs(yt[bb, e] - want) <= 1e-13 * (1 + abs(want)), \
+                    (t, bb, e, yt[bb, e], want)
+        # the buffer holds the last K inputs, oldest first, zeros before
+        for k in range(K):
+            src = t - (K - 1) + k
+            want = v[:, src] if src >= 0 else np.zeros((b, E))
+            assert np.array_equal(conv[:, :, k], want), (t, k)
+
+
+def pin_step_conv_feeds_scan(o):
+    """With the convolution on, decoding equals the scan of the convolved
+    input.
+
+    [abhik] "5. Put the selective operator inside the complete mixer": the
+    scan runs on x = SiLU(CausalDWConv(v)), with D x and the gate on that x;
+    "6. Carry both buffers" decodes the same thing token by token. The
+    convolved input is formed here with numpy's convolution, then the scan
+    oracle (pinned above) gives the expected outputs and final state.
+    """
+    rng = np.random.default_rng(53)
+    b, E, N, K, L = 2, 3, 4, 3, 15
+    case = random_case(59, b, L, E, N)
+    v = rng.standard_normal((b, L, E))
+    w = rng.standard_normal((E, K))
+    cbias = rng.standard_normal(E)
+    xc = np.empty_like(v)
+    for bb in range(b):
+        for e in range(E):
+            pre = np.convolve(v[bb, :, e], w[e, ::-1])[:L] + cbias[e]
+            xc[bb, :, e] = pre / (1.0 + np.exp(-pre))
+    y, h_last = o.scan(**dict(case, x=xc), delta_softplus=True)
+    state = case["h0"].copy()
+    conv = np.zeros((b, E, K))
+    for t in range(L):
+        yt, state, conv = o.step(v[:, t], case["delta"][:, t], case["A_log"],
+                                 case["B"][:, t], case["C"][:, t], state,
+                                 conv_state=conv, conv_weight=w,
+                                 conv_bias=cbias, D=case["D"],
+                                 z=case["z"][:, t],
+                                 delta_bias=case["delta_bias"])
+        _close(yt, y[:, t], 1e-12, 1e-10, "decode with conv, step %d" % t)
+    _close(state, h_last, 1e-12, 1e-10, "decode with conv, state")
+
+
 # ---------------------------------------------------------------- softplus
 def pin_step_size(o):
     """delta = softplus(raw + bias), PyTorch default softplus.
@@ -550,4 +646,6 @@ def pin_step_size(o):
 ALL_PINS = (pin_associative_prefix, pin_lti_convolution, pin_forgetting,
             pin_freezing, pin_retention_bounds, pin_continuation,
             pin_decode_step, pin_linearity, pin_independence, pin_degenerate,
-            pin_step_size, pin_zoh_lti, pin_zoh_fixed_point, pin_zoh_small_step)
+            pin_step_size, pin_zoh_lti, pin_zoh_fixed_point, pin_zoh_small_step,
+            pin_step_matches_scan, pin_step_causal_convolution,
+            pin_step_conv_feeds_scan)

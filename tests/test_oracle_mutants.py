@@ -30,6 +30,13 @@ MUTANTS = [
      [(": step) * B[r + n] * xv",
        ": step) * B[(t ? r - dstate : r) + n] * xv")]),
     ("write without x", [(": step) * B[r + n] * xv;", ": step) * B[r + n];")]),
+    ("decode buffer shifted the wrong way",
+     [("buf[k] = buf[k + 1];", "buf[k + 1] = buf[k];")]),
+    ("decode convolution without its bias",
+     [("double acc = conv_bias ? conv_bias[c] : 0.0;", "double acc = 0.0;")]),
+    ("decode write uses the raw input, not the convolved one",
+     [("* B[b * dstate + n]\n                    * xv;",
+       "* B[b * dstate + n]\n                    * x_new[i];")]),
     ("zero-order hold without dividing by A",
      [("return expm1(step * A) / A;", "return expm1(step * A);")]),
     ("zero-order hold with exp instead of expm1",
