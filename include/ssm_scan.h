@@ -195,6 +195,39 @@ SSM_API int ssm_scan_last_variant(ssm_scan_t h, int *variant, int *segments);
 SSM_API int ssm_scan_sync_status(ssm_scan_t h, struct CUstream_st *stream);
 
 /*
+ * ssm_scan_step: one decode step for `dims.batch` sequences at once, updating
+ * the convolution buffer and the state in place ("Mamba: Linear-Time Sequence
+ * Modeling with Selective State Spaces", www.abhik.ai/papers/mamba, section
+ * "Original paper, equations and runnable CPU code", row "6. Carry both
+ * buffers to the next token", with the causal convolution of row "4. Add
+ * causal local context before selecting coefficients"):
+ *     conv_state <- shift left by one sample, append x_new
+ *     x     = SiLU(sum_k conv_state[k] * conv_weight[e, k] + conv_bias[e])
+ *     delta = softplus(delta_raw + delta_bias)   (SSM_DELTA_SOFTPLUS)
+ *     state <- exp(delta A) * state + delta * B * x  (or the SSM_WRITE_ZOH write)
+ *     y     = (sum_n C[n] * state[n] + D[e] * x) * SiLU(z)
+ * Layouts (dense, row-major): x_new, delta, z, y: [batch, dim] activation
+ * dtype; conv_state: [batch, dim, conv_width] activation dtype (oldest sample
+ * first); conv_weight: [dim, conv_width] float32; conv_bias, D, delta_bias:
+ * [dim] float32; A_log: [dim, dstate] float32; B, C: [batch, dstate]
+ * activation dtype; state: [batch, dim, dstate] float32.
+ *   conv_state : NULL skips the convolution (x = x_new); otherwise
+ *                conv_weight is required and 1 <= conv_width <= 8.
+ *   conv_bias, D, z, delta_bias : NULL means absent (0 / no gate).
+ *   dims.seqlen must be 1; dims.dstate is 1..64.
+ * state, conv_state and y must not overlap each other or any input. Launches
+ * on `stream` without waiting. Errors as for ssm_scan_fwd.
+ */
+SSM_API int ssm_scan_step(ssm_scan_t h, const void *x_new, void *conv_state,
+                          const float *conv_weight, const float *conv_bias,
+                          int conv_width, const void *delta,
+                          const float *delta_bias, const float *A_log,
+                          const void *B, const void *C, const float *D,
+                          const void *z, uint32_t flags, float *state, void *y,
+                          ssm_scan_dims dims, int dtype,
+                          struct CUstream_st *stream);
+
+/*
  * ssm_scan_fwd_static_scratch: the forward pass of ssm_scan_fwd for callers
  * that cannot allocate device memory. The source pages have no counterpart:
  * this entry exists for users of the library, not for the method.

@@ -81,6 +81,10 @@ def library() -> ctypes.CDLL:
             lib.ssm_scan_last_variant.restype = i32
             lib.ssm_scan_sync_status.argtypes = [vp, vp]
             lib.ssm_scan_sync_status.restype = i32
+            lib.ssm_scan_step.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, vp,
+                                          vp, vp, vp, vp, u32, vp, vp,
+                                          ssm_scan_dims, i32, vp]
+            lib.ssm_scan_step.restype = i32
             lib.ssm_scan_fwd_static_scratch.argtypes = [
                 i32, vp, vp, vp, vp, vp, vp, vp, vp, u32, vp, vp, vp,
                 ssm_scan_dims, i32, i32, vp, vp]
@@ -162,6 +166,21 @@ def ssm_scan_fwd(h, x, delta, A_log, B, C, D, z, delta_bias, flags, h0, y,
     return _check(rc, "ssm_scan_fwd") if check else rc
 
 
+def ssm_scan_step(h, x_new, conv_state, conv_weight, conv_bias, conv_width,
+                  delta, delta_bias, A_log, B, C, D, z, flags, state, y, dims,
+                  dtype, stream=None, check=True) -> int:
+    """Call ssm_scan_step (one batched decode step; see include/ssm_scan.h).
+    dims is (batch, 1, dim, dstate)."""
+    if not isinstance(dims, ssm_scan_dims):
+        dims = ssm_scan_dims(*[int(d) for d in dims])
+    rc = library().ssm_scan_step(
+        h, _ptr(x_new), _ptr(conv_state), _ptr(conv_weight), _ptr(conv_bias),
+        int(conv_width), _ptr(delta), _ptr(delta_bias), _ptr(A_log), _ptr(B),
+        _ptr(C), _ptr(D), _ptr(z), int(flags), _ptr(state), _ptr(y), dims,
+        int(dtype), _stream(stream))
+    return _check(rc, "ssm_scan_step") if check else rc
+
+
 def ssm_scan_fwd_static_scratch(device, x, delta, A_log, B, C, D, z,
                                 delta_bias, flags, h0, y, h_last, dims, dtype,
                                 segments=0, status=None, stream=None,
@@ -216,6 +235,28 @@ class SelectiveScan:
         if stream is None:
             stream = torch.cuda.current_stream(self.device)
         return ssm_scan_sync_status(self.handle, stream)
+
+    def step(self, x_new, delta, A_log, B, C, state, conv_state=None,
+             conv_weight=None, conv_bias=None, D=None, z=None,
+             delta_bias=None, delta_softplus=True, write_zoh=False, y=None,
+             stream=None):
+        """One decode step; state (and conv_state) are updated in place.
+        Returns y [batch, dim]."""
+        import torch
+        dtype = SSM_F32 if x_new.dtype == torch.float32 else SSM_BF16
+        b, E = x_new.shape
+        N = A_log.shape[-1]
+        K = 0 if conv_state is None else conv_state.shape[-1]
+        if y is None:
+            y = torch.empty_like(x_new)
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device)
+        flags = (SSM_DELTA_SOFTPLUS if delta_softplus else 0) | \
+            (SSM_WRITE_ZOH if write_zoh else 0)
+        ssm_scan_step(self.handle, x_new, conv_state, conv_weight, conv_bias,
+                      K, delta, delta_bias, A_log, B, C, D, z, flags, state, y,
+                      (b, 1, E, N), dtype, stream)
+        return y
 
     def __call__(self, x, delta, A_log, B, C, D=None, z=None, delta_bias=None,
                  delta_softplus=True, h0=None, y=None, h_last=None,

@@ -9,6 +9,7 @@
 #include "../../include/ssm_scan.h"
 #include "kernel_chunked.cuh"
 #include "kernel_sequential.cuh"
+#include "kernel_step.cuh"
 
 constexpr unsigned kDefaultSpinLimit = 1000u * 1000u;  // ~1 s of polls
 
@@ -228,9 +229,82 @@ int dispatch_chunked(ssm_scan_s *h, ssm::ScanParams &p, int dtype, int tb,
   return SSM_ERR_UNSUPPORTED;
 }
 
+template <typename T, int QP>
+int launch_step_qp(const ssm::StepParams &p, bool vec, cudaStream_t s) {
+  const int64_t threads = p.batch * p.dim * QP;
+  const int64_t blocks = (threads + 255) / 256;
+  if (blocks > 0x7fffffff) return SSM_ERR_UNSUPPORTED;
+  if (vec)
+    ssm::scan_step_kernel<T, QP, true><<<unsigned(blocks), 256, 0, s>>>(p);
+  else
+    ssm::scan_step_kernel<T, QP, false><<<unsigned(blocks), 256, 0, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+template <typename T>
+int launch_step(const ssm::StepParams &p, bool vec, cudaStream_t s) {
+  const int groups = (p.dstate + 3) / 4;
+  if (groups <= 1) return launch_step_qp<T, 1>(p, vec, s);
+  if (groups <= 2) return launch_step_qp<T, 2>(p, vec, s);
+  if (groups <= 4) return launch_step_qp<T, 4>(p, vec, s);
+  if (groups <= 8) return launch_step_qp<T, 8>(p, vec, s);
+  return launch_step_qp<T, 16>(p, vec, s);
+}
+
 }  // namespace
 
 extern "C" {
+
+int ssm_scan_step(ssm_scan_t h, const void *x_new, void *conv_state,
+                  const float *conv_weight, const float *conv_bias,
+                  int conv_width, const void *delta, const float *delta_bias,
+                  const float *A_log, const void *B, const void *C,
+                  const float *D, const void *z, uint32_t flags, float *state,
+                  void *y, ssm_scan_dims dims, int dtype,
+                  struct CUstream_st *stream) {
+  if (!h || !x_new || !delta || !A_log || !B || !C || !state || !y)
+    return SSM_ERR_INVALID;
+  if (dims.batch <= 0 || dims.dim <= 0 || dims.dstate <= 0 || dims.seqlen != 1)
+    return SSM_ERR_INVALID;
+  if (flags & ~uint32_t(SSM_DELTA_SOFTPLUS | SSM_WRITE_ZOH))
+    return SSM_ERR_INVALID;
+  if (conv_state && (!conv_weight || conv_width < 1 ||
+                     conv_width > ssm::kMaxConvWidth))
+    return SSM_ERR_INVALID;
+  if (dtype != SSM_F32 && dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
+  if (dims.dstate > 64) return SSM_ERR_UNSUPPORTED;
+  int64_t chans = 0, st = 0;
+  if (!mul_ok(dims.batch, dims.dim, &chans) ||
+      !mul_ok(chans, dims.dstate, &st) || st > (int64_t(1) << 56))
+    return SSM_ERR_INVALID;
+  const size_t esz = dtype == SSM_F32 ? 4 : 2;
+  const void *acts[] = {x_new, conv_state, delta, B, C, z, y};
+  for (const void *q : acts)
+    if (q && !aligned(q, esz)) return SSM_ERR_ALIGN;
+  const float *params[] = {conv_weight, conv_bias, delta_bias, A_log, D,
+                           state};
+  for (const float *q : params)
+    if (q && !aligned(q, 4)) return SSM_ERR_ALIGN;
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) {
+    cudaGetLastError();
+    return SSM_ERR_CUDA;
+  }
+  if (cur != h->device) return SSM_ERR_INVALID;
+
+  ssm::StepParams p{};
+  p.x_new = x_new; p.conv_state = conv_state; p.conv_weight = conv_weight;
+  p.conv_bias = conv_bias; p.conv_width = conv_state ? conv_width : 0;
+  p.delta = delta; p.delta_bias = delta_bias; p.A_log = A_log;
+  p.B = B; p.C = C; p.D = D; p.z = z; p.state = state; p.y = y;
+  p.batch = dims.batch; p.dim = dims.dim; p.dstate = int(dims.dstate);
+  p.softplus = (flags & SSM_DELTA_SOFTPLUS) ? 1 : 0;
+  p.write_zoh = (flags & SSM_WRITE_ZOH) ? 1 : 0;
+  const bool vec = (dims.dstate % 4 == 0) && aligned(state, 16);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return dtype == SSM_F32 ? launch_step<float>(p, vec, s)
+                          : launch_step<__nv_bfloat16>(p, vec, s);
+}
 
 int ssm_scan_create(ssm_scan_t *out, int device) {
   if (!out) return SSM_ERR_INVALID;
