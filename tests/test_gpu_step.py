@@ -45,9 +45,11 @@ def test_step_parity(scan, dtype, N, conv, zoh, gate):
     cw = rng.standard_normal((E, conv)).astype(np.float32) if conv else None
     cb = rng.standard_normal(E).astype(np.float32) if conv else None
     conv_h = rng.standard_normal((b, E, conv)) if conv else None
-    if conv and dtype == W.BF16:     # the buffer lives in bfloat16
-        conv_h = W.bf16_bits_to_f32(W.round_to_bf16_bits(
-            conv_h.astype(np.float32))).astype(np.float64)
+    if conv:   # the buffer lives in the activation type
+        conv_h = conv_h.astype(np.float32).astype(np.float64)
+        if dtype == W.BF16:
+            conv_h = W.bf16_bits_to_f32(W.round_to_bf16_bits(
+                conv_h.astype(np.float32))).astype(np.float64)
     conv_t = _dev(conv_h, dtype) if conv else None
     A_log = torch.from_numpy(wl.dev["A_log"]).cuda()
     D = torch.from_numpy(wl.dev["D"]).cuda()
