@@ -81,6 +81,11 @@ class OracleLib:
         lib.ssm_oracle_scan_ex.argtypes = [i64, i64, i64, i64, d, d, d, d, d,
                                            d, d, d, ctypes.c_int, ctypes.c_int,
                                            d, d, d, d, ctypes.c_int]
+        lib.ssm_oracle_scan_conv.restype = ctypes.c_int
+        lib.ssm_oracle_scan_conv.argtypes = [i64, i64, i64, i64, i64, d, d, d,
+                                             d, d, d, d, d, d, d,
+                                             ctypes.c_int, ctypes.c_int, d, d,
+                                             d, ctypes.c_int]
         lib.ssm_oracle_step.restype = ctypes.c_int
         lib.ssm_oracle_step.argtypes = [i64, i64, i64, i64, d, d, d, d, d, d,
                                         ctypes.c_int, ctypes.c_int, d, d, d, d,
@@ -139,6 +144,33 @@ class OracleLib:
             return y, h_last, states
         return y, h_last
 
+
+    def scan_conv(self, v, conv_weight, delta, A_log, B, C, conv_bias=None,
+                  D=None, z=None, delta_bias=None, delta_softplus=True,
+                  h0=None, write_zoh=False, nthreads=0):
+        """The scan of x = SiLU(causal_conv(v)) (left zero padding). Returns
+        (y [b, L, E], h_last [b, E, N])."""
+        va = np.asarray(v)
+        b, L, E = va.shape
+        N = np.asarray(A_log).shape[-1]
+        K = np.asarray(conv_weight).shape[-1]
+        y = np.empty((b, L, E), dtype=np.float64)
+        h_last = np.empty((b, E, N), dtype=np.float64)
+        rc = self.lib.ssm_oracle_scan_conv(
+            b, L, E, N, K, _ptr(_f64(va, (b, L, E), "v")),
+            _ptr(_f64(conv_weight, (E, K), "conv_weight")),
+            _ptr(_f64(conv_bias, (E,), "conv_bias")),
+            _ptr(_f64(delta, (b, L, E), "delta")),
+            _ptr(_f64(A_log, (E, N), "A_log")), _ptr(_f64(B, (b, L, N), "B")),
+            _ptr(_f64(C, (b, L, N), "C")), _ptr(_f64(D, (E,), "D")),
+            _ptr(_f64(z, (b, L, E), "z")),
+            _ptr(_f64(delta_bias, (E,), "delta_bias")),
+            int(bool(delta_softplus)), int(bool(write_zoh)),
+            _ptr(_f64(h0, (b, E, N), "h0")), _ptr(y), _ptr(h_last),
+            int(nthreads))
+        if rc != 0:
+            raise ValueError("oracle rejected its arguments (rc=%d)" % rc)
+        return y, h_last
 
     def step(self, x_new, delta, A_log, B, C, state, conv_state=None,
              conv_weight=None, conv_bias=None, D=None, z=None,
@@ -204,6 +236,17 @@ def scan(x, delta, A_log, B, C, D=None, z=None, delta_bias=None,
                         delta_bias=delta_bias, delta_softplus=delta_softplus,
                         h0=h0, return_states=return_states, nthreads=nthreads,
                         write_zoh=write_zoh)
+
+
+def scan_conv(v, conv_weight, delta, A_log, B, C, conv_bias=None, D=None,
+              z=None, delta_bias=None, delta_softplus=True, h0=None,
+              write_zoh=False, nthreads=0):
+    """The scan of SiLU(causal_conv(v)) (see OracleLib.scan_conv)."""
+    return _load().scan_conv(v, conv_weight, delta, A_log, B, C,
+                             conv_bias=conv_bias, D=D, z=z,
+                             delta_bias=delta_bias,
+                             delta_softplus=delta_softplus, h0=h0,
+                             write_zoh=write_zoh, nthreads=nthreads)
 
 
 def step(x_new, delta, A_log, B, C, state, conv_state=None, conv_weight=None,

@@ -260,3 +260,50 @@ int ssm_oracle_step(int64_t batch, int64_t dim, int64_t dstate, int64_t width,
     }
     return 0;
 }
+
+/*
+ * The scan with the causal depthwise convolution in front ("Mamba:
+ * Linear-Time Sequence Modeling with Selective State Spaces",
+ * www.abhik.ai/papers/mamba, section "Original paper, equations and runnable
+ * CPU code", row "4. Add causal local context before selecting
+ * coefficients" and row "5. Put the selective operator inside the complete
+ * mixer"):
+ *   x[t, c] = SiLU(conv_bias[c] + sum_{k<K} w[c, k] * v[t - K + 1 + k, c])
+ * with zeros before the start (left padding), then ssm_oracle_scan_ex on x
+ * (D x and the gate use this x). v: [batch, seqlen, dim]; w: [dim, K].
+ */
+int ssm_oracle_scan_conv(int64_t batch, int64_t seqlen, int64_t dim,
+                         int64_t dstate, int64_t width, const double *v,
+                         const double *conv_weight, const double *conv_bias,
+                         const double *delta, const double *A_log,
+                         const double *B, const double *C, const double *D,
+                         const double *z, const double *delta_bias,
+                         int delta_softplus, int write_zoh, const double *h0,
+                         double *y, double *h_last, int nthreads)
+{
+    if (!v || !conv_weight || width <= 0 || batch <= 0 || seqlen <= 0 ||
+        dim <= 0)
+        return -1;
+    const int64_t n = batch * seqlen * dim;
+    double *x = (double *)malloc((size_t)n * sizeof(double));
+    if (!x)
+        return -1;
+    for (int64_t b = 0; b < batch; ++b)
+        for (int64_t t = 0; t < seqlen; ++t)
+            for (int64_t c = 0; c < dim; ++c) {
+                double acc = conv_bias ? conv_bias[c] : 0.0;
+                for (int64_t k = 0; k < width; ++k) {
+                    const int64_t s = t - width + 1 + k;
+                    if (s >= 0)
+                        acc += conv_weight[c * width + k] *
+                               v[(b * seqlen + s) * dim + c];
+                }
+                x[(b * seqlen + t) * dim + c] = silu(acc);
+            }
+    const int rc = ssm_oracle_scan_ex(batch, seqlen, dim, dstate, x, delta,
+                                      A_log, B, C, D, z, delta_bias,
+                                      delta_softplus, write_zoh, h0, y, h_last,
+                                      NULL, nthreads);
+    free(x);
+    return rc;
+}

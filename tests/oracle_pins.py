@@ -616,6 +616,43 @@ def pin_step_conv_feeds_scan(o):
     _close(state, h_last, 1e-12, 1e-10, "decode with conv, state")
 
 
+def pin_scan_conv(o):
+    """The scan with the causal convolution in front.
+
+    [abhik] "4. Add causal local context before selecting coefficients" and
+    "5. Put the selective operator inside the complete mixer": the scan runs
+    on x = SiLU(CausalDWConv(v)) with left zero padding. Checked against (i)
+    the pinned scan of x formed with numpy's convolution, and (ii) decoding
+    the sequence token by token through the conv buffer ("6. Carry both
+    buffers").
+    """
+    rng = np.random.default_rng(61)
+    b, L, E, N, K = 2, 21, 3, 4, 4
+    case = random_case(67, b, L, E, N)
+    v = rng.standard_normal((b, L, E))
+    w = rng.standard_normal((E, K))
+    cb = rng.standard_normal(E)
+    y, h = o.scan_conv(v, w, case["delta"], case["A_log"], case["B"],
+                       case["C"], conv_bias=cb, D=case["D"], z=case["z"],
+                       delta_bias=case["delta_bias"], h0=case["h0"])
+    xc = np.empty_like(v)
+    for bb in range(b):
+        for e in range(E):
+            pre = np.convolve(v[bb, :, e], w[e, ::-1])[:L] + cb[e]
+            xc[bb, :, e] = pre / (1.0 + np.exp(-pre))
+    y2, h2 = o.scan(**dict(case, x=xc), delta_softplus=True)
+    _close(y, y2, 1e-12, 1e-10, "scan_conv vs scan of numpy conv")
+    _close(h, h2, 1e-12, 1e-10, "scan_conv state")
+    state, conv = case["h0"].copy(), np.zeros((b, E, K))
+    for t in range(L):
+        yt, state, conv = o.step(v[:, t], case["delta"][:, t], case["A_log"],
+                                 case["B"][:, t], case["C"][:, t], state,
+                                 conv_state=conv, conv_weight=w, conv_bias=cb,
+                                 D=case["D"], z=case["z"][:, t],
+                                 delta_bias=case["delta_bias"])
+        _close(yt, y[:, t], 1e-12, 1e-10, "decode vs scan_conv step %d" % t)
+
+
 # ---------------------------------------------------------------- softplus
 def pin_step_size(o):
     """delta = softplus(raw + bias), PyTorch default softplus.
@@ -648,4 +685,4 @@ ALL_PINS = (pin_associative_prefix, pin_lti_convolution, pin_forgetting,
             pin_decode_step, pin_linearity, pin_independence, pin_degenerate,
             pin_step_size, pin_zoh_lti, pin_zoh_fixed_point, pin_zoh_small_step,
             pin_step_matches_scan, pin_step_causal_convolution,
-            pin_step_conv_feeds_scan)
+            pin_step_conv_feeds_scan, pin_scan_conv)

@@ -37,6 +37,11 @@ MUTANTS = [
     ("decode write uses the raw input, not the convolved one",
      [("* B[b * dstate + n]\n                    * xv;",
        "* B[b * dstate + n]\n                    * x_new[i];")]),
+    ("scan convolution reads the future",
+     [("const int64_t s = t - width + 1 + k;", "const int64_t s = t + k;")]),
+    ("scan convolution without SiLU",
+     [("x[(b * seqlen + t) * dim + c] = silu(acc);",
+       "x[(b * seqlen + t) * dim + c] = acc;")]),
     ("zero-order hold without dividing by A",
      [("return expm1(step * A) / A;", "return expm1(step * A);")]),
     ("zero-order hold with exp instead of expm1",
