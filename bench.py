@@ -8,7 +8,7 @@ SiLU gate, y and h_last stores). Default workload: the Mamba-2.8B-shaped layer
 seeded inputs (selective_state_space_51_b200.workloads, shape 3).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--shape I]
-                    [--impl reference]
+                    [--impl reference] [--op scan|conv|step]
 
 Prints ONE JSON line (rank 0). Multi-GPU runs are launched by torchrun with
 one process per GPU; each rank scans its own batch of sequences (weak
@@ -18,6 +18,14 @@ The metric: scan elements (b*L*E*N) per second, with the achieved GB/s of
 algorithmic traffic and the fraction of the min(HBM, SFU-exp) roofline:
 T_roof = max(bytes / HBM peak, exps / SFU peak), fraction = T_roof / T.
 `--impl reference` times the float64 CPU oracle instead (rank 0 only).
+
+Two more operations print a line of the same form: `--op conv` times the scan
+with the causal depthwise convolution (width 4) + SiLU fused in front
+(ssm_scan_fwd_conv, same workload and roofline), and `--op step` times one
+batched decode step (ssm_scan_step: conv buffer shift, conv + SiLU, state
+update, readout) over a [1024 x 5120 x 16] float32 state with bfloat16
+activations, against the HBM roofline (it moves the state twice and does
+little arithmetic).
 """
 from __future__ import annotations
 
@@ -64,7 +72,11 @@ def max_over_ranks(value: float, dist=None, device=None) -> float:
 
 
 # ----------------------------------------------------------------- workload
-def algorithmic_bytes(wl) -> int:
+CONV_WIDTH = 4
+DECODE_BATCH = 1024
+
+
+def algorithmic_bytes(wl, op: str = "scan") -> int:
     """Each input read once, y written once, h0/h_last once; no [b,L,E,N]."""
     b, L, E, N = wl.batch, wl.seqlen, wl.dim, wl.dstate
     act = 4 if wl.dtype == "f32" else 2
@@ -78,6 +90,22 @@ def algorithmic_bytes(wl) -> int:
     n += E * 4 if wl.dev["delta_bias"] is not None else 0
     n += b * E * N * 4                 # h_last
     n += b * E * N * 4 if wl.dev["h0"] is not None else 0
+    if op == "conv":
+        n += E * CONV_WIDTH * 4 + E * 4    # filter taps and bias
+    return n
+
+
+def decode_bytes(wl) -> int:
+    """One decode step: the float32 state and the conv buffer are read and
+    written once; x_new, raw step, z, y once per channel; B, C once per row;
+    the parameters once."""
+    b, E, N = wl.batch, wl.dim, wl.dstate
+    act = 4 if wl.dtype == "f32" else 2
+    n = 2 * b * E * N * 4                      # state in and out
+    n += 2 * b * E * CONV_WIDTH * act          # conv buffer in and out
+    n += 4 * b * E * act                       # x_new, delta, z, y
+    n += 2 * b * N * act                       # B, C
+    n += E * N * 4 + E * CONV_WIDTH * 4 + 3 * E * 4  # A_log, taps, biases, D
     return n
 
 
@@ -225,11 +253,102 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------- GPU leg
+def _to_device(arrays, dev):
+    import torch
+    out = {}
+    for k, v in arrays.items():
+        if v is None:
+            out[k] = None
+        elif v.dtype == np.uint16:
+            out[k] = torch.from_numpy(v.view(np.int16)).to(dev).view(
+                torch.bfloat16)
+        else:
+            out[k] = torch.from_numpy(np.ascontiguousarray(v)).to(dev)
+    return out
+
+
+class ScanOp:
+    """One forward scan (optionally with the fused convolution) per step."""
+
+    def __init__(self, args, plan, dev, scan):
+        import torch
+        from selective_state_space_51_b200 import workloads as W
+        self.name = args.op
+        self.wl = wl = W.make(plan["shape"], seed=plan["seed"])
+        self.t = _to_device(wl.dev, dev)
+        self.conv = None
+        if args.op == "conv":
+            w, cb = W.conv_params(wl.dim, CONV_WIDTH)
+            self.conv = (torch.from_numpy(w).to(dev),
+                         torch.from_numpy(cb).to(dev))
+        self.scan = scan
+        self.y = torch.empty_like(self.t["x"])
+        self.h_last = torch.empty((wl.batch, wl.dim, wl.dstate),
+                                  dtype=torch.float32, device=dev)
+        self.per_step_in = ("x", "delta", "z", "B", "C", "h0")
+        self.units = wl.elements             # b*L*E*N per step
+        self.nbytes = algorithmic_bytes(wl, args.op)
+        self.workload = W.shape_description(args.shape) + (
+            "; causal depthwise conv width %d + SiLU fused in front"
+            % CONV_WIDTH if self.conv else "")
+
+    def run(self, t, stream):
+        kw = {}
+        if self.conv:
+            kw = dict(conv_weight=self.conv[0], conv_bias=self.conv[1])
+        self.scan(t["x"], t["delta"], t["A_log"], t["B"], t["C"], D=t["D"],
+                  z=t["z"], delta_bias=t["delta_bias"], h0=t["h0"], y=self.y,
+                  h_last=self.h_last, stream=stream, **kw)
+
+    def outputs(self):
+        return (self.y, self.h_last)
+
+
+class StepOp:
+    """One batched decode step per step (state updated in place)."""
+
+    def __init__(self, args, plan, dev, scan):
+        import torch
+        from selective_state_space_51_b200 import workloads as W
+        self.name = "step"
+        wl = W.make(plan["shape"], seed=plan["seed"], batch=DECODE_BATCH,
+                    seqlen=1, with_h0=True)
+        self.wl = wl
+        w, cb = W.conv_params(wl.dim, CONV_WIDTH)
+        d = {k: (v if v is None or k in ("A_log", "D", "delta_bias", "h0")
+                 else v.reshape(v.shape[0], v.shape[2]))
+             for k, v in wl.dev.items()}
+        self.t = _to_device(d, dev)
+        self.state = self.t.pop("h0")
+        act = self.t["x"].dtype
+        self.conv_state = torch.zeros((wl.batch, wl.dim, CONV_WIDTH),
+                                      dtype=act, device=dev)
+        self.conv = (torch.from_numpy(w).to(dev), torch.from_numpy(cb).to(dev))
+        self.scan = scan
+        self.y = torch.empty_like(self.t["x"])
+        self.per_step_in = ("x", "delta", "z", "B", "C")
+        self.units = wl.batch * wl.dim * wl.dstate
+        self.nbytes = decode_bytes(wl)
+        self.workload = (
+            "decode step, Mamba-2.8B layer shape: %d sequences x E=%d x N=%d "
+            "float32 state, conv width %d, %s activations" % (
+                wl.batch, wl.dim, wl.dstate, CONV_WIDTH, wl.dtype))
+
+    def run(self, t, stream):
+        self.scan.step(t["x"], t["delta"], t["A_log"], t["B"], t["C"],
+                       self.state, conv_state=self.conv_state,
+                       conv_weight=self.conv[0], conv_bias=self.conv[1],
+                       D=t["D"], z=t["z"], delta_bias=t["delta_bias"],
+                       y=self.y, stream=stream)
+
+    def outputs(self):
+        return (self.y,)
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
     import selective_state_space_51_b200 as S
-    from selective_state_space_51_b200 import workloads as W
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -244,33 +363,17 @@ def run_gpu(args):
                                 device_id=dev)
 
     plan = shard_for_rank(rank, world, args.shape)
-    wl = W.make(plan["shape"], seed=plan["seed"])
-    t = {}
-    for k, v in wl.dev.items():
-        if v is None:
-            t[k] = None
-        elif v.dtype == np.uint16:
-            t[k] = torch.from_numpy(v.view(np.int16)).to(dev).view(
-                torch.bfloat16)
-        else:
-            t[k] = torch.from_numpy(np.ascontiguousarray(v)).to(dev)
     scan = S.SelectiveScan(local)
-    y = torch.empty_like(t["x"])
-    h_last = torch.empty((wl.batch, wl.dim, wl.dstate), dtype=torch.float32,
-                         device=dev)
+    op = (StepOp if args.op == "step" else ScanOp)(args, plan, dev, scan)
+    t = op.t
     stream = torch.cuda.current_stream(dev)
-
-    def step():
-        scan(t["x"], t["delta"], t["A_log"], t["B"], t["C"], D=t["D"],
-             z=t["z"], delta_bias=t["delta_bias"], h0=t["h0"], y=y,
-             h_last=h_last, stream=stream)
 
     def barrier():
         if world > 1:
             dist.barrier(device_ids=[local])
 
     for _ in range(args.warmup):
-        step()
+        op.run(t, stream)
     torch.cuda.synchronize(dev)
     if scan.sync_status(stream) != S.SSM_OK:
         raise SystemExit("device status error during warm-up")
@@ -286,7 +389,7 @@ def run_gpu(args):
         t_begin.record(stream)
         for i in range(args.steps):
             starts[i].record(stream)
-            step()
+            op.run(t, stream)
             ends[i].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize(dev)
@@ -299,37 +402,33 @@ def run_gpu(args):
     kernel_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends))
     total_ms = max_over_ranks(local_ms, dist if world > 1 else None, dev)
     kernel_ms = max_over_ranks(kernel_ms, dist if world > 1 else None, dev)
-    variant = scan.last_variant()
+    variant = scan.last_variant() if op.name != "step" else (0, 0)
 
     # ---- end to end through the public API with pinned host buffers
     if args.no_e2e:
-        return _finish(args, wl, world, rank, local, dev, dist, scan, clocks,
+        return _finish(args, op, world, rank, local, dev, dist, scan, clocks,
                        total_ms, kernel_ms, variant, None, 0, 0)
     host = {k: (None if v is None else v.cpu().pin_memory())
             for k, v in t.items()}
-    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-    h_host = torch.empty(h_last.shape, dtype=h_last.dtype).pin_memory()
+    outs = op.outputs()
+    out_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory()
+                for o in outs]
     dev_in = {k: (None if v is None else torch.empty_like(v))
               for k, v in t.items()}
-    per_step_in = ("x", "delta", "z", "B", "C", "h0")
     h2d = sum(host[k].numel() * host[k].element_size()
-              for k in per_step_in if host[k] is not None)
-    d2h = y_host.numel() * y_host.element_size() + \
-        h_host.numel() * h_host.element_size()
+              for k in op.per_step_in if host.get(k) is not None)
+    d2h = sum(o.numel() * o.element_size() for o in out_host)
     for k, v in host.items():
         if v is not None:
             dev_in[k].copy_(v)
 
     def e2e_step():
-        for k in per_step_in:
-            if host[k] is not None:
+        for k in op.per_step_in:
+            if host.get(k) is not None:
                 dev_in[k].copy_(host[k], non_blocking=True)
-        scan(dev_in["x"], dev_in["delta"], dev_in["A_log"], dev_in["B"],
-             dev_in["C"], D=dev_in["D"], z=dev_in["z"],
-             delta_bias=dev_in["delta_bias"], h0=dev_in["h0"], y=y,
-             h_last=h_last, stream=stream)
-        y_host.copy_(y, non_blocking=True)
-        h_host.copy_(h_last, non_blocking=True)
+        op.run(dev_in, stream)
+        for o, oh in zip(outs, out_host):
+            oh.copy_(o, non_blocking=True)
 
     e2e_steps = max(3, min(args.steps, args.e2e_steps))
     for _ in range(2):
@@ -346,68 +445,82 @@ def run_gpu(args):
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps,
                             dist if world > 1 else None, dev)
-    return _finish(args, wl, world, rank, local, dev, dist, scan, clocks,
+    return _finish(args, op, world, rank, local, dev, dist, scan, clocks,
                    total_ms, kernel_ms, variant, e2e_ms, h2d, d2h)
 
 
-def _finish(args, wl, world, rank, local, dev, dist, scan, clocks, total_ms,
+def _finish(args, op, world, rank, local, dev, dist, scan, clocks, total_ms,
             kernel_ms, variant, e2e_ms, h2d, d2h):
     import torch
-    from selective_state_space_51_b200 import workloads as W
     peaks = load_peaks()
     clk = clocks.summary()
-    nbytes = algorithmic_bytes(wl)
-    exps = wl.elements
+    wl = op.wl
+    nbytes = op.nbytes
+    units = op.units
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     ms = total_ms / args.steps
-    value = world * exps / (ms * 1e-3)
+    value = world * units / (ms * 1e-3)
     gbps = nbytes / (kernel_ms * 1e-3) / 1e9
     sfu_peak_max = sms * SFU_EX2_PER_CLK_PER_SM * peaks["sm_max_mhz"] * 1e6
     sfu_peak_run = (sms * SFU_EX2_PER_CLK_PER_SM * clk["sm_mhz"] * 1e6
                     if clk["sm_mhz"] else None)
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
-    t_sfu = exps / sfu_peak_max
+    t_sfu = units / sfu_peak_max       # one retention exp per unit
     t_roof = max(t_hbm, t_sfu)
-    achieved_exp = exps / (kernel_ms * 1e-3)
+    achieved_exp = units / (kernel_ms * 1e-3)
+    if op.name == "step":
+        metric = ("decode step (b·E·N) state elements/s; GB/s; "
+                  "% of HBM roofline")
+        unit = "state elements/s"
+        roof = {"bound": "hbm", "unit": "GB/s", "achieved": gbps,
+                "peak": peaks["hbm_gbs"], "frac": gbps / peaks["hbm_gbs"],
+                "peak_note": "%s HBM copy bandwidth" % peaks["source"],
+                "traffic": None}
+        l2 = ("state of %.0f MB, larger than L2, rewritten every step"
+              % (wl.batch * wl.dim * wl.dstate * 4 / 1e6))
+    else:
+        metric, unit = METRIC, UNIT
+        roof = {"bound": "alu", "unit": "Gexp/s",
+                "achieved": achieved_exp / 1e9,
+                "peak": sfu_peak_max / 1e9,
+                "frac": achieved_exp / sfu_peak_max,
+                "peak_note": "SFU ex2: %d SMs x %d/clk x %.0f MHz (max SM "
+                             "clock, %s)" % (sms, SFU_EX2_PER_CLK_PER_SM,
+                                             peaks["sm_max_mhz"],
+                                             peaks["source"]),
+                "frac_at_sampled_clock": (achieved_exp / sfu_peak_run
+                                          if sfu_peak_run else None),
+                "traffic": None}
+        l2 = "inputs larger than L2 (%.0f MB read per step)" % (nbytes / 1e6)
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "metric": metric, "value": value, "unit": unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "io_dtype": wl.dtype, "data": "synthetic",
-        "config": {"workload": W.shape_description(args.shape),
+        "config": {"workload": op.workload, "op": op.name,
                    "global_batch": world * wl.batch, "seq_len": wl.seqlen,
                    "dim": wl.dim, "dstate": wl.dstate,
-                   "parallelism": "dp%d" % world,
-                   "l2": "inputs larger than L2 (%.0f MB read per step)"
-                         % (nbytes / 1e6)},
+                   "parallelism": "dp%d" % world, "l2": l2},
         "gb_per_s": gbps,
-        "roofline_min_hbm_sfu": {
+        "roofline": roof,
+        "e2e": (None if e2e_ms is None else
+                {"value": world * units / (e2e_ms * 1e-3), "unit": unit,
+                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                 "ms_per_step": e2e_ms}),
+        "gpu_launches": args.steps,
+        "clocks": clk,
+    }
+    if op.name != "step":
+        line["roofline_min_hbm_sfu"] = {
             "t_hbm_us": t_hbm * 1e6, "t_sfu_us_at_max_clock": t_sfu * 1e6,
             "t_kernel_us": kernel_ms * 1e3,
             "frac": t_roof / (kernel_ms * 1e-3),
             "hbm_peak_gbs": peaks["hbm_gbs"], "hbm_source": peaks["source"],
             "frac_at_8tbs_hbm": max(nbytes / (HBM_NOMINAL_GBS * 1e9), t_sfu)
-            / (kernel_ms * 1e-3)},
-        "roofline": {"bound": "alu", "unit": "Gexp/s",
-                     "achieved": achieved_exp / 1e9,
-                     "peak": sfu_peak_max / 1e9,
-                     "frac": achieved_exp / sfu_peak_max,
-                     "peak_note": "SFU ex2: %d SMs x %d/clk x %.0f MHz (max "
-                                  "SM clock, %s)" % (
-                                      sms, SFU_EX2_PER_CLK_PER_SM,
-                                      peaks["sm_max_mhz"], peaks["source"]),
-                     "frac_at_sampled_clock": (achieved_exp / sfu_peak_run
-                                               if sfu_peak_run else None),
-                     "traffic": None},
-        "e2e": (None if e2e_ms is None else
-                {"value": world * exps / (e2e_ms * 1e-3), "unit": UNIT,
-                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                 "ms_per_step": e2e_ms}),
-        "gpu_launches": args.steps,
-        "kernel": {"variant": variant[0], "segments": variant[1]},
-        "clocks": clk,
-    }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            / (kernel_ms * 1e-3)}
+        line["kernel"] = {"variant": variant[0], "segments": variant[1]}
+    if (rank == 0 and world == 1 and not args.no_cpu_baseline
+            and op.name == "scan"):
         line["cpu_baseline"] = cpu_oracle_rate(wl, args.reference_seconds)
     scan.close()
     if world > 1:
@@ -426,6 +539,9 @@ def main(argv=None):
     ap.add_argument("--shape", type=int, default=3,
                     help="workload shape index (default 3: Mamba-2.8B layer)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--op", choices=["scan", "conv", "step"], default="scan",
+                    help="scan (default), the scan with the fused "
+                         "convolution, or the batched decode step")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--reference-seconds", type=float, default=10.0,
                     help="CPU seconds of the oracle sample in cpu_baseline")

@@ -148,6 +148,34 @@ SSM_API int ssm_scan_fwd(ssm_scan_t h, const void *x, const void *delta,
                  ssm_scan_dims dims, int dtype, struct CUstream_st *stream);
 
 /*
+ * ssm_scan_fwd_conv: ssm_scan_fwd with the causal depthwise convolution and
+ * SiLU that produce x fused in front ("Mamba: Linear-Time Sequence Modeling
+ * with Selective State Spaces", www.abhik.ai/papers/mamba, section "Original
+ * paper, equations and runnable CPU code", row "4. Add causal local context
+ * before selecting coefficients", and row "5. Put the selective operator
+ * inside the complete mixer"):
+ *     x[b, t, e] = SiLU(conv_bias[e] + sum_{k<K} conv_weight[e, k] *
+ *                       v[b, t - K + 1 + k, e]),  v = 0 before t = 0,
+ * then the scan of ssm_scan_fwd on x (D x and the gate use this x). x is
+ * formed in registers; it is never written to memory.
+ *   v           : [batch, seqlen, dim] activation dtype, required.
+ *   conv_weight : [dim, conv_width] float32, required (SSM_ERR_INVALID).
+ *   conv_bias   : [dim] float32, NULL means zero.
+ *   conv_width  : K, 1..SSM_SCAN_CONV_MAX_WIDTH (else SSM_ERR_INVALID).
+ * Everything else, and every error, as for ssm_scan_fwd.
+ */
+#define SSM_SCAN_CONV_MAX_WIDTH 4
+SSM_API int ssm_scan_fwd_conv(ssm_scan_t h, const void *v,
+                              const float *conv_weight, const float *conv_bias,
+                              int conv_width, const void *delta,
+                              const float *A_log, const void *B, const void *C,
+                              const float *D, const void *z,
+                              const float *delta_bias, uint32_t flags,
+                              const float *h0, void *y, float *h_last,
+                              ssm_scan_dims dims, int dtype,
+                              struct CUstream_st *stream);
+
+/*
  * ssm_scan_set_variant: force a kernel variant for later calls on this
  * handle (SSM_VARIANT_*), or SSM_VARIANT_AUTO to choose by shape.
  * `segments` > 1 asks the chunked variant to split every sequence into that

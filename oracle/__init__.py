@@ -259,6 +259,26 @@ def step(x_new, delta, A_log, B, C, state, conv_state=None, conv_weight=None,
                         delta_softplus=delta_softplus, write_zoh=write_zoh)
 
 
+def scan_conv_channels(channels, v, conv_weight, delta, A_log, B, C,
+                       conv_bias=None, D=None, z=None, delta_bias=None,
+                       delta_softplus=True, h0=None, nthreads=0,
+                       write_zoh=False):
+    """scan_conv on a subset of channels. The convolution is depthwise (one
+    filter per channel), so channels stay independent as in scan_channels."""
+    ch = np.asarray(channels, dtype=np.int64)
+    sel = lambda a: None if a is None else np.asarray(a)[..., ch]  # noqa: E731
+    h0s = None if h0 is None else np.asarray(h0)[:, ch, :]
+    return scan_conv(sel(v), np.asarray(conv_weight)[ch], sel(delta),
+                     np.asarray(A_log)[ch], B, C,
+                     conv_bias=None if conv_bias is None
+                     else np.asarray(conv_bias)[ch],
+                     D=None if D is None else np.asarray(D)[ch], z=sel(z),
+                     delta_bias=None if delta_bias is None
+                     else np.asarray(delta_bias)[ch],
+                     delta_softplus=delta_softplus, h0=h0s,
+                     write_zoh=write_zoh, nthreads=nthreads)
+
+
 def scan_channels(channels, x, delta, A_log, B, C, D=None, z=None,
                   delta_bias=None, delta_softplus=True, h0=None, nthreads=0,
                   write_zoh=False):

@@ -74,6 +74,10 @@ def library() -> ctypes.CDLL:
                                          u32, vp, vp, vp, ssm_scan_dims, i32,
                                          vp]
             lib.ssm_scan_fwd.restype = i32
+            lib.ssm_scan_fwd_conv.argtypes = [vp, vp, vp, vp, i32, vp, vp, vp,
+                                              vp, vp, vp, vp, u32, vp, vp, vp,
+                                              ssm_scan_dims, i32, vp]
+            lib.ssm_scan_fwd_conv.restype = i32
             lib.ssm_scan_set_variant.argtypes = [vp, i32, i32]
             lib.ssm_scan_set_variant.restype = i32
             lib.ssm_scan_last_variant.argtypes = [vp, ctypes.POINTER(i32),
@@ -164,6 +168,21 @@ def ssm_scan_fwd(h, x, delta, A_log, B, C, D, z, delta_bias, flags, h0, y,
                                 int(flags), _ptr(h0), _ptr(y), _ptr(h_last),
                                 dims, int(dtype), _stream(stream))
     return _check(rc, "ssm_scan_fwd") if check else rc
+
+
+def ssm_scan_fwd_conv(h, v, conv_weight, conv_bias, conv_width, delta, A_log,
+                      B, C, D, z, delta_bias, flags, h0, y, h_last, dims,
+                      dtype, stream=None, check=True) -> int:
+    """Call ssm_scan_fwd_conv: the scan of SiLU(causal depthwise conv of v)
+    (see include/ssm_scan.h). dims is (batch, seqlen, dim, dstate)."""
+    if not isinstance(dims, ssm_scan_dims):
+        dims = ssm_scan_dims(*[int(d) for d in dims])
+    rc = library().ssm_scan_fwd_conv(
+        h, _ptr(v), _ptr(conv_weight), _ptr(conv_bias), int(conv_width),
+        _ptr(delta), _ptr(A_log), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+        _ptr(delta_bias), int(flags), _ptr(h0), _ptr(y), _ptr(h_last), dims,
+        int(dtype), _stream(stream))
+    return _check(rc, "ssm_scan_fwd_conv") if check else rc
 
 
 def ssm_scan_step(h, x_new, conv_state, conv_weight, conv_bias, conv_width,
@@ -260,7 +279,10 @@ class SelectiveScan:
 
     def __call__(self, x, delta, A_log, B, C, D=None, z=None, delta_bias=None,
                  delta_softplus=True, h0=None, y=None, h_last=None,
-                 return_last_state=True, stream=None, write_zoh=False):
+                 return_last_state=True, stream=None, write_zoh=False,
+                 conv_weight=None, conv_bias=None):
+        """The forward scan. With conv_weight ([E, K] float32) x is the input
+        of the causal depthwise convolution + SiLU fused in front."""
         import torch
         if x.dtype == torch.float32:
             dtype = SSM_F32
@@ -277,7 +299,9 @@ class SelectiveScan:
                 raise ValueError("%s must be a contiguous %s tensor on %s"
                                  % (name, x.dtype, self.device))
         for name, t in (("A_log", A_log), ("D", D),
-                        ("delta_bias", delta_bias), ("h0", h0)):
+                        ("delta_bias", delta_bias), ("h0", h0),
+                        ("conv_weight", conv_weight),
+                        ("conv_bias", conv_bias)):
             if t is not None and (t.dtype != torch.float32
                                   or not t.is_contiguous()
                                   or t.device != self.device):
@@ -292,6 +316,13 @@ class SelectiveScan:
             stream = torch.cuda.current_stream(self.device)
         flags = (SSM_DELTA_SOFTPLUS if delta_softplus else 0) | \
             (SSM_WRITE_ZOH if write_zoh else 0)
-        ssm_scan_fwd(self.handle, x, delta, A_log, B, C, D, z, delta_bias,
-                     flags, h0, y, h_last, (b, L, E, N), dtype, stream)
+        if conv_weight is not None:
+            ssm_scan_fwd_conv(self.handle, x, conv_weight, conv_bias,
+                              conv_weight.shape[-1], delta, A_log, B, C, D, z,
+                              delta_bias, flags, h0, y, h_last, (b, L, E, N),
+                              dtype, stream)
+        else:
+            ssm_scan_fwd(self.handle, x, delta, A_log, B, C, D, z,
+                         delta_bias, flags, h0, y, h_last, (b, L, E, N),
+                         dtype, stream)
         return (y, h_last) if return_last_state else y

@@ -191,11 +191,13 @@ __device__ __forceinline__ float2 transpose_reduce2(const float (&p)[2 * NG],
 
 enum { kWalkMain = 0, kWalkCorrect = 1 };
 
-template <class Cfg, bool SPLIT, bool ZOH = false>
+template <class Cfg, bool SPLIT, bool ZOH = false, bool CONV = false>
 __global__ void __launch_bounds__(Cfg::THREADS)
 scan_chunked_kernel(const ScanParams p) {
   static_assert(!ZOH || Cfg::TB == 1,
                 "the zero-order-hold write runs with one time block");
+  static_assert(!CONV || Cfg::TB == 1,
+                "the fused convolution runs with one time block");
   using T = typename Cfg::T;
   constexpr int NG = Cfg::NG, TB = Cfg::TB, K = Cfg::K, TW = Cfg::TW;
   constexpr int CW = Cfg::CW, G = Cfg::G, N = Cfg::N, ESZ = Cfg::ESZ;
@@ -203,6 +205,10 @@ scan_chunked_kernel(const ScanParams p) {
   constexpr unsigned FULL = 0xffffffffu;
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ unsigned s_word;
+  // fused convolution: the last KH inputs of the previous window, per channel
+  // of the tile, for each window parity
+  constexpr int KH = kScanConvMaxWidth - 1;
+  __shared__ float s_halo[CONV ? 2 * KH * G : 1];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q = lane % TB;
@@ -261,6 +267,21 @@ scan_chunked_kernel(const ScanParams p) {
   }
   const float bias = (ch_ok && p.delta_bias) ? p.delta_bias[e] : 0.0f;
   const float Dv = (ch_ok && p.D) ? p.D[e] : 0.0f;
+  // fused convolution weights, right-aligned: cw[kScanConvMaxWidth - 1]
+  // multiplies the newest input, leading taps of a narrower filter are zero
+  float cw[kScanConvMaxWidth] = {};
+  float cbias = 0.0f;
+  if constexpr (CONV) {
+    if (ch_ok) {
+      const int Kw = p.conv_width;
+#pragma unroll
+      for (int k = 0; k < kScanConvMaxWidth; ++k) {
+        const int kk = k - (kScanConvMaxWidth - Kw);
+        cw[k] = kk >= 0 ? p.conv_weight[e * Kw + kk] : 0.0f;
+      }
+      cbias = p.conv_bias ? p.conv_bias[e] : 0.0f;
+    }
+  }
   float2 P01 = make_float2(1.0f, 1.0f), P23 = P01;  // product of retentions
 
   float *const bf_conv = reinterpret_cast<float *>(smem + 2 * Cfg::STAGE_BYTES);
@@ -317,8 +338,23 @@ scan_chunked_kernel(const ScanParams p) {
     constexpr int MODE = decltype(mode_c)::value;
     stage(w_begin, 0);
     cp_async_commit();
+    if constexpr (CONV) {
+      if (MODE == kWalkMain) {
+        // inputs just before the first window (zeros before the sequence)
+        for (int idx = tid; idx < KH * G; idx += THREADS) {
+          const int r = idx / G, ch = idx - (idx / G) * G;
+          const int64_t t = w_begin * TW - KH + r;
+          const int64_t ec = e0 + ch;
+          s_halo[idx] = (t >= 0 && ec < E)
+                            ? Act<T>::load(gx + (b * L + t) * E + ec)
+                            : 0.0f;
+        }
+      }
+    }
     for (int64_t w = w_begin; w < w_end; ++w) {
       const int par = int((w - w_begin) & 1);
+      const int wpar = par;  // window parity (selects the halo)
+      (void)wpar;
       if (w + 1 < w_end) stage(w + 1, par ^ 1);
       cp_async_commit();
       cp_async_wait<1>();
@@ -398,13 +434,33 @@ scan_chunked_kernel(const ScanParams p) {
         const bool full = t0 + TW <= t_end;  // no step of the window is past
         T *const yw = gy + ybase;
 
+        // input of row r of the window; EDGE: r may be before the window
+        auto vat = [&](int r, auto edge_c) -> float {
+          if constexpr (decltype(edge_c)::value)
+            if (r < 0) return s_halo[(wpar * KH + KH + r) * G + cl];
+          return Act<T>::load(
+              reinterpret_cast<const T *>(sX + Cfg::raw_off(r) + cl * ESZ));
+        };
         auto produce2 = [&](int jb, int par, float2 &x2, float2 &z2,
-                            float2 &dd0, float2 &dd1) {
+                            float2 &dd0, float2 &dd1, auto edge_c) {
           const int r0 = jb * BS + 2 * g;
           const int o0 = Cfg::raw_off(r0) + cl * ESZ;
           const int o1 = Cfg::raw_off(r0 + 1) + cl * ESZ;
           x2 = make_float2(Act<T>::load(reinterpret_cast<const T *>(sX + o0)),
                            Act<T>::load(reinterpret_cast<const T *>(sX + o1)));
+          if constexpr (CONV) {
+            if (MODE == kWalkMain) {
+              // x(r) = SiLU(bias + sum_k cw[k] v(r - 3 + k)), rows r0, r0+1
+              const float vm3 = vat(r0 - 3, edge_c), vm2 = vat(r0 - 2, edge_c);
+              const float vm1 = vat(r0 - 1, edge_c);
+              float2 acc = make_float2(cbias, cbias);
+              acc = fma2(make_float2(cw[0], cw[0]), make_float2(vm3, vm2), acc);
+              acc = fma2(make_float2(cw[1], cw[1]), make_float2(vm2, vm1), acc);
+              acc = fma2(make_float2(cw[2], cw[2]), make_float2(vm1, x2.x), acc);
+              acc = fma2(make_float2(cw[3], cw[3]), x2, acc);
+              x2 = silu2(acc);
+            }
+          }
           const float2 v2 = add2(
               make_float2(Act<T>::load(reinterpret_cast<const T *>(sDL + o0)),
                           Act<T>::load(reinterpret_cast<const T *>(sDL + o1))),
@@ -448,7 +504,7 @@ scan_chunked_kernel(const ScanParams p) {
         };
 
         float2 x2, z2, e0, e1;
-        produce2(0, 0, x2, z2, e0, e1);
+        produce2(0, 0, x2, z2, e0, e1, std::true_type());
         __syncwarp();
 #pragma unroll 2
         for (int jb = 0; jb < NBW; ++jb) {
@@ -463,7 +519,10 @@ scan_chunked_kernel(const ScanParams p) {
             dd[1] = e1;
           }
           float2 xn = make_float2(0.f, 0.f), zn = xn, n0 = xn, n1 = xn;
-          if (jb + 1 < NBW) produce2(jb + 1, par ^ 1, xn, zn, n0, n1);
+          // a later block reaches before the window only with 2-step blocks
+          if (jb + 1 < NBW)
+            produce2(jb + 1, par ^ 1, xn, zn, n0, n1,
+                     std::integral_constant<bool, (BS < KH)>());
           float ps[BS];
 #pragma unroll
           for (int s = 0; s < BS; ++s) {
@@ -606,6 +665,17 @@ scan_chunked_kernel(const ScanParams p) {
             }
             finish(r0 + jb * NG + g, transpose_reduce<NG, TB>(ps, g), xs[jb],
                    zs[jb]);
+          }
+        }
+      }
+      if constexpr (CONV) {
+        if (MODE == kWalkMain && w + 1 < w_end) {
+          // the last KH inputs of this window open the next one
+          for (int idx = tid; idx < KH * G; idx += THREADS) {
+            const int r = idx / G, ch = idx - (idx / G) * G;
+            s_halo[((wpar ^ 1) * KH + r) * G + ch] =
+                Act<T>::load(reinterpret_cast<const T *>(
+                    sX + Cfg::raw_off(TW - KH + r) + ch * ESZ));
           }
         }
       }

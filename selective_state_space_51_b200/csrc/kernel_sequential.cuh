@@ -8,7 +8,10 @@
 // runnable CPU code", rows 1, 2 and 5): delta = softplus(raw + bias);
 // a = exp(delta * A) with A = -exp(A_log); h = a * h + delta * B * x;
 // y = sum_n C * h + D * x, read after the update; y *= SiLU(z). With the
-// exact zero-order-hold flag the write is expm1(delta A) / A * B * x.
+// exact zero-order-hold flag the write is expm1(delta A) / A * B * x. With a
+// convolution (row "4. Add causal local context before selecting
+// coefficients") x is SiLU of the causal depthwise convolution of the input,
+// zeros before the first step.
 #pragma once
 
 #include "device_math.cuh"
@@ -40,6 +43,20 @@ scan_sequential_kernel(const ScanParams p) {
       if (p.h0) h[n] = p.h0[(b * E + e) * N + n];
     }
   }
+  // convolution taps right-aligned to the newest input; win holds the
+  // previous kScanConvMaxWidth - 1 inputs, oldest first
+  const bool conv = p.conv_weight != nullptr;
+  float cw[kScanConvMaxWidth] = {};
+  float win[kScanConvMaxWidth - 1] = {};
+  float cbias = 0.0f;
+  if (conv) {
+#pragma unroll
+    for (int k = 0; k < kScanConvMaxWidth; ++k) {
+      const int kk = k - (kScanConvMaxWidth - p.conv_width);
+      cw[k] = kk >= 0 ? p.conv_weight[e * p.conv_width + kk] : 0.0f;
+    }
+    cbias = p.conv_bias ? p.conv_bias[e] : 0.0f;
+  }
   const float bias = p.delta_bias ? p.delta_bias[e] : 0.0f;
   const float Dv = p.D ? p.D[e] : 0.0f;
   const T *x = static_cast<const T *>(p.x);
@@ -54,7 +71,18 @@ scan_sequential_kernel(const ScanParams p) {
     const int64_t r = (b * L + t) * N;
     const float v = Act<T>::load(dl + i) + bias;
     const float step = p.softplus ? softplus(v) : v;
-    const float xv = Act<T>::load(x + i);
+    float xv = Act<T>::load(x + i);
+    if (conv) {
+      float acc = cbias;
+#pragma unroll
+      for (int k = 0; k < kScanConvMaxWidth - 1; ++k)
+        acc = fmaf(cw[k], win[k], acc);
+      acc = fmaf(cw[kScanConvMaxWidth - 1], xv, acc);
+#pragma unroll
+      for (int k = 0; k + 1 < kScanConvMaxWidth - 1; ++k) win[k] = win[k + 1];
+      win[kScanConvMaxWidth - 2] = xv;
+      xv = silu(acc);
+    }
     const float dx = step * xv;
     float acc = 0.0f;
 #pragma unroll

@@ -6,7 +6,8 @@
 namespace ssm {
 
 struct ScanParams {
-  const void *x;             // [b, L, E] activation dtype
+  const void *x;             // [b, L, E] activation dtype (the convolution's
+                             // input v when conv_weight is set)
   const void *delta;         // [b, L, E]
   const float *A_log;        // [E, N]
   const void *B;             // [b, L, N]
@@ -21,6 +22,11 @@ struct ScanParams {
   int dstate;
   int softplus;              // apply softplus to delta + bias
   int write_zoh;             // exact zero-order-hold write (see ssm_scan.h)
+  // Causal depthwise convolution in front of the scan: x = SiLU(conv_bias +
+  // sum_k conv_weight[e, k] v[t - K + 1 + k]), zeros before t = 0.
+  const float *conv_weight;  // [E, K] or nullptr (x is used as it is)
+  const float *conv_bias;    // [E] or nullptr
+  int conv_width;            // K, 1..kScanConvMaxWidth
   // Split sequences (chunked variant): each sequence is cut into `segments`
   // pieces of seg_len steps (a multiple of the window), scanned concurrently
   // from a zero state and joined by a decoupled look-back over per-piece
@@ -37,6 +43,9 @@ struct ScanParams {
   unsigned spin_limit;       // bounded wait: polls before giving up
   unsigned debug;            // kDebug* bits (tests only)
 };
+
+// Widest causal convolution the fused scan takes.
+constexpr int kScanConvMaxWidth = 4;
 
 // Device status codes written to ScanParams::status.
 enum { kStatusOk = 0, kStatusTimeout = 1 };

@@ -129,13 +129,13 @@ int ensure_workspace(ssm_scan_s *h, ssm::ScanParams &p, int64_t tiles,
 // Pieces per sequence: enough that the blocks fill every resident slot once,
 // each piece at least 64 windows long (so the start-up replay after the
 // look-back stays a small fraction), and 1 when channels alone fill the GPU.
-template <class Cfg, bool ZOH>
+template <class Cfg, bool ZOH, bool CONV>
 int64_t auto_segments(const ssm::ScanParams &p, int sm_count) {
   static int per_sm = 0;  // resident blocks per SM for this shape
   if (!per_sm) {
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-            &n, ssm::scan_chunked_kernel<Cfg, true, ZOH>, Cfg::THREADS,
+            &n, ssm::scan_chunked_kernel<Cfg, true, ZOH, CONV>, Cfg::THREADS,
             Cfg::SMEM_BYTES) != cudaSuccess) {
       cudaGetLastError();
       n = 1;
@@ -152,10 +152,10 @@ int64_t auto_segments(const ssm::ScanParams &p, int sm_count) {
   return segs < 2 ? 1 : segs;
 }
 
-template <class Cfg, bool SPLIT, bool ZOH>
+template <class Cfg, bool SPLIT, bool ZOH, bool CONV>
 int launch_kernel(const ssm::ScanParams &p, int64_t blocks, cudaStream_t s) {
   if (blocks > 0x7fffffff) return SSM_ERR_UNSUPPORTED;
-  auto kern = ssm::scan_chunked_kernel<Cfg, SPLIT, ZOH>;
+  auto kern = ssm::scan_chunked_kernel<Cfg, SPLIT, ZOH, CONV>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Cfg::SMEM_BYTES) != cudaSuccess) {
     cudaGetLastError();
@@ -165,12 +165,12 @@ int launch_kernel(const ssm::ScanParams &p, int64_t blocks, cudaStream_t s) {
   return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
-template <class Cfg, bool ZOH = false>
+template <class Cfg, bool ZOH = false, bool CONV = false>
 int launch_chunked(ssm_scan_s *h, ssm::ScanParams &p, int64_t segs_req,
                    cudaStream_t s) {
   const int64_t tiles = (p.dim + Cfg::G - 1) / Cfg::G;
-  int64_t segs =
-      segs_req > 0 ? segs_req : auto_segments<Cfg, ZOH>(p, h->sm_count);
+  int64_t segs = segs_req > 0 ? segs_req
+                              : auto_segments<Cfg, ZOH, CONV>(p, h->sm_count);
   int64_t seg_len = p.seqlen;
   if (segs > 1) {
     const int64_t wins = (p.seqlen + Cfg::TW - 1) / Cfg::TW;
@@ -181,10 +181,11 @@ int launch_chunked(ssm_scan_s *h, ssm::ScanParams &p, int64_t segs_req,
   p.segments = int(segs);
   p.seg_len = seg_len;
   h->last_segments = int(segs);
-  if (segs <= 1) return launch_kernel<Cfg, false, ZOH>(p, p.batch * tiles, s);
+  if (segs <= 1)
+    return launch_kernel<Cfg, false, ZOH, CONV>(p, p.batch * tiles, s);
   const int rc = ensure_workspace(h, p, tiles, segs, s);
   if (rc != SSM_OK) return rc;
-  return launch_kernel<Cfg, true, ZOH>(p, segs * p.batch * tiles, s);
+  return launch_kernel<Cfg, true, ZOH, CONV>(p, segs * p.batch * tiles, s);
 }
 
 // Whether the chunked variant can run these arguments: N of 4, 8 or 16, whole
@@ -208,7 +209,14 @@ int auto_time_blocks(const ssm::ScanParams &, int) { return 1; }
 template <class Cf1, class Cf2>
 int pick(ssm_scan_s *h, ssm::ScanParams &p, int tb, int64_t segs,
          cudaStream_t s) {
-  if (p.write_zoh)  // the zero-order-hold write runs with one time block
+  // the zero-order-hold write and the fused convolution run with one time
+  // block
+  if (p.conv_weight) {
+    if (tb != 1) return SSM_ERR_UNSUPPORTED;
+    return p.write_zoh ? launch_chunked<Cf1, true, true>(h, p, segs, s)
+                       : launch_chunked<Cf1, false, true>(h, p, segs, s);
+  }
+  if (p.write_zoh)
     return tb == 1 ? launch_chunked<Cf1, true>(h, p, segs, s)
                    : SSM_ERR_UNSUPPORTED;
   if (tb == 1) return launch_chunked<Cf1>(h, p, segs, s);
@@ -249,6 +257,81 @@ int launch_step(const ssm::StepParams &p, bool vec, cudaStream_t s) {
   if (groups <= 4) return launch_step_qp<T, 4>(p, vec, s);
   if (groups <= 8) return launch_step_qp<T, 8>(p, vec, s);
   return launch_step_qp<T, 16>(p, vec, s);
+}
+
+// The forward scan behind both entry points; conv_weight == nullptr: x is
+// the scan input as it is.
+int scan_fwd(ssm_scan_s *h, const void *x, const float *conv_weight,
+             const float *conv_bias, int conv_width, const void *delta,
+             const float *A_log, const void *B, const void *C, const float *D,
+             const void *z, const float *delta_bias, uint32_t flags,
+             const float *h0, void *y, float *h_last, ssm_scan_dims dims,
+             int dtype, cudaStream_t s) {
+  // ---- host-side validation: nothing touches the GPU before it passes
+  if (!h || !x || !delta || !A_log || !B || !C || !y) return SSM_ERR_INVALID;
+  if (dims.batch <= 0 || dims.seqlen <= 0 || dims.dim <= 0 || dims.dstate <= 0)
+    return SSM_ERR_INVALID;
+  if (flags & ~uint32_t(SSM_DELTA_SOFTPLUS | SSM_WRITE_ZOH))
+    return SSM_ERR_INVALID;
+  if (conv_weight &&
+      (conv_width < 1 || conv_width > ssm::kScanConvMaxWidth))
+    return SSM_ERR_INVALID;
+  if (dtype != SSM_F32 && dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
+  if (dims.dstate > 64) return SSM_ERR_UNSUPPORTED;
+  int64_t rows = 0, acts = 0, bc = 0, st = 0;
+  if (!mul_ok(dims.batch, dims.seqlen, &rows) ||
+      !mul_ok(rows, dims.dim, &acts) || !mul_ok(rows, dims.dstate, &bc) ||
+      !mul_ok(dims.batch * dims.dim, dims.dstate, &st) ||
+      acts > (int64_t(1) << 56))
+    return SSM_ERR_INVALID;
+  const size_t esz = dtype == SSM_F32 ? 4 : 2;
+  const void *acts_in[] = {x, delta, B, C, z, y};
+  for (const void *p : acts_in)
+    if (p && !aligned(p, esz)) return SSM_ERR_ALIGN;
+  const float *params[] = {A_log, D, delta_bias, h0, h_last, conv_weight,
+                           conv_bias};
+  for (const float *p : params)
+    if (p && !aligned(p, 4)) return SSM_ERR_ALIGN;
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) {
+    cudaGetLastError();
+    return SSM_ERR_CUDA;
+  }
+  if (cur != h->device) return SSM_ERR_INVALID;
+
+  ssm::ScanParams p{};
+  p.x = x; p.delta = delta; p.A_log = A_log; p.B = B; p.C = C;
+  p.D = D; p.z = z; p.delta_bias = delta_bias; p.h0 = h0;
+  p.y = y; p.h_last = h_last;
+  p.batch = dims.batch; p.seqlen = dims.seqlen; p.dim = dims.dim;
+  p.dstate = (int)dims.dstate;
+  p.softplus = (flags & SSM_DELTA_SOFTPLUS) ? 1 : 0;
+  p.write_zoh = (flags & SSM_WRITE_ZOH) ? 1 : 0;
+  p.conv_weight = conv_weight;
+  p.conv_bias = conv_weight ? conv_bias : nullptr;
+  p.conv_width = conv_weight ? conv_width : 0;
+  p.segments = 1;
+
+  int variant = h->variant;
+  const bool chunk_ok = chunked_supported(p, dtype);
+  if (variant == SSM_VARIANT_AUTO)
+    variant = chunk_ok ? SSM_VARIANT_CHUNKED : SSM_VARIANT_SEQUENTIAL;
+  int rc;
+  if (variant == SSM_VARIANT_CHUNKED) {
+    if (!chunk_ok) return SSM_ERR_UNSUPPORTED;
+    const int tb = h->time_blocks ? h->time_blocks
+                                  : auto_time_blocks(p, h->sm_count);
+    rc = dispatch_chunked(h, p, dtype, tb, h->segments, s);
+  } else if (dtype == SSM_F32) {
+    rc = dispatch_sequential<float>(p, s);
+  } else {
+    rc = dispatch_sequential<__nv_bfloat16>(p, s);
+  }
+  if (rc == SSM_OK) {
+    h->last_variant = variant;
+    if (variant != SSM_VARIANT_CHUNKED) h->last_segments = 1;
+  }
+  return rc;
 }
 
 }  // namespace
@@ -423,65 +506,23 @@ int ssm_scan_fwd(ssm_scan_t h, const void *x, const void *delta,
                  const float *D, const void *z, const float *delta_bias,
                  uint32_t flags, const float *h0, void *y, float *h_last,
                  ssm_scan_dims dims, int dtype, struct CUstream_st *stream) {
-  // ---- host-side validation: nothing touches the GPU before it passes
-  if (!h || !x || !delta || !A_log || !B || !C || !y) return SSM_ERR_INVALID;
-  if (dims.batch <= 0 || dims.seqlen <= 0 || dims.dim <= 0 || dims.dstate <= 0)
-    return SSM_ERR_INVALID;
-  if (flags & ~uint32_t(SSM_DELTA_SOFTPLUS | SSM_WRITE_ZOH))
-    return SSM_ERR_INVALID;
-  if (dtype != SSM_F32 && dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
-  if (dims.dstate > 64) return SSM_ERR_UNSUPPORTED;
-  int64_t rows = 0, acts = 0, bc = 0, st = 0;
-  if (!mul_ok(dims.batch, dims.seqlen, &rows) ||
-      !mul_ok(rows, dims.dim, &acts) || !mul_ok(rows, dims.dstate, &bc) ||
-      !mul_ok(dims.batch * dims.dim, dims.dstate, &st) ||
-      acts > (int64_t(1) << 56))
-    return SSM_ERR_INVALID;
-  const size_t esz = dtype == SSM_F32 ? 4 : 2;
-  const void *acts_in[] = {x, delta, B, C, z, y};
-  for (const void *p : acts_in)
-    if (p && !aligned(p, esz)) return SSM_ERR_ALIGN;
-  const float *params[] = {A_log, D, delta_bias, h0, h_last};
-  for (const float *p : params)
-    if (p && !aligned(p, 4)) return SSM_ERR_ALIGN;
-  int cur = -1;
-  if (cudaGetDevice(&cur) != cudaSuccess) {
-    cudaGetLastError();
-    return SSM_ERR_CUDA;
-  }
-  if (cur != h->device) return SSM_ERR_INVALID;
+  return scan_fwd(h, x, nullptr, nullptr, 0, delta, A_log, B, C, D, z,
+                  delta_bias, flags, h0, y, h_last, dims, dtype,
+                  reinterpret_cast<cudaStream_t>(stream));
+}
 
-  ssm::ScanParams p{};
-  p.x = x; p.delta = delta; p.A_log = A_log; p.B = B; p.C = C;
-  p.D = D; p.z = z; p.delta_bias = delta_bias; p.h0 = h0;
-  p.y = y; p.h_last = h_last;
-  p.batch = dims.batch; p.seqlen = dims.seqlen; p.dim = dims.dim;
-  p.dstate = (int)dims.dstate;
-  p.softplus = (flags & SSM_DELTA_SOFTPLUS) ? 1 : 0;
-  p.write_zoh = (flags & SSM_WRITE_ZOH) ? 1 : 0;
-  p.segments = 1;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-
-  int variant = h->variant;
-  const bool chunk_ok = chunked_supported(p, dtype);
-  if (variant == SSM_VARIANT_AUTO)
-    variant = chunk_ok ? SSM_VARIANT_CHUNKED : SSM_VARIANT_SEQUENTIAL;
-  int rc;
-  if (variant == SSM_VARIANT_CHUNKED) {
-    if (!chunk_ok) return SSM_ERR_UNSUPPORTED;
-    const int tb = h->time_blocks ? h->time_blocks
-                                  : auto_time_blocks(p, h->sm_count);
-    rc = dispatch_chunked(h, p, dtype, tb, h->segments, s);
-  } else if (dtype == SSM_F32) {
-    rc = dispatch_sequential<float>(p, s);
-  } else {
-    rc = dispatch_sequential<__nv_bfloat16>(p, s);
-  }
-  if (rc == SSM_OK) {
-    h->last_variant = variant;
-    if (variant != SSM_VARIANT_CHUNKED) h->last_segments = 1;
-  }
-  return rc;
+int ssm_scan_fwd_conv(ssm_scan_t h, const void *v, const float *conv_weight,
+                      const float *conv_bias, int conv_width,
+                      const void *delta, const float *A_log, const void *B,
+                      const void *C, const float *D, const void *z,
+                      const float *delta_bias, uint32_t flags,
+                      const float *h0, void *y, float *h_last,
+                      ssm_scan_dims dims, int dtype,
+                      struct CUstream_st *stream) {
+  if (!conv_weight) return SSM_ERR_INVALID;
+  return scan_fwd(h, v, conv_weight, conv_bias, conv_width, delta, A_log, B,
+                  C, D, z, delta_bias, flags, h0, y, h_last, dims, dtype,
+                  reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

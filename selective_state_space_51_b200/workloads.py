@@ -153,3 +153,16 @@ def make(index: int, seed: Optional[int] = None, batch: Optional[int] = None,
     dev.update(A_log=A_log, D=D, delta_bias=bias, h0=h0)
     return Workload(name=name, batch=b, seqlen=L, dim=E, dstate=N, dtype=act,
                     delta_softplus=True, dev=dev)
+
+
+def conv_params(dim: int, width: int = 4, seed: int = 51100):
+    """Weights [dim, width] and bias [dim] (float32) of a causal depthwise
+    convolution in front of the scan, drawn uniform in +-1/sqrt(width) (the
+    fan-in bound of a freshly initialised depthwise filter), weights first,
+    from PCG64(seed). When a convolution is used, the workload's x array is
+    its input v."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    bound = np.float32(1.0 / np.sqrt(width))
+    w = (rng.random((dim, width), dtype=np.float32) * 2 - 1) * bound
+    bias = (rng.random(dim, dtype=np.float32) * 2 - 1) * bound
+    return np.ascontiguousarray(w), np.ascontiguousarray(bias)
