@@ -86,6 +86,9 @@ class OracleLib:
                                              d, d, d, d, d, d, d,
                                              ctypes.c_int, ctypes.c_int, d, d,
                                              d, ctypes.c_int]
+        lib.ssm_oracle_scan_bwd.restype = ctypes.c_int
+        lib.ssm_oracle_scan_bwd.argtypes = [i64, i64, i64, i64] + [d] * 8 + [
+            ctypes.c_int, ctypes.c_int] + [d] * 12 + [ctypes.c_int]
         lib.ssm_oracle_step.restype = ctypes.c_int
         lib.ssm_oracle_step.argtypes = [i64, i64, i64, i64, d, d, d, d, d, d,
                                         ctypes.c_int, ctypes.c_int, d, d, d, d,
@@ -172,6 +175,38 @@ class OracleLib:
             raise ValueError("oracle rejected its arguments (rc=%d)" % rc)
         return y, h_last
 
+    def scan_bwd(self, x, delta, A_log, B, C, dy, D=None, z=None,
+                 delta_bias=None, delta_softplus=True, h0=None, dh_last=None,
+                 write_zoh=False, nthreads=0):
+        """Gradients of sum(dy * y) + sum(dh_last * h_last) with respect to
+        every input of scan(). Returns a dict: dx, ddelta, dz (or None), dB,
+        dC, dA_log, dD (or None), ddelta_bias (or None), dh0."""
+        xa = np.asarray(x)
+        b, L, E = xa.shape
+        N = np.asarray(A_log).shape[-1]
+        out = {k: np.empty(sh, dtype=np.float64) for k, sh in (
+            ("dx", (b, L, E)), ("ddelta", (b, L, E)), ("dA_log", (E, N)),
+            ("dB", (b, L, N)), ("dC", (b, L, N)), ("dh0", (b, E, N)))}
+        out["dz"] = np.empty((b, L, E)) if z is not None else None
+        out["dD"] = np.empty(E) if D is not None else None
+        out["ddelta_bias"] = np.empty(E) if delta_bias is not None else None
+        rc = self.lib.ssm_oracle_scan_bwd(
+            b, L, E, N, _ptr(_f64(xa, (b, L, E), "x")),
+            _ptr(_f64(delta, (b, L, E), "delta")),
+            _ptr(_f64(A_log, (E, N), "A_log")), _ptr(_f64(B, (b, L, N), "B")),
+            _ptr(_f64(C, (b, L, N), "C")), _ptr(_f64(D, (E,), "D")),
+            _ptr(_f64(z, (b, L, E), "z")),
+            _ptr(_f64(delta_bias, (E,), "delta_bias")),
+            int(bool(delta_softplus)), int(bool(write_zoh)),
+            _ptr(_f64(h0, (b, E, N), "h0")), _ptr(_f64(dy, (b, L, E), "dy")),
+            _ptr(_f64(dh_last, (b, E, N), "dh_last")), _ptr(out["dx"]),
+            _ptr(out["ddelta"]), _ptr(out["dA_log"]), _ptr(out["dB"]),
+            _ptr(out["dC"]), _ptr(out["dD"]), _ptr(out["dz"]),
+            _ptr(out["ddelta_bias"]), _ptr(out["dh0"]), int(nthreads))
+        if rc != 0:
+            raise ValueError("oracle rejected its arguments (rc=%d)" % rc)
+        return out
+
     def step(self, x_new, delta, A_log, B, C, state, conv_state=None,
              conv_weight=None, conv_bias=None, D=None, z=None,
              delta_bias=None, delta_softplus=True, write_zoh=False):
@@ -247,6 +282,17 @@ def scan_conv(v, conv_weight, delta, A_log, B, C, conv_bias=None, D=None,
                              delta_bias=delta_bias,
                              delta_softplus=delta_softplus, h0=h0,
                              write_zoh=write_zoh, nthreads=nthreads)
+
+
+def scan_bwd(x, delta, A_log, B, C, dy, D=None, z=None, delta_bias=None,
+             delta_softplus=True, h0=None, dh_last=None, write_zoh=False,
+             nthreads=0):
+    """Gradients of the scan (see OracleLib.scan_bwd)."""
+    return _load().scan_bwd(x, delta, A_log, B, C, dy, D=D, z=z,
+                            delta_bias=delta_bias,
+                            delta_softplus=delta_softplus, h0=h0,
+                            dh_last=dh_last, write_zoh=write_zoh,
+                            nthreads=nthreads)
 
 
 def step(x_new, delta, A_log, B, C, state, conv_state=None, conv_weight=None,

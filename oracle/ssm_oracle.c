@@ -51,6 +51,7 @@
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
+#include <string.h>
 #ifdef _OPENMP
 #include <omp.h>
 #endif
@@ -306,4 +307,196 @@ int ssm_oracle_scan_conv(int64_t batch, int64_t seqlen, int64_t dim,
                                       NULL, nthreads);
     free(x);
     return rc;
+}
+
+/*
+ * Backward pass of ssm_oracle_scan_ex: the gradients of
+ *   loss = sum dy_out * y_out + sum dh_last * h_last
+ * with respect to every input, by reverse-mode differentiation of the same
+ * recurrence ("Mamba: Linear-Time Sequence Modeling with Selective State
+ * Spaces", www.abhik.ai/papers/mamba, rows "1. Produce coefficients from the
+ * locally mixed input", "2. Retain, write and read each channel's state" and
+ * "5. Put the selective operator inside the complete mixer"; the pages
+ * describe training through the scan by recomputing the states on the way
+ * back instead of storing them, section "Compose the updates instead of
+ * waiting for every state").
+ *
+ * Per (b, e), with s = step size, a_n = exp(s A_n), w_n the write, the
+ * adjoint lam_n = d loss / d h_t[n] runs backwards in time:
+ *   g = dy_out[t]; dy = g SiLU(z) (g without a gate);
+ *   dz = g (C.h + D x) SiLU'(z);
+ *   lam_n += dy C[n];  dC[n] += dy h_t[n];  dD += dy x;  dx += dy D;
+ *   dw_n = lam_n;  da_n = lam_n h_{t-1}[n];
+ *   write s B x:          ds += sum lam B x;  dB += lam s x;  dx += sum lam s B;
+ *   write expm1(sA)/A B x (f = expm1(sA)/A, df/ds = a, df/dA = (s a - f)/A):
+ *                         ds += sum lam B x a; dB += lam f x; dx += sum lam f B;
+ *                         dA += lam B x (s a - f) / A;
+ *   retention:            ds += sum da a A;  dA += da a s;
+ *   lam_n <- lam_n a_n    (on to h_{t-1});
+ *   draw = ds sigmoid(raw + bias) (ds without softplus); dbias += draw;
+ * and at the start dh0 = lam. Finally dA_log = dA A (A = -exp(A_log)).
+ * The states h_t are recomputed forward per channel first.
+ *
+ * Outputs (all written; dB, dC, dA_log, dD, ddelta_bias are sums):
+ *   dx, ddelta, dz [batch, seqlen, dim]; dB, dC [batch, seqlen, dstate];
+ *   dA_log [dim, dstate]; dD, ddelta_bias [dim]; dh0 [batch, dim, dstate].
+ * dz may be NULL when z is; dD when D is; ddelta_bias when delta_bias is;
+ * dh0 may be NULL. dh_last may be NULL (zero).
+ */
+int ssm_oracle_scan_bwd(int64_t batch, int64_t seqlen, int64_t dim,
+                        int64_t dstate, const double *x, const double *delta,
+                        const double *A_log, const double *B, const double *C,
+                        const double *D, const double *z,
+                        const double *delta_bias, int delta_softplus,
+                        int write_zoh, const double *h0, const double *dy_out,
+                        const double *dh_last, double *dx, double *ddelta,
+                        double *dA_log, double *dB, double *dC, double *dD,
+                        double *dz, double *ddelta_bias, double *dh0,
+                        int nthreads)
+{
+    if (!x || !delta || !A_log || !B || !C || !dy_out || !dx || !ddelta ||
+        !dA_log || !dB || !dC)
+        return -1;
+    if ((z && !dz) || (D && !dD) || (delta_bias && !ddelta_bias))
+        return -1;
+    if (batch <= 0 || seqlen <= 0 || dim <= 0 || dstate <= 0)
+        return -1;
+    const int64_t L = seqlen, E = dim, N = dstate;
+    memset(dB, 0, (size_t)(batch * L * N) * sizeof(double));
+    memset(dC, 0, (size_t)(batch * L * N) * sizeof(double));
+    memset(dA_log, 0, (size_t)(E * N) * sizeof(double));
+    if (dD)
+        memset(dD, 0, (size_t)E * sizeof(double));
+    if (ddelta_bias)
+        memset(ddelta_bias, 0, (size_t)E * sizeof(double));
+#ifdef _OPENMP
+    if (nthreads <= 0)
+        nthreads = omp_get_max_threads();
+#else
+    (void)nthreads;
+#endif
+    int fail = 0;
+    for (int64_t b = 0; b < batch; ++b) {
+#ifdef _OPENMP
+#pragma omp parallel num_threads(nthreads)
+#endif
+        {
+            /* private sums over channels of dB and dC for this batch row */
+            double *pB = (double *)calloc((size_t)(L * N), sizeof(double));
+            double *pC = (double *)calloc((size_t)(L * N), sizeof(double));
+            double *hs = (double *)malloc((size_t)((L + 1) * N) * sizeof(double));
+            double *A = (double *)malloc((size_t)N * sizeof(double));
+            double *dA = (double *)malloc((size_t)N * sizeof(double));
+            double *lam = (double *)malloc((size_t)N * sizeof(double));
+            if (!pB || !pC || !hs || !A || !dA || !lam) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+                fail = 1;
+            } else {
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 1)
+#endif
+                for (int64_t c = 0; c < E; ++c) {
+                    const double bias = delta_bias ? delta_bias[c] : 0.0;
+                    for (int64_t n = 0; n < N; ++n) {
+                        A[n] = -exp(A_log[c * N + n]);
+                        dA[n] = 0.0;
+                        hs[n] = h0 ? h0[(b * E + c) * N + n] : 0.0;
+                    }
+                    /* forward: hs[(t + 1) N + n] = h_t[n] */
+                    for (int64_t t = 0; t < L; ++t) {
+                        const int64_t i = (b * L + t) * E + c;
+                        const int64_t r = (b * L + t) * N;
+                        const double v = delta[i] + bias;
+                        const double s = delta_softplus ? softplus_default(v) : v;
+                        for (int64_t n = 0; n < N; ++n) {
+                            const double f =
+                                write_zoh ? zoh_factor(s, A[n]) : s;
+                            hs[(t + 1) * N + n] = exp(s * A[n]) * hs[t * N + n] +
+                                                  f * B[r + n] * x[i];
+                        }
+                    }
+                    for (int64_t n = 0; n < N; ++n)
+                        lam[n] = dh_last ? dh_last[(b * E + c) * N + n] : 0.0;
+                    double sum_dD = 0.0, sum_dbias = 0.0;
+                    for (int64_t t = L - 1; t >= 0; --t) {
+                        const int64_t i = (b * L + t) * E + c;
+                        const int64_t r = (b * L + t) * N;
+                        const double v = delta[i] + bias;
+                        const double s = delta_softplus ? softplus_default(v) : v;
+                        const double xv = x[i];
+                        const double *h = hs + (t + 1) * N;
+                        const double *hp = hs + t * N;
+                        const double g = dy_out[i];
+                        double dy = g;
+                        if (z) {
+                            double pre = D ? D[c] * xv : 0.0;
+                            for (int64_t n = 0; n < N; ++n)
+                                pre += C[r + n] * h[n];
+                            const double sg = 1.0 / (1.0 + exp(-z[i]));
+                            dy = g * z[i] * sg;
+                            dz[i] = g * pre * sg * (1.0 + z[i] * (1.0 - sg));
+                        }
+                        double dxv = D ? dy * D[c] : 0.0;
+                        if (D)
+                            sum_dD += dy * xv;
+                        double ds = 0.0;
+                        for (int64_t n = 0; n < N; ++n) {
+                            pC[t * N + n] += dy * h[n];
+                            lam[n] += dy * C[r + n];
+                            const double a = exp(s * A[n]);
+                            const double da = lam[n] * hp[n];
+                            if (write_zoh) {
+                                const double f = zoh_factor(s, A[n]);
+                                ds += lam[n] * B[r + n] * xv * a;
+                                pB[t * N + n] += lam[n] * f * xv;
+                                dxv += lam[n] * f * B[r + n];
+                                dA[n] += lam[n] * B[r + n] * xv *
+                                         (s * a - f) / A[n];
+                            } else {
+                                ds += lam[n] * B[r + n] * xv;
+                                pB[t * N + n] += lam[n] * s * xv;
+                                dxv += lam[n] * s * B[r + n];
+                            }
+                            ds += da * a * A[n];
+                            dA[n] += da * a * s;
+                            lam[n] *= a;
+                        }
+                        const double draw =
+                            delta_softplus ? ds / (1.0 + exp(-v)) : ds;
+                        ddelta[i] = draw;
+                        sum_dbias += draw;
+                        dx[i] = dxv;
+                    }
+                    if (dh0)
+                        for (int64_t n = 0; n < N; ++n)
+                            dh0[(b * E + c) * N + n] = lam[n];
+                    /* channel c is this thread's alone within batch row b */
+                    for (int64_t n = 0; n < N; ++n)
+                        dA_log[c * N + n] += dA[n] * A[n];
+                    if (dD)
+                        dD[c] += sum_dD;
+                    if (ddelta_bias)
+                        ddelta_bias[c] += sum_dbias;
+                }
+#ifdef _OPENMP
+#pragma omp critical
+#endif
+                {
+                    for (int64_t k = 0; k < L * N; ++k) {
+                        dB[b * L * N + k] += pB[k];
+                        dC[b * L * N + k] += pC[k];
+                    }
+                }
+            }
+            free(pB);
+            free(pC);
+            free(hs);
+            free(A);
+            free(dA);
+            free(lam);
+        }
+    }
+    return fail ? -1 : 0;
 }

@@ -680,9 +680,68 @@ def pin_step_size(o):
         prev = cur
 
 
+# ---------------------------------------------------------------- backward
+def pin_backward_finite_differences(o):
+    """Every gradient of the backward oracle equals a central finite
+    difference of the (pinned) forward oracle.
+
+    The loss is sum(dy * y) + sum(dh * h_last) for random dy, dh; each input
+    entry is moved by +-eps and the loss recomputed by the forward oracle
+    ([abhik] rows 1, 2 and 5 and "Compose the updates instead of waiting for
+    every state", which trains through the scan). Central differences are
+    exact to O(eps^2) ~ 1e-12 here, so a dropped term, a wrong sign or a
+    transposed index shows as an O(1e-2..1) mismatch. Covered: both writes,
+    gate on and off, softplus on and off, with and without D and the bias.
+    """
+    variants = [dict(write_zoh=False), dict(write_zoh=True),
+                dict(write_zoh=False, gate=False, D=False, bias=False),
+                dict(write_zoh=True, softplus=False)]
+    for k, var in enumerate(variants):
+        zoh = var["write_zoh"]
+        softplus = var.get("softplus", True)
+        b, L, E, N = 2, 6, 3, 3
+        case = random_case(71 + k, b, L, E, N, gate=var.get("gate", True),
+                           D=var.get("D", True), bias=var.get("bias", True))
+        if not softplus:   # positive raw steps
+            case["delta"] = np.abs(case["delta"]) * 0.5 + 0.05
+            case["delta_bias"] = None
+        rng = np.random.default_rng(90 + k)
+        dy = rng.standard_normal((b, L, E))
+        dh = rng.standard_normal((b, E, N))
+
+        def loss(c):
+            y, h = o.scan(**c, delta_softplus=softplus, write_zoh=zoh)
+            return float(np.sum(dy * y) + np.sum(dh * h))
+
+        g = o.scan_bwd(case["x"], case["delta"], case["A_log"], case["B"],
+                       case["C"], dy, D=case["D"], z=case["z"],
+                       delta_bias=case["delta_bias"], delta_softplus=softplus,
+                       h0=case["h0"], dh_last=dh, write_zoh=zoh)
+        names = {"x": "dx", "delta": "ddelta", "A_log": "dA_log", "B": "dB",
+                 "C": "dC", "D": "dD", "z": "dz", "delta_bias": "ddelta_bias",
+                 "h0": "dh0"}
+        for key, gname in names.items():
+            if case[key] is None:
+                assert g[gname] is None or gname == "dh0", gname
+                continue
+            arr = case[key]
+            fd = np.empty_like(arr)
+            for idx in np.ndindex(arr.shape):
+                eps = 1e-6 * max(1.0, abs(arr[idx]))
+                c1 = dict(case)
+                c1[key] = arr.copy()
+                c1[key][idx] += eps
+                up = loss(c1)
+                c1[key][idx] -= 2 * eps
+                fd[idx] = (up - loss(c1)) / (2 * eps)
+            _close(g[gname], fd, 1e-6, 1e-6,
+                   "backward %s (variant %d)" % (gname, k))
+
+
 ALL_PINS = (pin_associative_prefix, pin_lti_convolution, pin_forgetting,
             pin_freezing, pin_retention_bounds, pin_continuation,
             pin_decode_step, pin_linearity, pin_independence, pin_degenerate,
             pin_step_size, pin_zoh_lti, pin_zoh_fixed_point, pin_zoh_small_step,
             pin_step_matches_scan, pin_step_causal_convolution,
-            pin_step_conv_feeds_scan, pin_scan_conv)
+            pin_step_conv_feeds_scan, pin_scan_conv,
+            pin_backward_finite_differences)

@@ -37,6 +37,17 @@ MUTANTS = [
     ("decode write uses the raw input, not the convolved one",
      [("* B[b * dstate + n]\n                    * xv;",
        "* B[b * dstate + n]\n                    * x_new[i];")]),
+    ("backward adjoint not carried through the retention",
+     [("                            lam[n] *= a;\n", "")]),
+    ("backward dB without x",
+     [("pB[t * N + n] += lam[n] * s * xv;", "pB[t * N + n] += lam[n] * s;")]),
+    ("backward step gradient without the softplus slope",
+     [("delta_softplus ? ds / (1.0 + exp(-v)) : ds;", "ds;")]),
+    ("backward gate gradient without the SiLU slope",
+     [("dz[i] = g * pre * sg * (1.0 + z[i] * (1.0 - sg));",
+       "dz[i] = g * pre * sg;")]),
+    ("backward readout gradient uses the previous state",
+     [("pC[t * N + n] += dy * h[n];", "pC[t * N + n] += dy * hp[n];")]),
     ("scan convolution reads the future",
      [("const int64_t s = t - width + 1 + k;", "const int64_t s = t + k;")]),
     ("scan convolution without SiLU",
