@@ -19,7 +19,9 @@ algorithmic traffic and the fraction of the min(HBM, SFU-exp) roofline:
 T_roof = max(bytes / HBM peak, exps / SFU peak), fraction = T_roof / T.
 `--impl reference` times the float64 CPU oracle instead (rank 0 only).
 
-Two more operations print a line of the same form: `--op conv` times the scan
+`--op bwd` times the backward pass (ssm_scan_bwd: a forward that writes a
+state checkpoint every 16 steps, then the reverse sweep) on the same
+workload. Two more operations print a line of the same form: `--op conv` times the scan
 with the causal depthwise convolution (width 4) + SiLU fused in front
 (ssm_scan_fwd_conv, same workload and roofline), and `--op step` times one
 batched decode step (ssm_scan_step: conv buffer shift, conv + SiLU, state
@@ -274,6 +276,7 @@ class ScanOp:
         import torch
         from selective_state_space_51_b200 import workloads as W
         self.name = args.op
+        self.launches_per_step = 1
         self.wl = wl = W.make(plan["shape"], seed=plan["seed"])
         self.t = _to_device(wl.dev, dev)
         self.conv = None
@@ -311,6 +314,7 @@ class StepOp:
         import torch
         from selective_state_space_51_b200 import workloads as W
         self.name = "step"
+        self.launches_per_step = 1
         wl = W.make(plan["shape"], seed=plan["seed"], batch=DECODE_BATCH,
                     seqlen=1, with_h0=True)
         self.wl = wl
@@ -345,6 +349,46 @@ class StepOp:
         return (self.y,)
 
 
+class BwdOp:
+    """One backward pass (training forward with checkpoints + reverse
+    sweep) per step, for seeded incoming gradients."""
+
+    def __init__(self, args, plan, dev, scan):
+        import torch
+        from selective_state_space_51_b200 import workloads as W
+        self.name = "bwd"
+        self.launches_per_step = 2   # checkpointing forward, reverse sweep
+        self.wl = wl = W.make(plan["shape"], seed=plan["seed"])
+        d = dict(wl.dev)
+        rng = np.random.Generator(np.random.PCG64(plan["seed"] + 7))
+        dy = rng.standard_normal((wl.batch, wl.seqlen, wl.dim),
+                                 dtype=np.float32)
+        d["dy"] = W.round_to_bf16_bits(dy) if wl.dtype == W.BF16 else dy
+        self.t = _to_device(d, dev)
+        self.scan = scan
+        self.per_step_in = ("x", "delta", "z", "B", "C", "h0", "dy")
+        self.units = wl.elements
+        act = 4 if wl.dtype == "f32" else 2
+        b, L, E, N = wl.batch, wl.seqlen, wl.dim, wl.dstate
+        gated = wl.dev["z"] is not None
+        # inputs once (x, raw step, z, dy, B, C), gradients once (dx, d raw,
+        # dz in the activation type; dB, dC float32), parameters
+        self.nbytes = ((3 + gated) * b * L * E * act + 2 * b * L * N * act
+                       + (2 + gated) * b * L * E * act + 2 * b * L * N * 4
+                       + 2 * E * N * 4 + 4 * E * 4)
+        self.grads = None
+        self.workload = W.shape_description(args.shape) + "; backward"
+
+    def run(self, t, stream):
+        self.grads = self.scan.backward(
+            t["x"], t["delta"], t["A_log"], t["B"], t["C"], t["dy"],
+            D=t["D"], z=t["z"], delta_bias=t["delta_bias"], h0=t["h0"],
+            stream=stream)
+
+    def outputs(self):
+        return tuple(v for v in self.grads.values() if v is not None)
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -364,7 +408,8 @@ def run_gpu(args):
 
     plan = shard_for_rank(rank, world, args.shape)
     scan = S.SelectiveScan(local)
-    op = (StepOp if args.op == "step" else ScanOp)(args, plan, dev, scan)
+    op = {"step": StepOp, "bwd": BwdOp}.get(args.op, ScanOp)(args, plan, dev,
+                                                              scan)
     t = op.t
     stream = torch.cuda.current_stream(dev)
 
@@ -402,7 +447,7 @@ def run_gpu(args):
     kernel_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends))
     total_ms = max_over_ranks(local_ms, dist if world > 1 else None, dev)
     kernel_ms = max_over_ranks(kernel_ms, dist if world > 1 else None, dev)
-    variant = scan.last_variant() if op.name != "step" else (0, 0)
+    variant = scan.last_variant() if op.name in ("scan", "conv") else (0, 0)
 
     # ---- end to end through the public API with pinned host buffers
     if args.no_e2e:
@@ -507,9 +552,14 @@ def _finish(args, op, world, rank, local, dev, dist, scan, clocks, total_ms,
                 {"value": world * units / (e2e_ms * 1e-3), "unit": unit,
                  "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                  "ms_per_step": e2e_ms}),
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * op.launches_per_step,
         "clocks": clk,
     }
+    if op.name == "bwd":
+        line["roofline"]["peak_note"] += (
+            "; one retention exp per element counted (the pass evaluates "
+            "three: the checkpointing forward, the window recompute and the "
+            "reverse sweep)")
     if op.name != "step":
         line["roofline_min_hbm_sfu"] = {
             "t_hbm_us": t_hbm * 1e6, "t_sfu_us_at_max_clock": t_sfu * 1e6,
@@ -518,7 +568,8 @@ def _finish(args, op, world, rank, local, dev, dist, scan, clocks, total_ms,
             "hbm_peak_gbs": peaks["hbm_gbs"], "hbm_source": peaks["source"],
             "frac_at_8tbs_hbm": max(nbytes / (HBM_NOMINAL_GBS * 1e9), t_sfu)
             / (kernel_ms * 1e-3)}
-        line["kernel"] = {"variant": variant[0], "segments": variant[1]}
+        if op.name != "bwd":
+            line["kernel"] = {"variant": variant[0], "segments": variant[1]}
     if (rank == 0 and world == 1 and not args.no_cpu_baseline
             and op.name == "scan"):
         line["cpu_baseline"] = cpu_oracle_rate(wl, args.reference_seconds)
@@ -539,9 +590,11 @@ def main(argv=None):
     ap.add_argument("--shape", type=int, default=3,
                     help="workload shape index (default 3: Mamba-2.8B layer)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--op", choices=["scan", "conv", "step"], default="scan",
+    ap.add_argument("--op", choices=["scan", "conv", "step", "bwd"],
+                    default="scan",
                     help="scan (default), the scan with the fused "
-                         "convolution, or the batched decode step")
+                         "convolution, the batched decode step, or the "
+                         "backward pass")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--reference-seconds", type=float, default=10.0,
                     help="CPU seconds of the oracle sample in cpu_baseline")

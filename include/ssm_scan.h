@@ -176,6 +176,46 @@ SSM_API int ssm_scan_fwd_conv(ssm_scan_t h, const void *v,
                               struct CUstream_st *stream);
 
 /*
+ * ssm_scan_bwd: the backward pass of ssm_scan_fwd: the gradients of
+ *     loss = sum(dy * y) + sum(dh_last * h_last)
+ * with respect to every input, by reverse-mode differentiation of the
+ * recurrence ("Mamba: Linear-Time Sequence Modeling with Selective State
+ * Spaces", www.abhik.ai/papers/mamba, section "Original paper, equations and
+ * runnable CPU code", rows 1, 2 and 5; the states are recomputed on the way
+ * back rather than stored, as section "Compose the updates instead of
+ * waiting for every state" describes). Two launches on `stream`: the forward
+ * with a state checkpoint every 16 steps into a workspace the handle grows
+ * (b * ceil(L / 16) * dim * dstate floats; SSM_ERR_NOMEM if it cannot), then
+ * a reverse sweep from those checkpoints.
+ *   inputs     : as ssm_scan_fwd (x, delta, A_log, B, C, D, z, delta_bias,
+ *                flags, h0); dy [batch, seqlen, dim] activation dtype,
+ *                required; dh_last [batch, dim, dstate] float32 or NULL (0).
+ *   dx, ddelta : [batch, seqlen, dim] activation dtype, required; ddelta is
+ *                the gradient of the raw step (before bias and softplus).
+ *   dz         : [batch, seqlen, dim] activation dtype; required with z.
+ *   dB, dC     : [batch, seqlen, dstate] float32, required (sums over the
+ *                channels).
+ *   dA_log     : [dim, dstate] float32, required (sum over the batch).
+ *   dD, ddelta_bias : [dim] float32; required with D / delta_bias.
+ *   dh0        : [batch, dim, dstate] float32 or NULL (not written).
+ * The summed outputs are cleared by the call. dstate must be 4, 8 or 16
+ * (8 or 16 for bfloat16), dim * element size a multiple of 16 bytes, and x,
+ * delta, z, dy, B, C, A_log, h0, dh_last, dh0 16-byte aligned
+ * (SSM_ERR_UNSUPPORTED / SSM_ERR_ALIGN otherwise). Outputs must not overlap
+ * inputs. Other errors as for ssm_scan_fwd.
+ */
+SSM_API int ssm_scan_bwd(ssm_scan_t h, const void *x, const void *delta,
+                         const float *A_log, const void *B, const void *C,
+                         const float *D, const void *z,
+                         const float *delta_bias, uint32_t flags,
+                         const float *h0, const void *dy,
+                         const float *dh_last, void *dx, void *ddelta,
+                         float *dA_log, float *dB, float *dC, float *dD,
+                         void *dz, float *ddelta_bias, float *dh0,
+                         ssm_scan_dims dims, int dtype,
+                         struct CUstream_st *stream);
+
+/*
  * ssm_scan_set_variant: force a kernel variant for later calls on this
  * handle (SSM_VARIANT_*), or SSM_VARIANT_AUTO to choose by shape.
  * `segments` > 1 asks the chunked variant to split every sequence into that

@@ -78,6 +78,9 @@ def library() -> ctypes.CDLL:
                                               vp, vp, vp, vp, u32, vp, vp, vp,
                                               ssm_scan_dims, i32, vp]
             lib.ssm_scan_fwd_conv.restype = i32
+            lib.ssm_scan_bwd.argtypes = [vp] * 9 + [u32] + [vp] * 12 + [
+                ssm_scan_dims, i32, vp]
+            lib.ssm_scan_bwd.restype = i32
             lib.ssm_scan_set_variant.argtypes = [vp, i32, i32]
             lib.ssm_scan_set_variant.restype = i32
             lib.ssm_scan_last_variant.argtypes = [vp, ctypes.POINTER(i32),
@@ -185,6 +188,21 @@ def ssm_scan_fwd_conv(h, v, conv_weight, conv_bias, conv_width, delta, A_log,
     return _check(rc, "ssm_scan_fwd_conv") if check else rc
 
 
+def ssm_scan_bwd(h, x, delta, A_log, B, C, D, z, delta_bias, flags, h0, dy,
+                 dh_last, dx, ddelta, dA_log, dB, dC, dD, dz, ddelta_bias,
+                 dh0, dims, dtype, stream=None, check=True) -> int:
+    """Call ssm_scan_bwd (gradients of the scan; see include/ssm_scan.h)."""
+    if not isinstance(dims, ssm_scan_dims):
+        dims = ssm_scan_dims(*[int(d) for d in dims])
+    rc = library().ssm_scan_bwd(
+        h, _ptr(x), _ptr(delta), _ptr(A_log), _ptr(B), _ptr(C), _ptr(D),
+        _ptr(z), _ptr(delta_bias), int(flags), _ptr(h0), _ptr(dy),
+        _ptr(dh_last), _ptr(dx), _ptr(ddelta), _ptr(dA_log), _ptr(dB),
+        _ptr(dC), _ptr(dD), _ptr(dz), _ptr(ddelta_bias), _ptr(dh0), dims,
+        int(dtype), _stream(stream))
+    return _check(rc, "ssm_scan_bwd") if check else rc
+
+
 def ssm_scan_step(h, x_new, conv_state, conv_weight, conv_bias, conv_width,
                   delta, delta_bias, A_log, B, C, D, z, flags, state, y, dims,
                   dtype, stream=None, check=True) -> int:
@@ -254,6 +272,42 @@ class SelectiveScan:
         if stream is None:
             stream = torch.cuda.current_stream(self.device)
         return ssm_scan_sync_status(self.handle, stream)
+
+    def backward(self, x, delta, A_log, B, C, dy, D=None, z=None,
+                 delta_bias=None, delta_softplus=True, h0=None, dh_last=None,
+                 write_zoh=False, stream=None):
+        """Gradients of sum(dy * y) + sum(dh_last * h_last) for the scan of
+        these inputs. Returns a dict: dx, ddelta, dz (activation dtype; dz
+        None without z), dB, dC, dA_log, dD, ddelta_bias, dh0 (float32; dD /
+        ddelta_bias None without D / delta_bias)."""
+        import torch
+        if x.dtype == torch.float32:
+            dtype = SSM_F32
+        elif x.dtype == torch.bfloat16:
+            dtype = SSM_BF16
+        else:
+            raise TypeError("activations must be float32 or bfloat16")
+        b, L, E = x.shape
+        N = A_log.shape[-1]
+        f32 = dict(dtype=torch.float32, device=self.device)
+        g = {"dx": torch.empty_like(x), "ddelta": torch.empty_like(x),
+             "dz": torch.empty_like(x) if z is not None else None,
+             "dB": torch.empty((b, L, N), **f32),
+             "dC": torch.empty((b, L, N), **f32),
+             "dA_log": torch.empty((E, N), **f32),
+             "dD": torch.empty((E,), **f32) if D is not None else None,
+             "ddelta_bias": torch.empty((E,), **f32)
+             if delta_bias is not None else None,
+             "dh0": torch.empty((b, E, N), **f32)}
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device)
+        flags = (SSM_DELTA_SOFTPLUS if delta_softplus else 0) | \
+            (SSM_WRITE_ZOH if write_zoh else 0)
+        ssm_scan_bwd(self.handle, x, delta, A_log, B, C, D, z, delta_bias,
+                     flags, h0, dy, dh_last, g["dx"], g["ddelta"], g["dA_log"],
+                     g["dB"], g["dC"], g["dD"], g["dz"], g["ddelta_bias"],
+                     g["dh0"], (b, L, E, N), dtype, stream)
+        return g
 
     def step(self, x_new, delta, A_log, B, C, state, conv_state=None,
              conv_weight=None, conv_bias=None, D=None, z=None,

@@ -137,6 +137,52 @@ __device__ __forceinline__ float2 silu2(float2 z) {
   return mul2(z, make_float2(rcp(d.x), rcp(d.y)));
 }
 
+// tanh on the SFU (one MUFU.TANH; relative error about 2^-11).
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Cheaper forms for bfloat16 activations, whose inputs already carry a
+// relative rounding of 2^-9:
+// softplus as log2(1 + 2^(v log2 e)) ln 2 (2 MUFU, no series). Rounding
+// 1 + e^v and the SFU log cost at most ~3e-7 absolute, which is what is left
+// of a very negative v's e^v; PyTorch's threshold (v above 20) is kept.
+__device__ __forceinline__ float2 softplus2_fast(float2 v) {
+  const float2 e = mul2(v, make_float2(kLog2e, kLog2e));
+  const float2 w = add2(make_float2(ex2(e.x), ex2(e.y)),
+                        make_float2(1.0f, 1.0f));
+  const float2 r =
+      mul2(make_float2(lg2(w.x), lg2(w.y)), make_float2(kLn2, kLn2));
+  return make_float2(v.x > 20.0f ? v.x : r.x, v.y > 20.0f ? v.y : r.y);
+}
+
+// SiLU as h + h tanh(h), h = z/2 (z sigmoid(z) with sigmoid(z) =
+// (1 + tanh(z/2)) / 2): 1 MUFU, absolute error of the sigmoid below 2.5e-4.
+__device__ __forceinline__ float2 silu2_fast(float2 z) {
+  const float2 h = mul2(z, make_float2(0.5f, 0.5f));
+  return fma2(h, make_float2(tanh_approx(h.x), tanh_approx(h.y)), h);
+}
+
+// The step-size softplus and the SiLU the chunked kernel applies to packed
+// pairs: exact-rounding-order forms for float32 activations, the cheaper
+// forms above for bfloat16.
+template <typename T> struct PairMath {
+  static __device__ __forceinline__ float2 softplus(float2 v) {
+    return softplus2(v);
+  }
+  static __device__ __forceinline__ float2 silu(float2 z) { return silu2(z); }
+};
+template <> struct PairMath<__nv_bfloat16> {
+  static __device__ __forceinline__ float2 softplus(float2 v) {
+    return softplus2_fast(v);
+  }
+  static __device__ __forceinline__ float2 silu(float2 z) {
+    return silu2_fast(z);
+  }
+};
+
 // Exact zero-order-hold write factor expm1(z) / A, z = d A, for one state:
 // given zl = z log2(e) (so a = 2^zl) and invA = 1/A. For |z| < 1/8 it is
 // d phi(z) with phi(z) = (e^z - 1)/z = 1 + z/2 + z^2/6 + z^3/24 + z^4/120 +

@@ -1,0 +1,369 @@
+// Backward pass of the selective scan: the reverse sweep.
+//
+// Page "Mamba: Linear-Time Sequence Modeling with Selective State Spaces"
+// (www.abhik.ai/papers/mamba), section "Original paper, equations and
+// runnable CPU code", rows 1, 2 and 5 define the forward recurrence; section
+// "Compose the updates instead of waiting for every state" trains through it
+// by recomputing states on the way back instead of storing them. With step
+// size s, retention a_n = exp(s A_n), write w_n and the adjoint
+// lam_n = d loss / d h_t[n], going backwards in time:
+//   dy = g SiLU(z) (g = incoming gradient of the output), dz = g pre SiLU'(z)
+//   with pre = C.h_t + D x;
+//   lam += dy C;  dC[t, n] += dy h_t;  dD += dy x;  dx = dy D + sum lam f B;
+//   ds = sum lam B x (f = s) or sum lam B x a (f = expm1(s A)/A)
+//        + sum lam h_{t-1} a A;
+//   dA += lam h_{t-1} a s  (+ lam B x (s a - f)/A for the zero-order hold);
+//   dB[t, n] += lam f x;  lam <- lam a;  d raw = ds sigmoid(raw + bias).
+//
+// A thread block owns (batch row, G-channel tile) and the same (c, g) lanes
+// as the forward kernel (NG lanes per channel, 4 states per lane). It walks
+// windows of 16 steps from the last to the first. For each window:
+//   1. the x, raw step, z, incoming-gradient, B and C tiles arrive by
+//      cp.async (the previous window's are already in flight);
+//   2. a pre-pass forms each (t, e)'s step size, x, dy, gate slope and
+//      softplus slope once, in shared memory;
+//   3. every lane recomputes its 4 states through the window from the
+//      forward's checkpoint (the state before the window), keeping them in
+//      shared memory;
+//   4. the reverse sweep updates lam in registers; per-channel sums over a
+//      channel's NG lanes are a shuffle butterfly, and the sums of dB and dC
+//      over the tile's channels a transposing butterfly over the warp's
+//      channels followed by shared-memory accumulation across warps, added to
+//      HBM once per (t, n) and block.
+#pragma once
+
+#include "kernel_chunked.cuh"
+
+namespace ssm {
+
+struct BwdParams {
+  const void *x, *delta, *z, *dy, *B, *C;  // activation dtype
+  const float *A_log, *D, *delta_bias, *h0, *dh_last;
+  const float *ckpt;  // [b, ceil(L / 16), E, N]: state before step 16 k
+  void *dx, *ddelta, *dz;  // [b, L, E] activation dtype (dz: with z only)
+  float *dB, *dC;          // [b, L, N], summed into (zero before the launch)
+  float *dA_log;           // [E, N], summed into
+  float *dD, *ddelta_bias;  // [E], summed into (with D / delta_bias only)
+  float *dh0;              // [b, E, N] or nullptr
+  int64_t batch, seqlen, dim;
+  int dstate;
+  int softplus;
+};
+
+template <typename T, int NG, int NW>
+struct BwdCfg {
+  static constexpr int N = 4 * NG, CW = 32 / NG, G = CW * NW;
+  static constexpr int THREADS = 32 * NW, TW = kCkptSteps;
+  static constexpr int ESZ = sizeof(T);
+  // raw tiles of one stage: x, raw step, z, dy [TW][G] and B, C [TW][N]
+  static constexpr int ACT_BYTES = TW * G * ESZ;
+  static constexpr int BC_BYTES = TW * N * ESZ;
+  static constexpr int STAGE = 4 * ACT_BYTES + 2 * BC_BYTES;
+  // per-window float arrays: s, x, dy, gate slope, softplus slope [TW][G];
+  // B, C [TW][N]; the states [TW][THREADS] float4; dB, dC sums [TW][2N]
+  static constexpr int SCAL_BYTES = 5 * TW * G * 4;
+  static constexpr int BCF_BYTES = 2 * TW * N * 4;
+  static constexpr int HIST_BYTES = TW * THREADS * 16;
+  static constexpr int ACC_BYTES = TW * 2 * N * 4;
+  static constexpr int SMEM_BYTES =
+      2 * STAGE + SCAL_BYTES + BCF_BYTES + HIST_BYTES + ACC_BYTES;
+  static_assert(THREADS % G == 0, "a pre-pass thread keeps one channel");
+  static_assert((G * ESZ) % 16 == 0 && (N * ESZ) % 16 == 0,
+                "tile rows are whole 16-byte chunks");
+};
+
+template <typename T, int NG, int NW, bool ZOH>
+__global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
+  using Cfg = BwdCfg<T, NG, NW>;
+  constexpr int N = Cfg::N, CW = Cfg::CW, G = Cfg::G, TW = Cfg::TW;
+  constexpr int THREADS = Cfg::THREADS, ESZ = Cfg::ESZ;
+  constexpr unsigned FULL = 0xffffffffu;
+  extern __shared__ __align__(16) unsigned char smem[];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane % NG;
+  const int c = lane / NG;
+  const int cl = warp * CW + c;  // channel within the tile
+
+  const int64_t L = p.seqlen, E = p.dim;
+  const int64_t tiles = (E + G - 1) / G;
+  const int64_t b = blockIdx.x / tiles;
+  const int64_t e0 = (blockIdx.x - b * tiles) * G;
+  const int64_t e = e0 + cl;
+  const bool ch_ok = e < E;
+  const int64_t nck = (L + TW - 1) / TW;
+
+  float *const sS = reinterpret_cast<float *>(smem + 2 * Cfg::STAGE);
+  float *const sX = sS + TW * G;
+  float *const sDY = sX + TW * G;
+  float *const sGZ = sDY + TW * G;
+  float *const sSG = sGZ + TW * G;
+  float *const sBF = sSG + TW * G;
+  float *const sCF = sBF + TW * N;
+  float4 *const sH = reinterpret_cast<float4 *>(sCF + TW * N);
+  float *const sAcc = reinterpret_cast<float *>(sH + TW * THREADS);
+
+  const T *gx = static_cast<const T *>(p.x);
+  const T *gdl = static_cast<const T *>(p.delta);
+  const T *gz = static_cast<const T *>(p.z);
+  const T *gdy = static_cast<const T *>(p.dy);
+  const T *gB = static_cast<const T *>(p.B);
+  const T *gC = static_cast<const T *>(p.C);
+  const bool has_z = gz != nullptr;
+
+  // per lane: A log2(e), 1/A, A for its 4 states
+  float A2[4] = {}, iA[4] = {}, Av[4] = {};
+  float lam[4] = {}, dA[4] = {};
+  if (ch_ok) {
+    const float *al = p.A_log + e * N + 4 * g;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      Av[i] = -expf(al[i]);
+      A2[i] = fmaxf(Av[i] * kLog2e, -FLT_MAX);
+      iA[i] = -expf(-al[i]);
+    }
+    if (p.dh_last) {
+      const float4 v = *reinterpret_cast<const float4 *>(
+          p.dh_last + (b * E + e) * N + 4 * g);
+      lam[0] = v.x; lam[1] = v.y; lam[2] = v.z; lam[3] = v.w;
+    }
+  }
+  // the pre-pass channel of this thread (THREADS is a multiple of G)
+  const int pc = tid % G;
+  const int64_t pe = e0 + pc;
+  const bool pe_ok = pe < E;
+  const float pbias = (pe_ok && p.delta_bias) ? p.delta_bias[pe] : 0.0f;
+  const float Dv = (ch_ok && p.D) ? p.D[e] : 0.0f;
+  float sum_dD = 0.0f, sum_db = 0.0f;
+
+  for (int i = tid; i < TW * 2 * N; i += THREADS) sAcc[i] = 0.0f;
+
+  auto stage = [&](int64_t w, int s) {
+    unsigned char *base = smem + s * Cfg::STAGE;
+    const int64_t t0 = w * TW;
+    constexpr int CPR = G * ESZ / 16, EPC = 16 / ESZ;
+    for (int idx = tid; idx < TW * CPR; idx += THREADS) {
+      const int r = idx / CPR, k = idx - (idx / CPR) * CPR;
+      const int64_t t = t0 + r, ec = e0 + k * EPC;
+      const bool ok = t < L && ec < E;
+      const int64_t go = ok ? (b * L + t) * E + ec : 0;
+      const int so = r * G * ESZ + k * 16;
+      cp_async16(base + so, gx + go, ok);
+      cp_async16(base + Cfg::ACT_BYTES + so, gdl + go, ok);
+      if (has_z) cp_async16(base + 2 * Cfg::ACT_BYTES + so, gz + go, ok);
+      cp_async16(base + 3 * Cfg::ACT_BYTES + so, gdy + go, ok);
+    }
+    unsigned char *bc = base + 4 * Cfg::ACT_BYTES;
+    constexpr int CH = TW * N * ESZ / 16;
+    for (int idx = tid; idx < CH; idx += THREADS) {
+      const int r = idx * 16 / (N * ESZ);
+      const bool ok = t0 + r < L;
+      const int64_t go = ok ? (b * L + t0) * N + int64_t(idx) * (16 / ESZ) : 0;
+      cp_async16(bc + idx * 16, gB + go, ok);
+      cp_async16(bc + Cfg::BC_BYTES + idx * 16, gC + go, ok);
+    }
+  };
+
+  const int64_t w_last = nck - 1;
+  stage(w_last, 0);
+  cp_async_commit();
+  for (int64_t w = w_last; w >= 0; --w) {
+    const int par = int((w_last - w) & 1);
+    if (w > 0) stage(w - 1, par ^ 1);
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();
+
+    const int64_t t0 = w * TW;
+    const unsigned char *base = smem + par * Cfg::STAGE;
+    // ---- 2. per (t, e) scalars, once
+    for (int idx = tid; idx < TW * G; idx += THREADS) {
+      const int r = idx / G;  // idx % G == pc
+      const bool ok = pe_ok && t0 + r < L;
+      const int o = (r * G + pc) * ESZ;
+      const float raw =
+          Act<T>::load(reinterpret_cast<const T *>(base + Cfg::ACT_BYTES + o)) +
+          pbias;
+      const float xv = Act<T>::load(reinterpret_cast<const T *>(base + o));
+      const float gv = Act<T>::load(
+          reinterpret_cast<const T *>(base + 3 * Cfg::ACT_BYTES + o));
+      float dyv = gv, gzv = 0.0f;
+      if (has_z) {
+        const float zv = Act<T>::load(
+            reinterpret_cast<const T *>(base + 2 * Cfg::ACT_BYTES + o));
+        const float sg = rcp(1.0f + ex2(-zv * kLog2e));
+        dyv = gv * zv * sg;
+        gzv = gv * sg * fmaf(zv, 1.0f - sg, 1.0f);
+      }
+      float sv = raw, slope = 1.0f;
+      if (p.softplus) {
+        sv = softplus(raw);
+        slope = rcp(1.0f + ex2(-raw * kLog2e));
+      }
+      sS[idx] = ok ? sv : 0.0f;
+      sX[idx] = ok ? xv : 0.0f;
+      sDY[idx] = ok ? dyv : 0.0f;
+      sGZ[idx] = ok ? gzv : 0.0f;
+      sSG[idx] = slope;
+    }
+    {
+      const unsigned char *bc = base + 4 * Cfg::ACT_BYTES;
+      for (int idx = tid; idx < TW * N; idx += THREADS) {
+        sBF[idx] = Act<T>::load(reinterpret_cast<const T *>(bc) + idx);
+        sCF[idx] =
+            Act<T>::load(reinterpret_cast<const T *>(bc + Cfg::BC_BYTES) + idx);
+      }
+    }
+    __syncthreads();
+
+    // ---- 3. recompute this lane's states through the window
+    float hs[4] = {};
+    if (ch_ok) {
+      const float4 v = *reinterpret_cast<const float4 *>(
+          p.ckpt + ((b * nck + w) * E + e) * N + 4 * g);
+      hs[0] = v.x; hs[1] = v.y; hs[2] = v.z; hs[3] = v.w;
+    }
+    {
+      float h[4] = {hs[0], hs[1], hs[2], hs[3]};
+#pragma unroll 4
+      for (int r = 0; r < TW; ++r) {
+        const float sv = sS[r * G + cl];
+        const float xv = sX[r * G + cl];
+        const float4 Bq = *reinterpret_cast<const float4 *>(sBF + r * N + 4 * g);
+        const float Bv[4] = {Bq.x, Bq.y, Bq.z, Bq.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float zl = sv * A2[i];
+          const float a = ex2(zl);
+          const float f = ZOH ? zoh_factor(sv, zl, a, iA[i]) : sv;
+          h[i] = fmaf(a, h[i], f * xv * Bv[i]);
+        }
+        sH[r * THREADS + tid] = make_float4(h[0], h[1], h[2], h[3]);
+      }
+    }
+
+    // ---- 4. the reverse sweep
+#pragma unroll 1
+    for (int r = TW - 1; r >= 0; --r) {
+      const float4 hc = sH[r * THREADS + tid];
+      const float4 hp4 =
+          r > 0 ? sH[(r - 1) * THREADS + tid]
+                : make_float4(hs[0], hs[1], hs[2], hs[3]);
+      const float hcur[4] = {hc.x, hc.y, hc.z, hc.w};
+      const float hprev[4] = {hp4.x, hp4.y, hp4.z, hp4.w};
+      const float sv = sS[r * G + cl];
+      const float xv = sX[r * G + cl];
+      const float dyv = sDY[r * G + cl];
+      const float4 Bq = *reinterpret_cast<const float4 *>(sBF + r * N + 4 * g);
+      const float4 Cq = *reinterpret_cast<const float4 *>(sCF + r * N + 4 * g);
+      const float Bv[4] = {Bq.x, Bq.y, Bq.z, Bq.w};
+      const float Cv[4] = {Cq.x, Cq.y, Cq.z, Cq.w};
+      float pre = 0.0f, dxp = 0.0f, dsp = 0.0f;
+      float v8[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float zl = sv * A2[i];
+        const float a = ex2(zl);
+        pre = fmaf(Cv[i], hcur[i], pre);
+        v8[4 + i] = dyv * hcur[i];       // dC
+        lam[i] = fmaf(dyv, Cv[i], lam[i]);
+        const float da = lam[i] * hprev[i];
+        if (ZOH) {
+          const float f = zoh_factor(sv, zl, a, iA[i]);
+          const float lbx = lam[i] * Bv[i] * xv;
+          dsp = fmaf(lbx, a, dsp);
+          v8[i] = lam[i] * f * xv;       // dB
+          dxp = fmaf(lam[i] * f, Bv[i], dxp);
+          dA[i] = fmaf(lbx, (sv * a - f) * iA[i], dA[i]);
+        } else {
+          dsp = fmaf(lam[i] * Bv[i], xv, dsp);
+          v8[i] = lam[i] * sv * xv;      // dB
+          dxp = fmaf(lam[i] * sv, Bv[i], dxp);
+        }
+        dsp = fmaf(da * a, Av[i], dsp);
+        dA[i] = fmaf(da * a, sv, dA[i]);
+        lam[i] *= a;
+      }
+      // per-channel sums over the channel's NG lanes (all lanes get them)
+#pragma unroll
+      for (int m = 1; m < NG; m <<= 1) {
+        pre += __shfl_xor_sync(FULL, pre, m);
+        dxp += __shfl_xor_sync(FULL, dxp, m);
+        dsp += __shfl_xor_sync(FULL, dsp, m);
+      }
+      // dB, dC summed over the warp's channels: a transposing butterfly over
+      // lane bits 4, 3, 2 leaves value j = (lane >> 2) & 7 in v8[0]; channel
+      // bits below bit 2 (NG < 4) are summed plainly
+      {
+        bool hi = lane & 16;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float send = hi ? v8[i] : v8[i + 4];
+          const float keep = hi ? v8[i + 4] : v8[i];
+          v8[i] = keep + __shfl_xor_sync(FULL, send, 16);
+        }
+        hi = lane & 8;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const float send = hi ? v8[i] : v8[i + 2];
+          const float keep = hi ? v8[i + 2] : v8[i];
+          v8[i] = keep + __shfl_xor_sync(FULL, send, 8);
+        }
+        hi = lane & 4;
+        {
+          const float send = hi ? v8[0] : v8[1];
+          const float keep = hi ? v8[1] : v8[0];
+          v8[0] = keep + __shfl_xor_sync(FULL, send, 4);
+        }
+        if (NG <= 2) v8[0] += __shfl_xor_sync(FULL, v8[0], 2);
+        if (NG == 1) v8[0] += __shfl_xor_sync(FULL, v8[0], 1);
+        if ((lane & 3 & ~(NG - 1)) == 0) {
+          const int j = (lane >> 2) & 7;
+          atomicAdd(sAcc + r * 2 * N + (j >> 2) * N + 4 * g + (j & 3), v8[0]);
+        }
+      }
+      // the channel's outputs at step t
+      const int64_t t = t0 + r;
+      if (g == 0 && ch_ok && t < L) {
+        const int64_t i = (b * L + t) * E + e;
+        const float dxv = fmaf(dyv, Dv, dxp);
+        const float draw = dsp * sSG[r * G + cl];
+        Act<T>::store(static_cast<T *>(p.dx) + i, dxv);
+        Act<T>::store(static_cast<T *>(p.ddelta) + i, draw);
+        if (has_z)
+          Act<T>::store(static_cast<T *>(p.dz) + i,
+                        sGZ[r * G + cl] * fmaf(Dv, xv, pre));
+        sum_dD = fmaf(dyv, xv, sum_dD);
+        sum_db += draw;
+      }
+    }
+    __syncthreads();
+    // ---- dB, dC of the window into HBM, once per (t, n) and block
+    for (int idx = tid; idx < TW * 2 * N; idx += THREADS) {
+      const int r = idx / (2 * N), k = idx - r * 2 * N;
+      const int64_t t = t0 + r;
+      if (t < L) {
+        float *dst = (k < N ? p.dB : p.dC) + (b * L + t) * N + (k % N);
+        atomicAdd(dst, sAcc[idx]);
+      }
+      sAcc[idx] = 0.0f;
+    }
+    __syncthreads();
+  }
+  cp_async_wait<0>();
+
+  if (ch_ok) {
+    if (p.dh0)
+      *reinterpret_cast<float4 *>(p.dh0 + (b * E + e) * N + 4 * g) =
+          make_float4(lam[0], lam[1], lam[2], lam[3]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      atomicAdd(p.dA_log + e * N + 4 * g + i, dA[i] * Av[i]);
+    if (g == 0) {
+      if (p.dD) atomicAdd(p.dD + e, sum_dD);
+      if (p.ddelta_bias) atomicAdd(p.ddelta_bias + e, sum_db);
+    }
+  }
+}
+
+}  // namespace ssm

@@ -128,6 +128,8 @@ struct ChunkCfg {
                 "cp.async destinations are 16-byte aligned");
   static_assert((TB > 1 ? K / NG : TW / (2 * NG)) % 2 == 0,
                 "exchange slots alternate parity from block to block");
+  static_assert(TW % kCkptSteps == 0 && kCkptSteps % (2 * NG) == 0,
+                "checkpoints fall on block starts");
 
   __device__ static __forceinline__ int raw_off(int r) {
     return r * RAW_P + (r / BLK) * RAW_PB;
@@ -244,6 +246,7 @@ scan_chunked_kernel(const ScanParams p) {
   const T *gC = static_cast<const T *>(p.C);
   T *gy = static_cast<T *>(p.y);
   const bool has_z = gz != nullptr;
+  const bool store_y = gy != nullptr;
 
   float2 A01 = make_float2(0.0f, 0.0f), A23 = A01;  // A * log2(e)
   float2 iA01 = A01, iA23 = A01;  // 1 / A (zero-order-hold write only)
@@ -408,7 +411,7 @@ scan_chunked_kernel(const ScanParams p) {
         const int64_t t = t0 + r;
         if (MODE == kWalkMain) yv = fmaf(Dv, xm, yv);
         if (has_z) yv *= silu(zm);
-        if (ch_ok && t < t_end) {
+        if (ch_ok && store_y && t < t_end) {
           T *yp = gy + ybase + int64_t(r) * E;
           if (MODE == kWalkCorrect) yv += Act<T>::load(yp);
           Act<T>::store(yp, yv);
@@ -458,7 +461,7 @@ scan_chunked_kernel(const ScanParams p) {
               acc = fma2(make_float2(cw[1], cw[1]), make_float2(vm2, vm1), acc);
               acc = fma2(make_float2(cw[2], cw[2]), make_float2(vm1, x2.x), acc);
               acc = fma2(make_float2(cw[3], cw[3]), x2, acc);
-              x2 = silu2(acc);
+              x2 = PairMath<T>::silu(acc);
             }
           }
           const float2 v2 = add2(
@@ -469,7 +472,7 @@ scan_chunked_kernel(const ScanParams p) {
                            Act<T>::load(reinterpret_cast<const T *>(sZ + o0)),
                            Act<T>::load(reinterpret_cast<const T *>(sZ + o1)))
                      : make_float2(0.0f, 0.0f);
-          float2 d2 = p.softplus ? softplus2(v2) : v2;
+          float2 d2 = p.softplus ? PairMath<T>::softplus(v2) : v2;
           if (!full) {
             if (t0 + r0 >= t_end) d2.x = 0.0f;
             if (t0 + r0 + 1 >= t_end) d2.y = 0.0f;
@@ -489,8 +492,8 @@ scan_chunked_kernel(const ScanParams p) {
         auto finish2 = [&](int jb, float2 y2, float2 x2, float2 z2) {
           const int r0 = jb * BS + 2 * g;
           if (MODE == kWalkMain) y2 = fma2(make_float2(Dv, Dv), x2, y2);
-          if (has_z) y2 = mul2(y2, silu2(z2));
-          if (ch_ok) {
+          if (has_z) y2 = mul2(y2, PairMath<T>::silu(z2));
+          if (ch_ok && store_y) {
             T *yp = yw + int64_t(r0) * E;
             if (full || t0 + r0 < t_end) {
               if (MODE == kWalkCorrect) y2.x += Act<T>::load(yp);
@@ -509,6 +512,17 @@ scan_chunked_kernel(const ScanParams p) {
 #pragma unroll 2
         for (int jb = 0; jb < NBW; ++jb) {
           const int par = jb & 1;
+          if constexpr (!SPLIT) {
+            // training forward: the state before every kCkptSteps-th step
+            if (MODE == kWalkMain && p.ckpt && (jb * BS) % kCkptSteps == 0 &&
+                ch_ok && t0 + jb * BS < t_end) {
+              const int64_t k = (t0 + jb * BS) / kCkptSteps;
+              const int64_t nck = (L + kCkptSteps - 1) / kCkptSteps;
+              *reinterpret_cast<float4 *>(
+                  p.ckpt + ((b * nck + k) * E + e) * N + 4 * g) =
+                  make_float4(h01.x, h01.y, h23.x, h23.y);
+            }
+          }
           float2 dd[BS];
           if constexpr (NG > 1) {
 #pragma unroll

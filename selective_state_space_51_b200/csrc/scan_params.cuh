@@ -27,6 +27,10 @@ struct ScanParams {
   const float *conv_weight;  // [E, K] or nullptr (x is used as it is)
   const float *conv_bias;    // [E] or nullptr
   int conv_width;            // K, 1..kScanConvMaxWidth
+  // Training forward (unsplit, one time block): the state before every
+  // kCkptSteps-th step goes to ckpt [b, ceil(L / kCkptSteps), E, N]; y may
+  // then be nullptr (not written).
+  float *ckpt;
   // Split sequences (chunked variant): each sequence is cut into `segments`
   // pieces of seg_len steps (a multiple of the window), scanned concurrently
   // from a zero state and joined by a decoupled look-back over per-piece
@@ -43,6 +47,9 @@ struct ScanParams {
   unsigned spin_limit;       // bounded wait: polls before giving up
   unsigned debug;            // kDebug* bits (tests only)
 };
+
+// Steps between the forward checkpoints the backward pass restarts from.
+constexpr int kCkptSteps = 16;
 
 // Widest causal convolution the fused scan takes.
 constexpr int kScanConvMaxWidth = 4;

@@ -7,6 +7,7 @@
 #include <new>
 
 #include "../../include/ssm_scan.h"
+#include "kernel_bwd.cuh"
 #include "kernel_chunked.cuh"
 #include "kernel_sequential.cuh"
 #include "kernel_step.cuh"
@@ -29,6 +30,9 @@ struct ssm_scan_s {
   // split-sequence workspace: flags, then three state arrays
   void *ws = nullptr;
   size_t ws_bytes = 0;
+  // backward: the forward's state checkpoints
+  float *ckpt = nullptr;
+  size_t ckpt_bytes = 0;
 };
 
 namespace {
@@ -237,26 +241,29 @@ int dispatch_chunked(ssm_scan_s *h, ssm::ScanParams &p, int dtype, int tb,
   return SSM_ERR_UNSUPPORTED;
 }
 
-template <typename T, int QP>
-int launch_step_qp(const ssm::StepParams &p, bool vec, cudaStream_t s) {
-  const int64_t threads = p.batch * p.dim * QP;
-  const int64_t blocks = (threads + 255) / 256;
-  if (blocks > 0x7fffffff) return SSM_ERR_UNSUPPORTED;
+template <typename T, int SPT, int QP>
+int launch_step_cfg(const ssm::StepParams &p, bool vec, cudaStream_t s) {
+  const int64_t threads = p.dim * QP;
+  const int64_t bx = (threads + 127) / 128;
+  if (bx > 0x7fffffff) return SSM_ERR_UNSUPPORTED;
+  // batch rows beyond the grid's y extent are taken by a stride loop
+  const dim3 grid(unsigned(bx), unsigned(p.batch < 65535 ? p.batch : 65535));
   if (vec)
-    ssm::scan_step_kernel<T, QP, true><<<unsigned(blocks), 256, 0, s>>>(p);
+    ssm::scan_step_kernel<T, SPT, QP, true><<<grid, 128, 0, s>>>(p);
   else
-    ssm::scan_step_kernel<T, QP, false><<<unsigned(blocks), 256, 0, s>>>(p);
+    ssm::scan_step_kernel<T, SPT, QP, false><<<grid, 128, 0, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
+// States per thread: the whole channel up to 16, else 16 per thread and 2 or
+// 4 threads per channel.
 template <typename T>
 int launch_step(const ssm::StepParams &p, bool vec, cudaStream_t s) {
-  const int groups = (p.dstate + 3) / 4;
-  if (groups <= 1) return launch_step_qp<T, 1>(p, vec, s);
-  if (groups <= 2) return launch_step_qp<T, 2>(p, vec, s);
-  if (groups <= 4) return launch_step_qp<T, 4>(p, vec, s);
-  if (groups <= 8) return launch_step_qp<T, 8>(p, vec, s);
-  return launch_step_qp<T, 16>(p, vec, s);
+  if (p.dstate <= 4) return launch_step_cfg<T, 4, 1>(p, vec, s);
+  if (p.dstate <= 8) return launch_step_cfg<T, 8, 1>(p, vec, s);
+  if (p.dstate <= 16) return launch_step_cfg<T, 16, 1>(p, vec, s);
+  if (p.dstate <= 32) return launch_step_cfg<T, 16, 2>(p, vec, s);
+  return launch_step_cfg<T, 16, 4>(p, vec, s);
 }
 
 // The forward scan behind both entry points; conv_weight == nullptr: x is
@@ -332,6 +339,36 @@ int scan_fwd(ssm_scan_s *h, const void *x, const float *conv_weight,
     if (variant != SSM_VARIANT_CHUNKED) h->last_segments = 1;
   }
   return rc;
+}
+
+// ---- backward
+template <typename T, int NG, bool ZOH>
+int launch_bwd(const ssm::BwdParams &p, cudaStream_t s) {
+  using Cfg = ssm::BwdCfg<T, NG, 4>;
+  const int64_t tiles = (p.dim + Cfg::G - 1) / Cfg::G;
+  const int64_t blocks = p.batch * tiles;
+  if (blocks > 0x7fffffff) return SSM_ERR_UNSUPPORTED;
+  auto kern = ssm::scan_bwd_kernel<T, NG, 4, ZOH>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           Cfg::SMEM_BYTES) != cudaSuccess) {
+    cudaGetLastError();
+    return SSM_ERR_CUDA;
+  }
+  kern<<<unsigned(blocks), Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+// The training forward (checkpoints, no y) and the reverse sweep for one
+// (forward config, activation type, states per lane).
+template <class Cf, typename T, int NG>
+int run_bwd(ssm::ScanParams &fp, const ssm::BwdParams &bp, cudaStream_t s) {
+  const int64_t tiles = (fp.dim + Cf::G - 1) / Cf::G;
+  int rc = fp.write_zoh
+               ? launch_kernel<Cf, false, true, false>(fp, fp.batch * tiles, s)
+               : launch_kernel<Cf, false, false, false>(fp, fp.batch * tiles, s);
+  if (rc != SSM_OK) return rc;
+  return fp.write_zoh ? launch_bwd<T, NG, true>(bp, s)
+                      : launch_bwd<T, NG, false>(bp, s);
 }
 
 }  // namespace
@@ -420,12 +457,13 @@ int ssm_scan_create(ssm_scan_t *out, int device) {
 int ssm_scan_destroy(ssm_scan_t h) {
   if (!h) return SSM_OK;
   int rc = SSM_OK;
-  if (h->ws || h->ctl) {
+  if (h->ws || h->ctl || h->ckpt) {
     int prev = 0;
     cudaGetDevice(&prev);
     cudaSetDevice(h->device);
     if (h->ws && cudaFree(h->ws) != cudaSuccess) rc = SSM_ERR_CUDA;
     if (h->ctl && cudaFree(h->ctl) != cudaSuccess) rc = SSM_ERR_CUDA;
+    if (h->ckpt && cudaFree(h->ckpt) != cudaSuccess) rc = SSM_ERR_CUDA;
     cudaSetDevice(prev);
   }
   delete h;
@@ -523,6 +561,112 @@ int ssm_scan_fwd_conv(ssm_scan_t h, const void *v, const float *conv_weight,
   return scan_fwd(h, v, conv_weight, conv_bias, conv_width, delta, A_log, B,
                   C, D, z, delta_bias, flags, h0, y, h_last, dims, dtype,
                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+int ssm_scan_bwd(ssm_scan_t h, const void *x, const void *delta,
+                 const float *A_log, const void *B, const void *C,
+                 const float *D, const void *z, const float *delta_bias,
+                 uint32_t flags, const float *h0, const void *dy,
+                 const float *dh_last, void *dx, void *ddelta, float *dA_log,
+                 float *dB, float *dC, float *dD, void *dz,
+                 float *ddelta_bias, float *dh0, ssm_scan_dims dims, int dtype,
+                 struct CUstream_st *stream) {
+  // ---- host-side validation: nothing touches the GPU before it passes
+  if (!h || !x || !delta || !A_log || !B || !C || !dy || !dx || !ddelta ||
+      !dA_log || !dB || !dC)
+    return SSM_ERR_INVALID;
+  if ((z && !dz) || (D && !dD) || (delta_bias && !ddelta_bias))
+    return SSM_ERR_INVALID;
+  if (dims.batch <= 0 || dims.seqlen <= 0 || dims.dim <= 0 || dims.dstate <= 0)
+    return SSM_ERR_INVALID;
+  if (flags & ~uint32_t(SSM_DELTA_SOFTPLUS | SSM_WRITE_ZOH))
+    return SSM_ERR_INVALID;
+  if (dtype != SSM_F32 && dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
+  const int64_t N = dims.dstate;
+  const size_t esz = dtype == SSM_F32 ? 4 : 2;
+  if (N != 4 && N != 8 && N != 16) return SSM_ERR_UNSUPPORTED;
+  if (N * int64_t(esz) < 16 || (dims.dim * int64_t(esz)) % 16 != 0)
+    return SSM_ERR_UNSUPPORTED;
+  int64_t rows = 0, acts = 0, st = 0, nck = 0, ck = 0;
+  if (!mul_ok(dims.batch, dims.seqlen, &rows) ||
+      !mul_ok(rows, dims.dim, &acts) ||
+      !mul_ok(dims.batch * dims.dim, N, &st) || acts > (int64_t(1) << 56))
+    return SSM_ERR_INVALID;
+  nck = (dims.seqlen + ssm::kCkptSteps - 1) / ssm::kCkptSteps;
+  if (!mul_ok(st, nck, &ck) || ck > (int64_t(1) << 56)) return SSM_ERR_INVALID;
+  const void *tiles_in[] = {x, delta, z, dy, B, C};
+  for (const void *q : tiles_in)
+    if (q && !aligned(q, 16)) return SSM_ERR_ALIGN;
+  const void *acts_out[] = {dx, ddelta, dz};
+  for (const void *q : acts_out)
+    if (q && !aligned(q, esz)) return SSM_ERR_ALIGN;
+  const float *f4[] = {h0, dh_last, dh0, A_log};
+  for (const float *q : f4)
+    if (q && !aligned(q, 16)) return SSM_ERR_ALIGN;
+  const float *f1[] = {D, delta_bias, dA_log, dB, dC, dD, ddelta_bias};
+  for (const float *q : f1)
+    if (q && !aligned(q, 4)) return SSM_ERR_ALIGN;
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) {
+    cudaGetLastError();
+    return SSM_ERR_CUDA;
+  }
+  if (cur != h->device) return SSM_ERR_INVALID;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  // ---- checkpoint workspace, and the summed outputs cleared
+  const size_t need = size_t(ck) * sizeof(float);
+  if (need > h->ckpt_bytes) {
+    if (h->ckpt) cudaFreeAsync(h->ckpt, s);
+    h->ckpt = nullptr;
+    h->ckpt_bytes = 0;
+    if (cudaMallocAsync(reinterpret_cast<void **>(&h->ckpt), need, s) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return SSM_ERR_NOMEM;
+    }
+    h->ckpt_bytes = need;
+  }
+  const size_t bcn = size_t(rows) * N * sizeof(float);
+  if (cudaMemsetAsync(dB, 0, bcn, s) != cudaSuccess ||
+      cudaMemsetAsync(dC, 0, bcn, s) != cudaSuccess ||
+      cudaMemsetAsync(dA_log, 0, size_t(dims.dim) * N * sizeof(float), s) !=
+          cudaSuccess ||
+      (dD && cudaMemsetAsync(dD, 0, size_t(dims.dim) * sizeof(float), s) !=
+                 cudaSuccess) ||
+      (ddelta_bias &&
+       cudaMemsetAsync(ddelta_bias, 0, size_t(dims.dim) * sizeof(float), s) !=
+           cudaSuccess))
+    return SSM_ERR_CUDA;
+
+  ssm::ScanParams fp{};
+  fp.x = x; fp.delta = delta; fp.A_log = A_log; fp.B = B; fp.C = C;
+  fp.D = D; fp.z = z; fp.delta_bias = delta_bias; fp.h0 = h0;
+  fp.y = nullptr; fp.h_last = nullptr; fp.ckpt = h->ckpt;
+  fp.batch = dims.batch; fp.seqlen = dims.seqlen; fp.dim = dims.dim;
+  fp.dstate = int(N);
+  fp.softplus = (flags & SSM_DELTA_SOFTPLUS) ? 1 : 0;
+  fp.write_zoh = (flags & SSM_WRITE_ZOH) ? 1 : 0;
+  fp.segments = 1;
+
+  ssm::BwdParams bp{};
+  bp.x = x; bp.delta = delta; bp.z = z; bp.dy = dy; bp.B = B; bp.C = C;
+  bp.A_log = A_log; bp.D = D; bp.delta_bias = delta_bias; bp.h0 = h0;
+  bp.dh_last = dh_last; bp.ckpt = h->ckpt;
+  bp.dx = dx; bp.ddelta = ddelta; bp.dz = z ? dz : nullptr;
+  bp.dB = dB; bp.dC = dC; bp.dA_log = dA_log;
+  bp.dD = D ? dD : nullptr; bp.ddelta_bias = delta_bias ? ddelta_bias : nullptr;
+  bp.dh0 = dh0;
+  bp.batch = dims.batch; bp.seqlen = dims.seqlen; bp.dim = dims.dim;
+  bp.dstate = int(N); bp.softplus = fp.softplus;
+
+  if (dtype == SSM_BF16) {
+    if (N == 16) return run_bwd<C16b1, __nv_bfloat16, 4>(fp, bp, s);
+    return run_bwd<C8b1, __nv_bfloat16, 2>(fp, bp, s);
+  }
+  if (N == 16) return run_bwd<C16f1, float, 4>(fp, bp, s);
+  if (N == 8) return run_bwd<C8f1, float, 2>(fp, bp, s);
+  return run_bwd<C4f1, float, 1>(fp, bp, s);
 }
 
 }  // extern "C"

@@ -34,6 +34,33 @@ def test_every_declared_symbol_is_exported(lib):
         assert hasattr(lib, n), n
 
 
+def declared_arity():
+    """Number of parameters of each SSM_API function in include/*.h."""
+    out = {}
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        for m in re.finditer(r"SSM_API\s+[\w\s\*]*?\b(ssm_\w+)\s*\(([^)]*)\)",
+                             text):
+            params = [q for q in m.group(2).split(",") if q.strip()]
+            if len(params) == 1 and params[0].strip() == "void":
+                params = []
+            out[m.group(1)] = len(params)
+    return out
+
+
+def test_binding_signatures_match_the_header(lib):
+    """Every function the binding declares to ctypes takes exactly the
+    header's parameter count."""
+    arity = declared_arity()
+    checked = 0
+    for name, n in arity.items():
+        fn = getattr(lib, name)
+        if fn.argtypes is not None:
+            assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
+            checked += 1
+    assert checked >= 8
+
+
 def test_library_built_for_sm100a():
     assert "arch=compute_100a,code=sm_100a" in " ".join(B.NVCC_FLAGS)
 
