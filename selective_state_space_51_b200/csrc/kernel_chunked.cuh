@@ -106,9 +106,14 @@ struct ChunkCfg {
   static constexpr int STAGE_BYTES =
       3 * RAW_BYTES + (ESZ == 2 ? 2 * BCRAW_BYTES : 2 * BF_BYTES);
   // time-block-1 blocks: BS = 2 NG steps, 2 per lane; exchange rows of the
-  // (delta, delta * x) pairs of a block, padded by 2 pairs per channel
+  // (delta, delta * x) pairs of a block, one row of BS pairs per channel.
+  // Channels whose bit XRB is set keep their row's halves swapped (pair s at
+  // s ^ BS/2), which makes both the 16-byte stores (8 lanes: 2 channels x 4
+  // groups at N = 16) and the 8-byte loads (16 lanes: 4 channels) free of
+  // bank conflicts.
   static constexpr int BS = 2 * NG;
-  static constexpr int SLOT = BS + 2;
+  static constexpr int SLOT = BS;
+  static constexpr int XRB = NG == 4 ? 1 : 2;
   // per warp, 2 parities of: CW rows of SLOT pairs (time blocks 1) or 32
   // single slots (time blocks > 1)
   static constexpr int XCH_PER_WARP = TB == 1 ? CW * SLOT : 32;
@@ -434,6 +439,14 @@ scan_chunked_kernel(const ScanParams p) {
         // read of a row precedes the __syncwarp that ends its iteration.
         constexpr int BS = Cfg::BS, NBW = TW / BS, SLOT = Cfg::SLOT;
         (void)SLOT;
+        // this channel's exchange row halves (see ChunkCfg::XRB)
+        const int xswap = (c >> Cfg::XRB) & 1;
+        const int xlo = c * SLOT + (xswap ? BS / 2 : 0);  // pairs 0 .. BS/2-1
+        const int xhi = c * SLOT + (xswap ? 0 : BS / 2);  // pairs BS/2 ..
+        const int xst = c * SLOT + ((2 * g) ^ (xswap ? BS / 2 : 0));
+        (void)xlo;
+        (void)xhi;
+        (void)xst;
         const bool full = t0 + TW <= t_end;  // no step of the window is past
         T *const yw = gy + ybase;
 
@@ -485,8 +498,7 @@ scan_chunked_kernel(const ScanParams p) {
           dd0 = make_float2(d2.x, dx2.x);
           dd1 = make_float2(d2.y, dx2.y);
           if constexpr (NG > 1)
-            *reinterpret_cast<float4 *>(xch + par * CW * SLOT + c * SLOT +
-                                        2 * g) =
+            *reinterpret_cast<float4 *>(xch + par * CW * SLOT + xst) =
                 make_float4(d2.x, dx2.x, d2.y, dx2.y);
         };
         auto finish2 = [&](int jb, float2 y2, float2 x2, float2 z2) {
@@ -527,7 +539,8 @@ scan_chunked_kernel(const ScanParams p) {
           if constexpr (NG > 1) {
 #pragma unroll
             for (int s = 0; s < BS; ++s)
-              dd[s] = xch[par * CW * SLOT + c * SLOT + s];
+              dd[s] = xch[par * CW * SLOT +
+                          (s < BS / 2 ? xlo + s : xhi + s - BS / 2)];
           } else {
             dd[0] = e0;
             dd[1] = e1;

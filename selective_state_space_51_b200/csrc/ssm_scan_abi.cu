@@ -242,12 +242,18 @@ int dispatch_chunked(ssm_scan_s *h, ssm::ScanParams &p, int dtype, int tb,
 }
 
 template <typename T, int SPT, int QP>
-int launch_step_cfg(const ssm::StepParams &p, bool vec, cudaStream_t s) {
+int launch_step_cfg(const ssm::StepParams &p, bool vec, int sm_count,
+                    cudaStream_t s) {
   const int64_t threads = p.dim * QP;
   const int64_t bx = (threads + 127) / 128;
   if (bx > 0x7fffffff) return SSM_ERR_UNSUPPORTED;
-  // batch rows beyond the grid's y extent are taken by a stride loop
-  const dim3 grid(unsigned(bx), unsigned(p.batch < 65535 ? p.batch : 65535));
+  // enough batch-row strides to give every SM about 8 blocks; each thread
+  // walks batch / grid.y rows with its channel's constants in registers
+  int64_t by = (int64_t(sm_count) * 8 + bx - 1) / bx;
+  if (by > p.batch) by = p.batch;
+  if (by > 65535) by = 65535;
+  if (by < 1) by = 1;
+  const dim3 grid{static_cast<unsigned>(bx), static_cast<unsigned>(by), 1u};
   if (vec)
     ssm::scan_step_kernel<T, SPT, QP, true><<<grid, 128, 0, s>>>(p);
   else
@@ -258,12 +264,12 @@ int launch_step_cfg(const ssm::StepParams &p, bool vec, cudaStream_t s) {
 // States per thread: the whole channel up to 16, else 16 per thread and 2 or
 // 4 threads per channel.
 template <typename T>
-int launch_step(const ssm::StepParams &p, bool vec, cudaStream_t s) {
-  if (p.dstate <= 4) return launch_step_cfg<T, 4, 1>(p, vec, s);
-  if (p.dstate <= 8) return launch_step_cfg<T, 8, 1>(p, vec, s);
-  if (p.dstate <= 16) return launch_step_cfg<T, 16, 1>(p, vec, s);
-  if (p.dstate <= 32) return launch_step_cfg<T, 16, 2>(p, vec, s);
-  return launch_step_cfg<T, 16, 4>(p, vec, s);
+int launch_step(const ssm::StepParams &p, bool vec, int sms, cudaStream_t s) {
+  if (p.dstate <= 4) return launch_step_cfg<T, 4, 1>(p, vec, sms, s);
+  if (p.dstate <= 8) return launch_step_cfg<T, 8, 1>(p, vec, sms, s);
+  if (p.dstate <= 16) return launch_step_cfg<T, 16, 1>(p, vec, sms, s);
+  if (p.dstate <= 32) return launch_step_cfg<T, 16, 2>(p, vec, sms, s);
+  return launch_step_cfg<T, 16, 4>(p, vec, sms, s);
 }
 
 // The forward scan behind both entry points; conv_weight == nullptr: x is
@@ -420,10 +426,12 @@ int ssm_scan_step(ssm_scan_t h, const void *x_new, void *conv_state,
   p.batch = dims.batch; p.dim = dims.dim; p.dstate = int(dims.dstate);
   p.softplus = (flags & SSM_DELTA_SOFTPLUS) ? 1 : 0;
   p.write_zoh = (flags & SSM_WRITE_ZOH) ? 1 : 0;
-  const bool vec = (dims.dstate % 4 == 0) && aligned(state, 16);
+  const bool vec = (dims.dstate % 4 == 0) && aligned(state, 16) &&
+                   aligned(B, 4 * esz) && aligned(C, 4 * esz);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return dtype == SSM_F32 ? launch_step<float>(p, vec, s)
-                          : launch_step<__nv_bfloat16>(p, vec, s);
+  return dtype == SSM_F32
+             ? launch_step<float>(p, vec, h->sm_count, s)
+             : launch_step<__nv_bfloat16>(p, vec, h->sm_count, s);
 }
 
 int ssm_scan_create(ssm_scan_t *out, int device) {
