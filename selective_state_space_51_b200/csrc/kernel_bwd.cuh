@@ -60,10 +60,12 @@ struct BwdCfg {
   static constexpr int BC_BYTES = TW * N * ESZ;
   static constexpr int STAGE = 4 * ACT_BYTES + 2 * BC_BYTES;
   // per-window float arrays: s, x, dy, gate slope, softplus slope [TW][G];
-  // B, C [TW][N]; the states [TW][THREADS] float4; dB, dC sums [TW][2N]
+  // B, C [TW][N]; the states of half a window [TW/2][THREADS] float4; dB,
+  // dC sums [TW][2N]
   static constexpr int SCAL_BYTES = 5 * TW * G * 4;
   static constexpr int BCF_BYTES = 2 * TW * N * 4;
-  static constexpr int HIST_BYTES = TW * THREADS * 16;
+  static constexpr int HALF = TW / 2;  // rows of state history kept at once
+  static constexpr int HIST_BYTES = HALF * THREADS * 16;
   static constexpr int ACC_BYTES = TW * 2 * N * 4;
   static constexpr int SMEM_BYTES =
       2 * STAGE + SCAL_BYTES + BCF_BYTES + HIST_BYTES + ACC_BYTES;
@@ -76,7 +78,7 @@ template <typename T, int NG, int NW, bool ZOH>
 __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
   using Cfg = BwdCfg<T, NG, NW>;
   constexpr int N = Cfg::N, CW = Cfg::CW, G = Cfg::G, TW = Cfg::TW;
-  constexpr int THREADS = Cfg::THREADS, ESZ = Cfg::ESZ;
+  constexpr int THREADS = Cfg::THREADS, ESZ = Cfg::ESZ, HALF = Cfg::HALF;
   constexpr unsigned FULL = 0xffffffffu;
   extern __shared__ __align__(16) unsigned char smem[];
 
@@ -101,7 +103,7 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
   float *const sBF = sSG + TW * G;
   float *const sCF = sBF + TW * N;
   float4 *const sH = reinterpret_cast<float4 *>(sCF + TW * N);
-  float *const sAcc = reinterpret_cast<float *>(sH + TW * THREADS);
+  float *const sAcc = reinterpret_cast<float *>(sH + Cfg::HALF * THREADS);
 
   const T *gx = static_cast<const T *>(p.x);
   const T *gdl = static_cast<const T *>(p.delta);
@@ -216,17 +218,19 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
     }
     __syncthreads();
 
-    // ---- 3. recompute this lane's states through the window
-    float hs[4] = {};
+    // ---- 3. recompute this lane's states from the checkpoint, half a
+    // window at a time (the later half first): the state history of the
+    // half being reversed is kept in shared memory
+    float hck[4] = {}, hmid[4];
     if (ch_ok) {
       const float4 v = *reinterpret_cast<const float4 *>(
           p.ckpt + ((b * nck + w) * E + e) * N + 4 * g);
-      hs[0] = v.x; hs[1] = v.y; hs[2] = v.z; hs[3] = v.w;
+      hck[0] = v.x; hck[1] = v.y; hck[2] = v.z; hck[3] = v.w;
     }
-    {
-      float h[4] = {hs[0], hs[1], hs[2], hs[3]};
+    // advance h over rows [r0, r0 + HALF); STORE: keep each state in sH
+    auto recompute = [&](float (&h)[4], int r0, bool store) {
 #pragma unroll 4
-      for (int r = 0; r < TW; ++r) {
+      for (int r = r0; r < r0 + HALF; ++r) {
         const float sv = sS[r * G + cl];
         const float xv = sX[r * G + cl];
         const float4 Bq = *reinterpret_cast<const float4 *>(sBF + r * N + 4 * g);
@@ -238,103 +242,126 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
           const float f = ZOH ? zoh_factor(sv, zl, a, iA[i]) : sv;
           h[i] = fmaf(a, h[i], f * xv * Bv[i]);
         }
-        sH[r * THREADS + tid] = make_float4(h[0], h[1], h[2], h[3]);
+        if (store)
+          sH[(r - r0) * THREADS + tid] = make_float4(h[0], h[1], h[2], h[3]);
       }
-    }
-
-    // ---- 4. the reverse sweep
+    };
+#pragma unroll
+    for (int i = 0; i < 4; ++i) hmid[i] = hck[i];
+    recompute(hmid, 0, false);  // the state before the later half
 #pragma unroll 1
-    for (int r = TW - 1; r >= 0; --r) {
-      const float4 hc = sH[r * THREADS + tid];
-      const float4 hp4 =
-          r > 0 ? sH[(r - 1) * THREADS + tid]
-                : make_float4(hs[0], hs[1], hs[2], hs[3]);
-      const float hcur[4] = {hc.x, hc.y, hc.z, hc.w};
-      const float hprev[4] = {hp4.x, hp4.y, hp4.z, hp4.w};
-      const float sv = sS[r * G + cl];
-      const float xv = sX[r * G + cl];
-      const float dyv = sDY[r * G + cl];
-      const float4 Bq = *reinterpret_cast<const float4 *>(sBF + r * N + 4 * g);
-      const float4 Cq = *reinterpret_cast<const float4 *>(sCF + r * N + 4 * g);
-      const float Bv[4] = {Bq.x, Bq.y, Bq.z, Bq.w};
-      const float Cv[4] = {Cq.x, Cq.y, Cq.z, Cq.w};
-      float pre = 0.0f, dxp = 0.0f, dsp = 0.0f;
-      float v8[8];
+    for (int half = 1; half >= 0; --half) {
+      const int rb = half * HALF;
+      float hst[4];  // the state before row rb
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float zl = sv * A2[i];
-        const float a = ex2(zl);
-        pre = fmaf(Cv[i], hcur[i], pre);
-        v8[4 + i] = dyv * hcur[i];       // dC
-        lam[i] = fmaf(dyv, Cv[i], lam[i]);
-        const float da = lam[i] * hprev[i];
-        if (ZOH) {
-          const float f = zoh_factor(sv, zl, a, iA[i]);
-          const float lbx = lam[i] * Bv[i] * xv;
-          dsp = fmaf(lbx, a, dsp);
-          v8[i] = lam[i] * f * xv;       // dB
-          dxp = fmaf(lam[i] * f, Bv[i], dxp);
-          dA[i] = fmaf(lbx, (sv * a - f) * iA[i], dA[i]);
-        } else {
-          dsp = fmaf(lam[i] * Bv[i], xv, dsp);
-          v8[i] = lam[i] * sv * xv;      // dB
-          dxp = fmaf(lam[i] * sv, Bv[i], dxp);
-        }
-        dsp = fmaf(da * a, Av[i], dsp);
-        dA[i] = fmaf(da * a, sv, dA[i]);
-        lam[i] *= a;
-      }
-      // per-channel sums over the channel's NG lanes (all lanes get them)
-#pragma unroll
-      for (int m = 1; m < NG; m <<= 1) {
-        pre += __shfl_xor_sync(FULL, pre, m);
-        dxp += __shfl_xor_sync(FULL, dxp, m);
-        dsp += __shfl_xor_sync(FULL, dsp, m);
-      }
-      // dB, dC summed over the warp's channels: a transposing butterfly over
-      // lane bits 4, 3, 2 leaves value j = (lane >> 2) & 7 in v8[0]; channel
-      // bits below bit 2 (NG < 4) are summed plainly
+      for (int i = 0; i < 4; ++i) hst[i] = half ? hmid[i] : hck[i];
       {
-        bool hi = lane & 16;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float send = hi ? v8[i] : v8[i + 4];
-          const float keep = hi ? v8[i + 4] : v8[i];
-          v8[i] = keep + __shfl_xor_sync(FULL, send, 16);
-        }
-        hi = lane & 8;
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const float send = hi ? v8[i] : v8[i + 2];
-          const float keep = hi ? v8[i + 2] : v8[i];
-          v8[i] = keep + __shfl_xor_sync(FULL, send, 8);
-        }
-        hi = lane & 4;
-        {
-          const float send = hi ? v8[0] : v8[1];
-          const float keep = hi ? v8[1] : v8[0];
-          v8[0] = keep + __shfl_xor_sync(FULL, send, 4);
-        }
-        if (NG <= 2) v8[0] += __shfl_xor_sync(FULL, v8[0], 2);
-        if (NG == 1) v8[0] += __shfl_xor_sync(FULL, v8[0], 1);
-        if ((lane & 3 & ~(NG - 1)) == 0) {
-          const int j = (lane >> 2) & 7;
-          atomicAdd(sAcc + r * 2 * N + (j >> 2) * N + 4 * g + (j & 3), v8[0]);
-        }
+        float h[4] = {hst[0], hst[1], hst[2], hst[3]};
+        recompute(h, rb, true);
       }
-      // the channel's outputs at step t
-      const int64_t t = t0 + r;
-      if (g == 0 && ch_ok && t < L) {
-        const int64_t i = (b * L + t) * E + e;
-        const float dxv = fmaf(dyv, Dv, dxp);
-        const float draw = dsp * sSG[r * G + cl];
-        Act<T>::store(static_cast<T *>(p.dx) + i, dxv);
-        Act<T>::store(static_cast<T *>(p.ddelta) + i, draw);
-        if (has_z)
-          Act<T>::store(static_cast<T *>(p.dz) + i,
-                        sGZ[r * G + cl] * fmaf(Dv, xv, pre));
-        sum_dD = fmaf(dyv, xv, sum_dD);
-        sum_db += draw;
+
+      // ---- 4. the reverse sweep over the half, in blocks of NG steps: the
+      // per-channel sums (C.h, the dx and d-step partials) are off the
+      // adjoint's critical path, so they are kept per step and summed over
+      // the channel's lanes once per block by a transposing butterfly that
+      // leaves lane g the totals of the block's step g, which it finishes
+#pragma unroll 1
+      for (int jb = HALF / NG - 1; jb >= 0; --jb) {
+        float pre_s[NG], dxp_s[NG], dsp_s[NG];
+#pragma unroll
+        for (int s = NG - 1; s >= 0; --s) {
+          const int r = rb + jb * NG + s;
+          const float4 hc = sH[(r - rb) * THREADS + tid];
+          const float4 hp4 =
+              r > rb ? sH[(r - rb - 1) * THREADS + tid]
+                     : make_float4(hst[0], hst[1], hst[2], hst[3]);
+          const float hcur[4] = {hc.x, hc.y, hc.z, hc.w};
+          const float hprev[4] = {hp4.x, hp4.y, hp4.z, hp4.w};
+          const float sv = sS[r * G + cl];
+          const float xv = sX[r * G + cl];
+          const float dyv = sDY[r * G + cl];
+          const float4 Bq = *reinterpret_cast<const float4 *>(sBF + r * N + 4 * g);
+          const float4 Cq = *reinterpret_cast<const float4 *>(sCF + r * N + 4 * g);
+          const float Bv[4] = {Bq.x, Bq.y, Bq.z, Bq.w};
+          const float Cv[4] = {Cq.x, Cq.y, Cq.z, Cq.w};
+          float &pre = pre_s[s], &dxp = dxp_s[s], &dsp = dsp_s[s];
+          pre = dxp = dsp = 0.0f;
+          float v8[8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float zl = sv * A2[i];
+            const float a = ex2(zl);
+            pre = fmaf(Cv[i], hcur[i], pre);
+            v8[4 + i] = dyv * hcur[i];       // dC
+            lam[i] = fmaf(dyv, Cv[i], lam[i]);
+            const float da = lam[i] * hprev[i];
+            if (ZOH) {
+              const float f = zoh_factor(sv, zl, a, iA[i]);
+              const float lbx = lam[i] * Bv[i] * xv;
+              dsp = fmaf(lbx, a, dsp);
+              v8[i] = lam[i] * f * xv;       // dB
+              dxp = fmaf(lam[i] * f, Bv[i], dxp);
+              dA[i] = fmaf(lbx, (sv * a - f) * iA[i], dA[i]);
+            } else {
+              dsp = fmaf(lam[i] * Bv[i], xv, dsp);
+              v8[i] = lam[i] * sv * xv;      // dB
+              dxp = fmaf(lam[i] * sv, Bv[i], dxp);
+            }
+            dsp = fmaf(da * a, Av[i], dsp);
+            dA[i] = fmaf(da * a, sv, dA[i]);
+            lam[i] *= a;
+          }
+          // dB, dC summed over the warp's channels: a transposing butterfly over
+          // lane bits 4, 3, 2 leaves value j = (lane >> 2) & 7 in v8[0]; channel
+          // bits below bit 2 (NG < 4) are summed plainly
+          {
+            bool hi = lane & 16;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float send = hi ? v8[i] : v8[i + 4];
+              const float keep = hi ? v8[i + 4] : v8[i];
+              v8[i] = keep + __shfl_xor_sync(FULL, send, 16);
+            }
+            hi = lane & 8;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const float send = hi ? v8[i] : v8[i + 2];
+              const float keep = hi ? v8[i + 2] : v8[i];
+              v8[i] = keep + __shfl_xor_sync(FULL, send, 8);
+            }
+            hi = lane & 4;
+            {
+              const float send = hi ? v8[0] : v8[1];
+              const float keep = hi ? v8[1] : v8[0];
+              v8[0] = keep + __shfl_xor_sync(FULL, send, 4);
+            }
+            if (NG <= 2) v8[0] += __shfl_xor_sync(FULL, v8[0], 2);
+            if (NG == 1) v8[0] += __shfl_xor_sync(FULL, v8[0], 1);
+            if ((lane & 3 & ~(NG - 1)) == 0) {
+              const int j = (lane >> 2) & 7;
+              atomicAdd(sAcc + r * 2 * N + (j >> 2) * N + 4 * g + (j & 3), v8[0]);
+            }
+          }
+        }
+        const float pre = transpose_reduce<NG, 1>(pre_s, g);
+        const float dxp = transpose_reduce<NG, 1>(dxp_s, g);
+        const float dsp = transpose_reduce<NG, 1>(dsp_s, g);
+        const int r = rb + jb * NG + g;
+        const int64_t t = t0 + r;
+        if (ch_ok && t < L) {
+          const int64_t i = (b * L + t) * E + e;
+          const float dyv = sDY[r * G + cl];
+          const float xv = sX[r * G + cl];
+          const float dxv = fmaf(dyv, Dv, dxp);
+          const float draw = dsp * sSG[r * G + cl];
+          Act<T>::store(static_cast<T *>(p.dx) + i, dxv);
+          Act<T>::store(static_cast<T *>(p.ddelta) + i, draw);
+          if (has_z)
+            Act<T>::store(static_cast<T *>(p.dz) + i,
+                          sGZ[r * G + cl] * fmaf(Dv, xv, pre));
+          sum_dD = fmaf(dyv, xv, sum_dD);
+          sum_db += draw;
+        }
       }
     }
     __syncthreads();
@@ -351,6 +378,12 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
     __syncthreads();
   }
   cp_async_wait<0>();
+  // every lane of a channel finished some of its steps: sum the partials
+#pragma unroll
+  for (int m = 1; m < NG; m <<= 1) {
+    sum_dD += __shfl_xor_sync(FULL, sum_dD, m);
+    sum_db += __shfl_xor_sync(FULL, sum_db, m);
+  }
 
   if (ch_ok) {
     if (p.dh0)

@@ -247,17 +247,29 @@ int launch_step_cfg(const ssm::StepParams &p, bool vec, int sm_count,
   const int64_t threads = p.dim * QP;
   const int64_t bx = (threads + 127) / 128;
   if (bx > 0x7fffffff) return SSM_ERR_UNSUPPORTED;
-  // enough batch-row strides to give every SM about 8 blocks; each thread
-  // walks batch / grid.y rows with its channel's constants in registers
-  int64_t by = (int64_t(sm_count) * 8 + bx - 1) / bx;
+  auto kern = vec ? ssm::scan_step_kernel<T, SPT, QP, true>
+                  : ssm::scan_step_kernel<T, SPT, QP, false>;
+  // one wave: as many batch-row strides as leave every block resident at
+  // once (each thread walks batch / grid.y rows with its channel's
+  // constants in registers), so no block starts late
+  static int occupancy[2] = {0, 0};  // resident blocks per SM, per kernel
+  int &per_sm = occupancy[vec ? 1 : 0];
+  if (per_sm < 1) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 128, 0) !=
+            cudaSuccess ||
+        n < 1) {
+      cudaGetLastError();
+      n = 1;
+    }
+    per_sm = n;
+  }
+  int64_t by = int64_t(sm_count) * per_sm / bx;
   if (by > p.batch) by = p.batch;
   if (by > 65535) by = 65535;
   if (by < 1) by = 1;
   const dim3 grid{static_cast<unsigned>(bx), static_cast<unsigned>(by), 1u};
-  if (vec)
-    ssm::scan_step_kernel<T, SPT, QP, true><<<grid, 128, 0, s>>>(p);
-  else
-    ssm::scan_step_kernel<T, SPT, QP, false><<<grid, 128, 0, s>>>(p);
+  kern<<<grid, 128, 0, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
