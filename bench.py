@@ -453,39 +453,66 @@ def run_gpu(args):
     if args.no_e2e:
         return _finish(args, op, world, rank, local, dev, dist, scan, clocks,
                        total_ms, kernel_ms, variant, None, 0, 0)
+    # Each step copies its own inputs in from pinned host memory and its own
+    # outputs back, all inside the timed region. Inputs are double-buffered:
+    # step i+1's host-to-device copy (its own stream) overlaps step i's
+    # kernel and device-to-host copy (a third stream); a buffer is refilled
+    # only after the kernel that read it has finished, and a kernel starts
+    # only after the previous step's outputs have been copied out.
     host = {k: (None if v is None else v.cpu().pin_memory())
             for k, v in t.items()}
-    outs = op.outputs()
-    out_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory()
-                for o in outs]
-    dev_in = {k: (None if v is None else torch.empty_like(v))
-              for k, v in t.items()}
+    dev_in = [{k: (None if v is None else torch.empty_like(v))
+               for k, v in t.items()} for _ in range(2)]
+    for buf in dev_in:
+        for k, v in host.items():
+            if v is not None:
+                buf[k].copy_(v)
     h2d = sum(host[k].numel() * host[k].element_size()
               for k in op.per_step_in if host.get(k) is not None)
+    op.run(dev_in[0], stream)
+    out_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory()
+                for o in op.outputs()]
     d2h = sum(o.numel() * o.element_size() for o in out_host)
-    for k, v in host.items():
-        if v is not None:
-            dev_in[k].copy_(v)
+    s_h2d = torch.cuda.Stream(dev)
+    s_d2h = torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_free = [torch.cuda.Event() for _ in range(2)]
+    ev_out = torch.cuda.Event()
+    ev_d2h = torch.cuda.Event()
+    torch.cuda.synchronize(dev)
 
-    def e2e_step():
-        for k in op.per_step_in:
-            if host.get(k) is not None:
-                dev_in[k].copy_(host[k], non_blocking=True)
-        op.run(dev_in, stream)
-        for o, oh in zip(outs, out_host):
-            oh.copy_(o, non_blocking=True)
+    def e2e_step(i):
+        j = i % 2
+        s_h2d.wait_event(ev_free[j])
+        with torch.cuda.stream(s_h2d):
+            for k in op.per_step_in:
+                if host.get(k) is not None:
+                    dev_in[j][k].copy_(host[k], non_blocking=True)
+        ev_in[j].record(s_h2d)
+        stream.wait_event(ev_in[j])
+        stream.wait_event(ev_d2h)
+        op.run(dev_in[j], stream)
+        ev_free[j].record(stream)
+        outs = op.outputs()
+        ev_out.record(stream)
+        s_d2h.wait_event(ev_out)
+        with torch.cuda.stream(s_d2h):
+            for o, oh in zip(outs, out_host):
+                o.record_stream(s_d2h)
+                oh.copy_(o, non_blocking=True)
+        ev_d2h.record(s_d2h)
 
     e2e_steps = max(3, min(args.steps, args.e2e_steps))
-    for _ in range(2):
-        e2e_step()
+    for i in range(2):
+        e2e_step(i)
     torch.cuda.synchronize(dev)
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
+    e0.record(s_h2d)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e1.record(s_d2h)
     torch.cuda.synchronize(dev)
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps,
