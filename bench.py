@@ -75,6 +75,12 @@ def max_over_ranks(value: float, dist=None, device=None) -> float:
 
 # ----------------------------------------------------------------- workload
 CONV_WIDTH = 4
+
+# DRAM bytes (read + write) of one launch of the timed kernel, from the ncu
+# capture summarised in profiles/scan_chunked_mamba2p8b_layer.md (current
+# build of the chunked kernel, Mamba-2.8B layer). Workloads without a capture
+# of their current kernel report null.
+NCU_TRAFFIC = {("scan", 3): 1.009863e9 + 0.316763e9}
 DECODE_BATCH = 1024
 
 
@@ -562,7 +568,8 @@ def _finish(args, op, world, rank, local, dev, dist, scan, clocks, total_ms,
                                              peaks["source"]),
                 "frac_at_sampled_clock": (achieved_exp / sfu_peak_run
                                           if sfu_peak_run else None),
-                "traffic": None}
+                "traffic": NCU_TRAFFIC.get((op.name, args.shape)),
+                "algorithmic_bytes": nbytes}
         l2 = "inputs larger than L2 (%.0f MB read per step)" % (nbytes / 1e6)
     line = {
         "metric": metric, "value": value, "unit": unit, "n_gpus": world,
@@ -585,8 +592,8 @@ def _finish(args, op, world, rank, local, dev, dist, scan, clocks, total_ms,
     if op.name == "bwd":
         line["roofline"]["peak_note"] += (
             "; one retention exp per element counted (the pass evaluates "
-            "three: the checkpointing forward, the window recompute and the "
-            "reverse sweep)")
+            "about four: the checkpointing forward, 1.5 in the window "
+            "recompute, the reverse sweep, and the pre-pass slopes)")
     if op.name != "step":
         line["roofline_min_hbm_sfu"] = {
             "t_hbm_us": t_hbm * 1e6, "t_sfu_us_at_max_clock": t_sfu * 1e6,

@@ -62,7 +62,11 @@ struct BwdCfg {
   // per-window float arrays: s, x, dy, gate slope, softplus slope [TW][G];
   // B, C [TW][N]; the states of half a window [TW/2][THREADS] float4; dB,
   // dC sums [TW][2N]
-  static constexpr int SCAL_BYTES = 5 * TW * G * 4;
+  // row stride of the per-(t, e) arrays: the G channels plus 32 / NG words,
+  // so that the NG lanes of a channel, which finish NG consecutive steps,
+  // read distinct banks
+  static constexpr int SP = G + (NG > 1 ? 32 / NG : 0);
+  static constexpr int SCAL_BYTES = 5 * TW * SP * 4;
   static constexpr int BCF_BYTES = 2 * TW * N * 4;
   static constexpr int HALF = TW / 2;  // rows of state history kept at once
   static constexpr int HIST_BYTES = HALF * THREADS * 16;
@@ -79,6 +83,7 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
   using Cfg = BwdCfg<T, NG, NW>;
   constexpr int N = Cfg::N, CW = Cfg::CW, G = Cfg::G, TW = Cfg::TW;
   constexpr int THREADS = Cfg::THREADS, ESZ = Cfg::ESZ, HALF = Cfg::HALF;
+  constexpr int SP = Cfg::SP;
   constexpr unsigned FULL = 0xffffffffu;
   extern __shared__ __align__(16) unsigned char smem[];
 
@@ -96,11 +101,11 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
   const int64_t nck = (L + TW - 1) / TW;
 
   float *const sS = reinterpret_cast<float *>(smem + 2 * Cfg::STAGE);
-  float *const sX = sS + TW * G;
-  float *const sDY = sX + TW * G;
-  float *const sGZ = sDY + TW * G;
-  float *const sSG = sGZ + TW * G;
-  float *const sBF = sSG + TW * G;
+  float *const sX = sS + TW * SP;
+  float *const sDY = sX + TW * SP;
+  float *const sGZ = sDY + TW * SP;
+  float *const sSG = sGZ + TW * SP;
+  float *const sBF = sSG + TW * SP;
   float *const sCF = sBF + TW * N;
   float4 *const sH = reinterpret_cast<float4 *>(sCF + TW * N);
   float *const sAcc = reinterpret_cast<float *>(sH + Cfg::HALF * THREADS);
@@ -202,11 +207,12 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
         sv = softplus(raw);
         slope = rcp(1.0f + ex2(-raw * kLog2e));
       }
-      sS[idx] = ok ? sv : 0.0f;
-      sX[idx] = ok ? xv : 0.0f;
-      sDY[idx] = ok ? dyv : 0.0f;
-      sGZ[idx] = ok ? gzv : 0.0f;
-      sSG[idx] = slope;
+      const int so = r * SP + pc;
+      sS[so] = ok ? sv : 0.0f;
+      sX[so] = ok ? xv : 0.0f;
+      sDY[so] = ok ? dyv : 0.0f;
+      sGZ[so] = ok ? gzv : 0.0f;
+      sSG[so] = slope;
     }
     {
       const unsigned char *bc = base + 4 * Cfg::ACT_BYTES;
@@ -231,16 +237,27 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
     auto recompute = [&](float (&h)[4], int r0, bool store) {
 #pragma unroll 4
       for (int r = r0; r < r0 + HALF; ++r) {
-        const float sv = sS[r * G + cl];
-        const float xv = sX[r * G + cl];
+        const float sv = sS[r * SP + cl];
+        const float xv = sX[r * SP + cl];
         const float4 Bq = *reinterpret_cast<const float4 *>(sBF + r * N + 4 * g);
-        const float Bv[4] = {Bq.x, Bq.y, Bq.z, Bq.w};
+        if constexpr (ZOH) {
+          const float Bv[4] = {Bq.x, Bq.y, Bq.z, Bq.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float zl = sv * A2[i];
-          const float a = ex2(zl);
-          const float f = ZOH ? zoh_factor(sv, zl, a, iA[i]) : sv;
-          h[i] = fmaf(a, h[i], f * xv * Bv[i]);
+          for (int i = 0; i < 4; ++i) {
+            const float zl = sv * A2[i];
+            const float a = ex2(zl);
+            h[i] = fmaf(a, h[i], zoh_factor(sv, zl, a, iA[i]) * xv * Bv[i]);
+          }
+        } else {  // packed pairs: a = 2^(s A'), h = a h + (s x) B
+          const float2 s2 = make_float2(sv, sv);
+          const float2 sx2 = make_float2(sv * xv, sv * xv);
+          const float2 a01 = ex2x2(mul2(s2, make_float2(A2[0], A2[1])));
+          const float2 a23 = ex2x2(mul2(s2, make_float2(A2[2], A2[3])));
+          const float2 h01 = fma2(a01, make_float2(h[0], h[1]),
+                                  mul2(sx2, make_float2(Bq.x, Bq.y)));
+          const float2 h23 = fma2(a23, make_float2(h[2], h[3]),
+                                  mul2(sx2, make_float2(Bq.z, Bq.w)));
+          h[0] = h01.x; h[1] = h01.y; h[2] = h23.x; h[3] = h23.y;
         }
         if (store)
           sH[(r - r0) * THREADS + tid] = make_float4(h[0], h[1], h[2], h[3]);
@@ -277,9 +294,9 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
                      : make_float4(hst[0], hst[1], hst[2], hst[3]);
           const float hcur[4] = {hc.x, hc.y, hc.z, hc.w};
           const float hprev[4] = {hp4.x, hp4.y, hp4.z, hp4.w};
-          const float sv = sS[r * G + cl];
-          const float xv = sX[r * G + cl];
-          const float dyv = sDY[r * G + cl];
+          const float sv = sS[r * SP + cl];
+          const float xv = sX[r * SP + cl];
+          const float dyv = sDY[r * SP + cl];
           const float4 Bq = *reinterpret_cast<const float4 *>(sBF + r * N + 4 * g);
           const float4 Cq = *reinterpret_cast<const float4 *>(sCF + r * N + 4 * g);
           const float Bv[4] = {Bq.x, Bq.y, Bq.z, Bq.w};
@@ -287,29 +304,63 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
           float &pre = pre_s[s], &dxp = dxp_s[s], &dsp = dsp_s[s];
           pre = dxp = dsp = 0.0f;
           float v8[8];
+          if constexpr (!ZOH) {
+            // packed pairs of states; sum_n lam B gives both the dx and the
+            // write part of the step-size partial: dx = s sum lam B,
+            // d step = x sum lam B + sum (lam h_{t-1} a) A
+            const float2 s2 = make_float2(sv, sv), dy2 = make_float2(dyv, dyv);
+            const float2 hc01 = make_float2(hcur[0], hcur[1]);
+            const float2 hc23 = make_float2(hcur[2], hcur[3]);
+            const float2 B01 = make_float2(Bv[0], Bv[1]);
+            const float2 B23 = make_float2(Bv[2], Bv[3]);
+            const float2 C01 = make_float2(Cv[0], Cv[1]);
+            const float2 C23 = make_float2(Cv[2], Cv[3]);
+            const float2 a01 = ex2x2(mul2(s2, make_float2(A2[0], A2[1])));
+            const float2 a23 = ex2x2(mul2(s2, make_float2(A2[2], A2[3])));
+            const float2 pr = fma2(C23, hc23, mul2(C01, hc01));
+            pre = pr.x + pr.y;
+            const float2 dC01 = mul2(dy2, hc01), dC23 = mul2(dy2, hc23);
+            float2 l01 = fma2(dy2, C01, make_float2(lam[0], lam[1]));
+            float2 l23 = fma2(dy2, C23, make_float2(lam[2], lam[3]));
+            const float2 lb = fma2(l23, B23, mul2(l01, B01));
+            const float slb = lb.x + lb.y;
+            const float2 sx2 = make_float2(sv * xv, sv * xv);
+            const float2 dB01 = mul2(l01, sx2), dB23 = mul2(l23, sx2);
+            const float2 g01 =
+                mul2(mul2(l01, make_float2(hprev[0], hprev[1])), a01);
+            const float2 g23 =
+                mul2(mul2(l23, make_float2(hprev[2], hprev[3])), a23);
+            const float2 gA = fma2(g23, make_float2(Av[2], Av[3]),
+                                   mul2(g01, make_float2(Av[0], Av[1])));
+            dsp = fmaf(xv, slb, gA.x + gA.y);
+            dxp = sv * slb;
+            const float2 dA01 = fma2(g01, s2, make_float2(dA[0], dA[1]));
+            const float2 dA23 = fma2(g23, s2, make_float2(dA[2], dA[3]));
+            dA[0] = dA01.x; dA[1] = dA01.y; dA[2] = dA23.x; dA[3] = dA23.y;
+            l01 = mul2(l01, a01);
+            l23 = mul2(l23, a23);
+            lam[0] = l01.x; lam[1] = l01.y; lam[2] = l23.x; lam[3] = l23.y;
+            v8[0] = dB01.x; v8[1] = dB01.y; v8[2] = dB23.x; v8[3] = dB23.y;
+            v8[4] = dC01.x; v8[5] = dC01.y; v8[6] = dC23.x; v8[7] = dC23.y;
+          } else {  // zero-order-hold write f = expm1(s A) / A, per state
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float zl = sv * A2[i];
-            const float a = ex2(zl);
-            pre = fmaf(Cv[i], hcur[i], pre);
-            v8[4 + i] = dyv * hcur[i];       // dC
-            lam[i] = fmaf(dyv, Cv[i], lam[i]);
-            const float da = lam[i] * hprev[i];
-            if (ZOH) {
+            for (int i = 0; i < 4; ++i) {
+              const float zl = sv * A2[i];
+              const float a = ex2(zl);
+              pre = fmaf(Cv[i], hcur[i], pre);
+              v8[4 + i] = dyv * hcur[i];       // dC
+              lam[i] = fmaf(dyv, Cv[i], lam[i]);
+              const float da = lam[i] * hprev[i];
               const float f = zoh_factor(sv, zl, a, iA[i]);
               const float lbx = lam[i] * Bv[i] * xv;
               dsp = fmaf(lbx, a, dsp);
-              v8[i] = lam[i] * f * xv;       // dB
+              v8[i] = lam[i] * f * xv;         // dB
               dxp = fmaf(lam[i] * f, Bv[i], dxp);
               dA[i] = fmaf(lbx, (sv * a - f) * iA[i], dA[i]);
-            } else {
-              dsp = fmaf(lam[i] * Bv[i], xv, dsp);
-              v8[i] = lam[i] * sv * xv;      // dB
-              dxp = fmaf(lam[i] * sv, Bv[i], dxp);
+              dsp = fmaf(da * a, Av[i], dsp);
+              dA[i] = fmaf(da * a, sv, dA[i]);
+              lam[i] *= a;
             }
-            dsp = fmaf(da * a, Av[i], dsp);
-            dA[i] = fmaf(da * a, sv, dA[i]);
-            lam[i] *= a;
           }
           // dB, dC summed over the warp's channels: a transposing butterfly over
           // lane bits 4, 3, 2 leaves value j = (lane >> 2) & 7 in v8[0]; channel
@@ -350,15 +401,15 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
         const int64_t t = t0 + r;
         if (ch_ok && t < L) {
           const int64_t i = (b * L + t) * E + e;
-          const float dyv = sDY[r * G + cl];
-          const float xv = sX[r * G + cl];
+          const float dyv = sDY[r * SP + cl];
+          const float xv = sX[r * SP + cl];
           const float dxv = fmaf(dyv, Dv, dxp);
-          const float draw = dsp * sSG[r * G + cl];
+          const float draw = dsp * sSG[r * SP + cl];
           Act<T>::store(static_cast<T *>(p.dx) + i, dxv);
           Act<T>::store(static_cast<T *>(p.ddelta) + i, draw);
           if (has_z)
             Act<T>::store(static_cast<T *>(p.dz) + i,
-                          sGZ[r * G + cl] * fmaf(Dv, xv, pre));
+                          sGZ[r * SP + cl] * fmaf(Dv, xv, pre));
           sum_dD = fmaf(dyv, xv, sum_dD);
           sum_db += draw;
         }
