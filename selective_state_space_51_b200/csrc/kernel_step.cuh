@@ -71,8 +71,19 @@ __device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16 *p,
 // group moves as SPT/4 16-byte accesses issued before any arithmetic, and
 // the channel's scalars (convolution, step size, gates) are computed once.
 // VEC: N % 4 == 0 and the state, B and C allow 4-element vector accesses.
+// Shared memory per 128-thread block: each thread's A log2(e) (SPT floats) and
+// filter taps (kMaxConvWidth floats), in rows padded by 4 words so that the
+// 16-byte reads of 8 consecutive threads fall in distinct banks. Each thread
+// reads back only its own rows, so no barrier is needed.
+template <int SPT>
+struct StepSmem {
+  static constexpr int A_ROW = SPT + 4, W_ROW = kMaxConvWidth + 4;
+  static constexpr int BYTES = 128 * (A_ROW + W_ROW) * 4;
+};
+
 template <typename T, int SPT, int QP, bool VEC>
 __global__ void __launch_bounds__(128) scan_step_kernel(const StepParams p) {
+  extern __shared__ __align__(16) float step_smem[];
   const int64_t tx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int q = int(tx % QP);
   const int64_t e = tx / QP;
@@ -83,21 +94,20 @@ __global__ void __launch_bounds__(128) scan_step_kernel(const StepParams p) {
   const int K = p.conv_width;
   const bool vec = VEC && n0 + SPT <= N;
 
-  // ---- the channel's constants, once
-  float A2[SPT];
+  // ---- the channel's constants, once, into this thread's shared rows
+  float *const A2 = step_smem + threadIdx.x * StepSmem<SPT>::A_ROW;
+  float *const cw = step_smem + 128 * StepSmem<SPT>::A_ROW +
+                    threadIdx.x * StepSmem<SPT>::W_ROW;
 #pragma unroll
   for (int i = 0; i < SPT; ++i)
     A2[i] = live && n0 + i < N
                 ? fmaxf(-expf(p.A_log[es * N + n0 + i]) * kLog2e, -FLT_MAX)
                 : 0.0f;
-  float cw[kMaxConvWidth] = {};
   float cbias = 0.0f;
-  if (p.conv_state && live) {
 #pragma unroll
-    for (int j = 0; j < kMaxConvWidth; ++j)
-      if (j < K) cw[j] = p.conv_weight[es * K + j];
-    cbias = p.conv_bias ? p.conv_bias[es] : 0.0f;
-  }
+  for (int j = 0; j < kMaxConvWidth; ++j)
+    cw[j] = (p.conv_state && live && j < K) ? p.conv_weight[es * K + j] : 0.0f;
+  if (p.conv_state && live) cbias = p.conv_bias ? p.conv_bias[es] : 0.0f;
   const float dbias = (live && p.delta_bias) ? p.delta_bias[es] : 0.0f;
   const float Dv = (live && p.D) ? p.D[es] : 0.0f;
 
@@ -126,10 +136,15 @@ __global__ void __launch_bounds__(128) scan_step_kernel(const StepParams p) {
     float acc = cbias;
     if (live && p.conv_state) {
       buf = static_cast<T *>(p.conv_state) + ch * K;
+      // the taps as two 16-byte reads of this thread's row
+      const float4 w0 = *reinterpret_cast<const float4 *>(cw);
+      const float4 w1 = *reinterpret_cast<const float4 *>(cw + 4);
+      const float taps[kMaxConvWidth] = {w0.x, w0.y, w0.z, w0.w,
+                                         w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
       for (int j = 0; j < kMaxConvWidth; ++j)
         if (j < K)
-          acc = fmaf(j + 1 < K ? Act<T>::load(buf + j + 1) : xv, cw[j], acc);
+          acc = fmaf(j + 1 < K ? Act<T>::load(buf + j + 1) : xv, taps[j], acc);
     }
     if (QP > 1) __syncwarp();  // the channel's threads have read the buffer
     if (buf) {
@@ -165,11 +180,13 @@ __global__ void __launch_bounds__(128) scan_step_kernel(const StepParams p) {
             Cv[i] = n0 + i0 + i < N ? Act<T>::load(Cm + i0 + i) : 0.0f;
           }
         }
+        const float4 a4 = *reinterpret_cast<const float4 *>(A2 + i0);
+        const float Aq[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int k = i0 + i;
           if (n0 + k < N) {
-            const float zl = step * A2[k];
+            const float zl = step * Aq[i];
             const float a = ex2(zl);
             const float wf =
                 p.write_zoh

@@ -256,8 +256,8 @@ int launch_step_cfg(const ssm::StepParams &p, bool vec, int sm_count,
   int &per_sm = occupancy[vec ? 1 : 0];
   if (per_sm < 1) {
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 128, 0) !=
-            cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &n, kern, 128, ssm::StepSmem<SPT>::BYTES) != cudaSuccess ||
         n < 1) {
       cudaGetLastError();
       n = 1;
@@ -269,7 +269,7 @@ int launch_step_cfg(const ssm::StepParams &p, bool vec, int sm_count,
   if (by > 65535) by = 65535;
   if (by < 1) by = 1;
   const dim3 grid{static_cast<unsigned>(bx), static_cast<unsigned>(by), 1u};
-  kern<<<grid, 128, 0, s>>>(p);
+  kern<<<grid, 128, ssm::StepSmem<SPT>::BYTES, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
