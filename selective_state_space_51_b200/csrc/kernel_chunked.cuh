@@ -521,7 +521,7 @@ scan_chunked_kernel(const ScanParams p) {
         float2 x2, z2, e0, e1;
         produce2(0, 0, x2, z2, e0, e1, std::true_type());
         __syncwarp();
-#pragma unroll 2
+#pragma unroll 4
         for (int jb = 0; jb < NBW; ++jb) {
           const int par = jb & 1;
           if constexpr (!SPLIT) {

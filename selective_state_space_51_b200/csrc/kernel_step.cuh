@@ -81,8 +81,11 @@ struct StepSmem {
   static constexpr int BYTES = 128 * (A_ROW + W_ROW) * 4;
 };
 
+// The vectorised kernels are held to 64 registers (8 blocks per SM): the step
+// is latency-bound, and the extra resident warps keep more loads in flight.
 template <typename T, int SPT, int QP, bool VEC>
-__global__ void __launch_bounds__(128) scan_step_kernel(const StepParams p) {
+__global__ void __launch_bounds__(128, VEC ? 8 : 1)
+    scan_step_kernel(const StepParams p) {
   extern __shared__ __align__(16) float step_smem[];
   const int64_t tx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int q = int(tx % QP);
