@@ -80,7 +80,7 @@ CONV_WIDTH = 4
 # capture summarised in profiles/scan_chunked_mamba2p8b_layer.md (current
 # build of the chunked kernel, Mamba-2.8B layer). Workloads without a capture
 # of their current kernel report null.
-NCU_TRAFFIC = {("scan", 3): 1.009863e9 + 0.316763e9}
+NCU_TRAFFIC = {("scan", 3): 1.010016e9 + 0.316603e9}
 DECODE_BATCH = 1024
 
 
@@ -589,6 +589,15 @@ def _finish(args, op, world, rank, local, dev, dist, scan, clocks, total_ms,
         "gpu_launches": args.steps * op.launches_per_step,
         "clocks": clk,
     }
+    if op.name != "step":
+        # the exp2 rate measured on this GPU right after the timed region
+        try:
+            import selective_state_space_51_b200 as S
+            rate = S.ssm_measure_ex2_rate(local)
+            line["roofline"]["ex2_measured_gexp_s"] = rate / 1e9
+            line["roofline"]["frac_of_measured_ex2"] = achieved_exp / rate
+        except Exception as exc:  # reported, never fatal to the bench line
+            line["roofline"]["ex2_measured_error"] = str(exc)[:200]
     if op.name == "bwd":
         line["roofline"]["peak_note"] += (
             "; one retention exp per element counted (the pass evaluates "

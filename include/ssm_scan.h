@@ -334,6 +334,19 @@ SSM_API int ssm_scan_fwd_static_scratch(
     struct CUstream_st *stream);
 
 /* ssm_scan_status_string: static English text for a status code. */
+/*
+ * ssm_measure_ex2_rate: the measured throughput of the SFU's exp2 on `device`
+ * (MUFU.EX2 operations per second, all SMs, at whatever clock the device runs):
+ * a kernel of independent exp2 chains, 2048 threads per SM, timed over five
+ * launches of about 2e11 operations (about 40 ms). The scan's roofline divides its
+ * one-exp-per-element count by this unit; the pages have no counterpart, it
+ * confirms the rate the roofline derives from the SM count, 16 ex2 per clock per
+ * SM and the clock. Allocates 4 bytes of device memory and synchronizes the
+ * device. Returns SSM_ERR_INVALID for a NULL output or a bad device,
+ * SSM_ERR_CUDA on a runtime error.
+ */
+SSM_API int ssm_measure_ex2_rate(int device, double *ex2_per_second);
+
 SSM_API const char *ssm_scan_status_string(int status);
 
 #ifdef __cplusplus

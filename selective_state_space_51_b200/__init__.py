@@ -96,6 +96,9 @@ def library() -> ctypes.CDLL:
                 i32, vp, vp, vp, vp, vp, vp, vp, vp, u32, vp, vp, vp,
                 ssm_scan_dims, i32, i32, vp, vp]
             lib.ssm_scan_fwd_static_scratch.restype = i32
+            lib.ssm_measure_ex2_rate.argtypes = [i32,
+                                                 ctypes.POINTER(ctypes.c_double)]
+            lib.ssm_measure_ex2_rate.restype = i32
             lib.ssm_scan_status_string.argtypes = [i32]
             lib.ssm_scan_status_string.restype = ctypes.c_char_p
             _lib = lib
@@ -123,6 +126,15 @@ def _check(status: int, where: str) -> int:
     if status != SSM_OK:
         raise SsmScanError(status, where)
     return status
+
+
+def ssm_measure_ex2_rate(device: int = 0) -> float:
+    """Measured MUFU exp2 operations per second on ``device`` (see
+    include/ssm_scan.h)."""
+    out = ctypes.c_double(0.0)
+    _check(library().ssm_measure_ex2_rate(int(device), ctypes.byref(out)),
+           "ssm_measure_ex2_rate")
+    return out.value
 
 
 def ssm_scan_status_string(status: int) -> str:
