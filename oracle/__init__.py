@@ -13,11 +13,20 @@ channel's state" and "5. Put the selective operator inside the complete mixer".
 The loop itself is plain C (``ssm_oracle.c``), compiled with gcc at -O2 without
 fast-math, run in float64 on inputs widened exactly from float32 or bfloat16.
 
+Beyond the scan it holds, from the same page: the scan with the causal
+depthwise convolution and SiLU in front (rows "4. Add causal local context
+before selecting coefficients" and 5), the batched decode step with its conv
+buffer (row "6. Carry both buffers to the next token"), the exact
+zero-order-hold write option, and the backward pass (reverse-mode gradients of
+the scan, recomputing each channel's states).
+
 Every function here is pinned by ``tests/test_oracle_pins.py`` to facts the
 pages and the mathematics fix (associative-prefix agreement over every
 bracketing, the LTI convolution closed form, forgetting and freezing limits,
 retention bounds, continuation, the one-token decode step, linearity, channel
-independence, degenerate skips).
+independence, degenerate skips, the zero-order-hold closed forms, numpy's
+causal convolution, and central finite differences of the forward for every
+gradient).
 """
 from __future__ import annotations
 

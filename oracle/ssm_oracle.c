@@ -47,6 +47,10 @@
  *
  * Parallelism: independent (batch, channel) pairs are spread over OpenMP
  * threads; each pair's loop over time stays strictly sequential.
+ *
+ * Further entry points, each with its own citation below: the decode step
+ * (ssm_oracle_step), the scan with the causal convolution in front
+ * (ssm_oracle_scan_conv) and the backward pass (ssm_oracle_scan_bwd).
  */
 #include <math.h>
 #include <stdint.h>
