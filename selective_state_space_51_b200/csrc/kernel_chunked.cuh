@@ -24,12 +24,17 @@
 // Per window: x, raw delta, z tiles [TW x G] and B, C tiles [TW x N] are
 // staged in shared memory with cp.async (double buffered, one window ahead;
 // rows padded so every lane access pattern is bank-conflict free); bfloat16
-// B and C are widened to float32 once per window. In each block of NG steps
-// lane g computes softplus for step g only and publishes (delta, delta*x) in
-// a per-warp exchange slot, so every (t, e) pays its softplus once. Readout
-// partials over each lane's 4 states are combined over the NG lanes by a
-// transposing butterfly that leaves lane g holding the full y of the block's
-// step g; lane g adds D x, applies the SiLU gate and stores.
+// B and C are widened to float32 once per window. With TB == 1 the steps go
+// in blocks of 2 NG: lane g computes the step sizes of steps 2g and 2g+1
+// (softplus on a packed pair) and publishes (delta, delta*x) for both in its
+// channel's exchange row, so every (t, e) pays its softplus once; one block's
+// step sizes are formed while the previous block's states are updated.
+// Readout partials over each lane's 4 states are combined over the NG lanes
+// by a transposing butterfly that leaves lane g the full y of steps 2g and
+// 2g+1; lane g adds D x, applies the SiLU gate and stores. (With TB > 1 the
+// blocks are NG steps, one per lane.) Options: the exact zero-order-hold
+// write (ZOH), the causal convolution + SiLU that forms x from the staged
+// input tile (CONV), and state checkpoints for the backward pass.
 //
 // Split sequences (SPLIT). For few channels and long sequences each sequence
 // is cut into pieces scanned concurrently. A piece starts from a zero state,
