@@ -184,8 +184,8 @@ SSM_API int ssm_scan_fwd_conv(ssm_scan_t h, const void *v,
  * runnable CPU code", rows 1, 2 and 5; the states are recomputed on the way
  * back rather than stored, as section "Compose the updates instead of
  * waiting for every state" describes). Two launches on `stream`: the forward
- * with a state checkpoint every 16 steps into a workspace the handle grows
- * (b * ceil(L / 16) * dim * dstate floats; SSM_ERR_NOMEM if it cannot), then
+ * with a state checkpoint every 8 steps into a workspace the handle grows
+ * (b * ceil(L / 8) * dim * dstate floats; SSM_ERR_NOMEM if it cannot), then
  * a reverse sweep from those checkpoints.
  *   inputs     : as ssm_scan_fwd (x, delta, A_log, B, C, D, z, delta_bias,
  *                flags, h0); dy [batch, seqlen, dim] activation dtype,

@@ -22,14 +22,16 @@
 //      cp.async (the previous window's are already in flight);
 //   2. a pre-pass forms each (t, e)'s step size, x, dy, gate slope and
 //      softplus slope once, in shared memory;
-//   3. every lane recomputes its 4 states through the window from the
-//      forward's checkpoint (the state before the window), keeping them in
-//      shared memory;
-//   4. the reverse sweep updates lam in registers; per-channel sums over a
-//      channel's NG lanes are a shuffle butterfly, and the sums of dB and dC
-//      over the tile's channels a transposing butterfly over the warp's
-//      channels followed by shared-memory accumulation across warps, added to
-//      HBM once per (t, n) and block.
+//   3. for each half window (one 8-step checkpoint interval), the later
+//      half first, every lane recomputes its 4 states from the forward's
+//      checkpoint at the start of that half, keeping them in shared memory;
+//   4. the reverse sweep over the half updates lam in registers. The
+//      per-channel sums (C.h, the dx and d-step partials) are buffered over
+//      NG steps and summed over the channel's lanes by one transposing
+//      butterfly; the sums of dB and dC over the tile's channels are a
+//      transposing butterfly over the warp's channel lanes followed by
+//      shared-memory accumulation across warps, added to HBM once per
+//      (t, n) and block.
 #pragma once
 
 #include "kernel_chunked.cuh"
@@ -39,7 +41,7 @@ namespace ssm {
 struct BwdParams {
   const void *x, *delta, *z, *dy, *B, *C;  // activation dtype
   const float *A_log, *D, *delta_bias, *h0, *dh_last;
-  const float *ckpt;  // [b, ceil(L / 16), E, N]: state before step 16 k
+  const float *ckpt;  // [b, ceil(L / 8), E, N]: state before step 8 k
   void *dx, *ddelta, *dz;  // [b, L, E] activation dtype (dz: with z only)
   float *dB, *dC;          // [b, L, N], summed into (zero before the launch)
   float *dA_log;           // [E, N], summed into
@@ -53,7 +55,9 @@ struct BwdParams {
 template <typename T, int NG, int NW>
 struct BwdCfg {
   static constexpr int N = 4 * NG, CW = 32 / NG, G = CW * NW;
-  static constexpr int THREADS = 32 * NW, TW = kCkptSteps;
+  // windows of two checkpoint intervals; the state history of one interval
+  // (half a window) is kept at a time
+  static constexpr int THREADS = 32 * NW, TW = 2 * kCkptSteps;
   static constexpr int ESZ = sizeof(T);
   // raw tiles of one stage: x, raw step, z, dy [TW][G] and B, C [TW][N]
   static constexpr int ACT_BYTES = TW * G * ESZ;
@@ -68,7 +72,7 @@ struct BwdCfg {
   static constexpr int SP = G + (NG > 1 ? 32 / NG : 0);
   static constexpr int SCAL_BYTES = 5 * TW * SP * 4;
   static constexpr int BCF_BYTES = 2 * TW * N * 4;
-  static constexpr int HALF = TW / 2;  // rows of state history kept at once
+  static constexpr int HALF = kCkptSteps;  // rows of state history kept
   static constexpr int HIST_BYTES = HALF * THREADS * 16;
   static constexpr int ACC_BYTES = TW * 2 * N * 4;
   static constexpr int SMEM_BYTES =
@@ -98,7 +102,8 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
   const int64_t e0 = (blockIdx.x - b * tiles) * G;
   const int64_t e = e0 + cl;
   const bool ch_ok = e < E;
-  const int64_t nck = (L + TW - 1) / TW;
+  const int64_t nwin = (L + TW - 1) / TW;
+  const int64_t nck = (L + kCkptSteps - 1) / kCkptSteps;  // checkpoints
 
   float *const sS = reinterpret_cast<float *>(smem + 2 * Cfg::STAGE);
   float *const sX = sS + TW * SP;
@@ -171,7 +176,7 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
     }
   };
 
-  const int64_t w_last = nck - 1;
+  const int64_t w_last = nwin - 1;
   stage(w_last, 0);
   cp_async_commit();
   for (int64_t w = w_last; w >= 0; --w) {
@@ -224,14 +229,21 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
     }
     __syncthreads();
 
-    // ---- 3. recompute this lane's states from the checkpoint, half a
-    // window at a time (the later half first): the state history of the
-    // half being reversed is kept in shared memory
-    float hck[4] = {}, hmid[4];
+    // ---- 3. recompute this lane's states from the checkpoints, half a
+    // window (one checkpoint interval) at a time, the later half first: the
+    // state history of the half being reversed is kept in shared memory.
+    // Both halves start from a stored state, so each step is recomputed once.
+    float hck[4] = {}, hmid[4] = {};
     if (ch_ok) {
       const float4 v = *reinterpret_cast<const float4 *>(
-          p.ckpt + ((b * nck + w) * E + e) * N + 4 * g);
+          p.ckpt + ((b * nck + 2 * w) * E + e) * N + 4 * g);
       hck[0] = v.x; hck[1] = v.y; hck[2] = v.z; hck[3] = v.w;
+      // the later half may lie wholly past the sequence (no checkpoint, and
+      // its steps change nothing): start it from the first one then
+      const int64_t k2 = 2 * w + 1 < nck ? 2 * w + 1 : 2 * w;
+      const float4 u = *reinterpret_cast<const float4 *>(
+          p.ckpt + ((b * nck + k2) * E + e) * N + 4 * g);
+      hmid[0] = u.x; hmid[1] = u.y; hmid[2] = u.z; hmid[3] = u.w;
     }
     // advance h over rows [r0, r0 + HALF); STORE: keep each state in sH
     auto recompute = [&](float (&h)[4], int r0, bool store) {
@@ -263,9 +275,6 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
           sH[(r - r0) * THREADS + tid] = make_float4(h[0], h[1], h[2], h[3]);
       }
     };
-#pragma unroll
-    for (int i = 0; i < 4; ++i) hmid[i] = hck[i];
-    recompute(hmid, 0, false);  // the state before the later half
 #pragma unroll 1
     for (int half = 1; half >= 0; --half) {
       const int rb = half * HALF;

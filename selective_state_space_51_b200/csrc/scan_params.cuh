@@ -49,7 +49,7 @@ struct ScanParams {
 };
 
 // Steps between the forward checkpoints the backward pass restarts from.
-constexpr int kCkptSteps = 16;
+constexpr int kCkptSteps = 8;
 
 // Widest causal convolution the fused scan takes.
 constexpr int kScanConvMaxWidth = 4;
