@@ -20,7 +20,7 @@ T_roof = max(bytes / HBM peak, exps / SFU peak), fraction = T_roof / T.
 `--impl reference` times the float64 CPU oracle instead (rank 0 only).
 
 `--op bwd` times the backward pass (ssm_scan_bwd: a forward that writes a
-state checkpoint every 16 steps, then the reverse sweep) on the same
+state checkpoint every 8 steps, then the reverse sweep) on the same
 workload. Two more operations print a line of the same form: `--op conv` times the scan
 with the causal depthwise convolution (width 4) + SiLU fused in front
 (ssm_scan_fwd_conv, same workload and roofline), and `--op step` times one
