@@ -1,4 +1,4 @@
-"""Python binding of libssmscan.so, the B200 selective-scan forward library.
+"""Python binding of libssmscan.so, the B200 selective-scan library.
 
 Argument marshalling only: every step of the scan runs in the CUDA kernels of
 the shared library; PyTorch supplies device memory and streams. The functions
@@ -8,7 +8,15 @@ importing works but the first call raises: there is no fallback path.
 
     from selective_state_space_51_b200 import SelectiveScan
     scan = SelectiveScan(device=0)
+    # forward (optionally write_zoh=True, or conv_weight=/conv_bias= to fuse
+    # the causal depthwise convolution + SiLU that forms x)
     y, h_last = scan(x, delta, A_log, B, C, D=D, z=z, delta_bias=bias)
+    # one decode token for a batch, updating state and conv buffer in place
+    y_t = scan.step(x_t, delta_t, A_log, B_t, C_t, state, conv_state=buf,
+                    conv_weight=w, conv_bias=cb, D=D, z=z_t, delta_bias=bias)
+    # gradients of sum(dy * y) + sum(dh_last * h_last)
+    grads = scan.backward(x, delta, A_log, B, C, dy, D=D, z=z,
+                          delta_bias=bias)
 """
 from __future__ import annotations
 
