@@ -123,7 +123,9 @@ __global__ void __launch_bounds__(128, VEC ? 8 : 1)
     if (live && vec) {
 #pragma unroll
       for (int i = 0; i < SPT; i += 4) {
-        const float4 v4 = *reinterpret_cast<const float4 *>(st + n0 + i);
+        // the state is read once and written once per step: streaming
+        // (evict-first) accesses
+        const float4 v4 = __ldcs(reinterpret_cast<const float4 *>(st + n0 + i));
         h[i] = v4.x; h[i + 1] = v4.y; h[i + 2] = v4.z; h[i + 3] = v4.w;
       }
     } else {
@@ -204,8 +206,8 @@ __global__ void __launch_bounds__(128, VEC ? 8 : 1)
       if (vec) {
 #pragma unroll
         for (int i = 0; i < SPT; i += 4)
-          *reinterpret_cast<float4 *>(st + n0 + i) =
-              make_float4(h[i], h[i + 1], h[i + 2], h[i + 3]);
+          __stcs(reinterpret_cast<float4 *>(st + n0 + i),
+                 make_float4(h[i], h[i + 1], h[i + 2], h[i + 3]));
       } else {
 #pragma unroll
         for (int i = 0; i < SPT; ++i)
