@@ -1,6 +1,8 @@
 /*
- * ssm_scan.h: C ABI of the B200 (sm_100a) selective-scan forward library
- * (libssmscan.so).
+ * ssm_scan.h: C ABI of the B200 (sm_100a) selective-scan library
+ * (libssmscan.so): the fused forward pass, the same with the causal
+ * convolution fused in front, the batched decode step, the backward pass, and
+ * a no-allocation forward for callers that cannot allocate.
  *
  * The operation is the selective state-space recurrence (Mamba-1 / S6) as
  * the page "Mamba: Linear-Time Sequence Modeling with Selective State Spaces"
@@ -44,8 +46,12 @@
  *     before anything is launched. A failed launch returns SSM_ERR_CUDA.
  *   - Thread safety: a handle may be used by one host thread at a time, and
  *     carries at most one in-flight call on any stream at a time when it
- *     needs workspace (long sequences with few channels). Different
- *     handles are independent.
+ *     needs workspace (long sequences with few channels, and the backward
+ *     pass's checkpoints). Different handles are independent.
+ *   - CUDA graphs: ssm_scan_step, and ssm_scan_fwd / ssm_scan_fwd_conv when
+ *     they do not split sequences, only enqueue kernels, so their calls can
+ *     be captured into a graph and replayed. Calls that grow a workspace do
+ *     so on their first use: make that call before capturing.
  */
 #ifndef SSM_SCAN_H
 #define SSM_SCAN_H
