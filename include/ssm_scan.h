@@ -206,7 +206,7 @@ SSM_API int ssm_scan_fwd_conv(ssm_scan_t h, const void *v,
  *   dh0        : [batch, dim, dstate] float32 or NULL (not written).
  * The summed outputs are cleared by the call. dstate must be 4, 8 or 16
  * (8 or 16 for bfloat16), dim * element size a multiple of 16 bytes, and x,
- * delta, z, dy, B, C, A_log, h0, dh_last, dh0 16-byte aligned
+ * delta, z, dy, B, C, A_log, h0, dh_last, dB, dC, dh0 16-byte aligned
  * (SSM_ERR_UNSUPPORTED / SSM_ERR_ALIGN otherwise). Outputs must not overlap
  * inputs. Other errors as for ssm_scan_fwd.
  */

@@ -28,10 +28,12 @@
 //   4. the reverse sweep over the half updates lam in registers. The
 //      per-channel sums (C.h, the dx and d-step partials) are buffered over
 //      NG steps and summed over the channel's lanes by one transposing
-//      butterfly; the sums of dB and dC over the tile's channels are a
-//      transposing butterfly over the warp's channel lanes followed by
-//      shared-memory accumulation across warps, added to HBM once per
-//      (t, n) and block.
+//      butterfly.
+// dB and dC are sums over channels. They stay off the sweep: before it, each
+// warp sums dy h over its own channels straight from the state history; the
+// sweep then overwrites each history slot, once no later step needs it, with
+// the lane's lam f x, and a second warp pass sums those. Each pass ends in
+// one 16-byte atomic add per lane into HBM.
 #pragma once
 
 #include "kernel_chunked.cuh"
@@ -64,8 +66,7 @@ struct BwdCfg {
   static constexpr int BC_BYTES = TW * N * ESZ;
   static constexpr int STAGE = 4 * ACT_BYTES + 2 * BC_BYTES;
   // per-window float arrays: s, x, dy, gate slope, softplus slope [TW][G];
-  // B, C [TW][N]; the states of half a window [TW/2][THREADS] float4; dB,
-  // dC sums [TW][2N]
+  // B, C [TW][N]; the states of half a window [TW/2][RS] float4
   // row stride of the per-(t, e) arrays: the G channels plus 32 / NG words,
   // so that the NG lanes of a channel, which finish NG consecutive steps,
   // read distinct banks
@@ -73,10 +74,17 @@ struct BwdCfg {
   static constexpr int SCAL_BYTES = 5 * TW * SP * 4;
   static constexpr int BCF_BYTES = 2 * TW * N * 4;
   static constexpr int HALF = kCkptSteps;  // rows of state history kept
-  static constexpr int HIST_BYTES = HALF * THREADS * 16;
-  static constexpr int ACC_BYTES = TW * 2 * N * 4;
+  // history row stride in float4: 4 past THREADS, so that the two rows a
+  // quarter-warp reads in the channel-sum passes fall on distinct banks
+  static constexpr int RS = THREADS + 4;
+  static constexpr int HIST_BYTES = HALF * RS * 16;
   static constexpr int SMEM_BYTES =
-      2 * STAGE + SCAL_BYTES + BCF_BYTES + HIST_BYTES + ACC_BYTES;
+      2 * STAGE + SCAL_BYTES + BCF_BYTES + HIST_BYTES;
+  // lanes per (history row, quad of states) in the channel-sum passes: a
+  // lane sums 8 channels of its warp
+  static constexpr int K = 4 / NG;
+  static_assert(HALF == 8 && CW == 8 * K,
+                "channel-sum passes: 8 rows x 4 lanes per warp");
   static_assert(THREADS % G == 0, "a pre-pass thread keeps one channel");
   static_assert((G * ESZ) % 16 == 0 && (N * ESZ) % 16 == 0,
                 "tile rows are whole 16-byte chunks");
@@ -87,7 +95,7 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
   using Cfg = BwdCfg<T, NG, NW>;
   constexpr int N = Cfg::N, CW = Cfg::CW, G = Cfg::G, TW = Cfg::TW;
   constexpr int THREADS = Cfg::THREADS, ESZ = Cfg::ESZ, HALF = Cfg::HALF;
-  constexpr int SP = Cfg::SP;
+  constexpr int SP = Cfg::SP, RS = Cfg::RS, K = Cfg::K;
   constexpr unsigned FULL = 0xffffffffu;
   extern __shared__ __align__(16) unsigned char smem[];
 
@@ -113,7 +121,6 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
   float *const sBF = sSG + TW * SP;
   float *const sCF = sBF + TW * N;
   float4 *const sH = reinterpret_cast<float4 *>(sCF + TW * N);
-  float *const sAcc = reinterpret_cast<float *>(sH + Cfg::HALF * THREADS);
 
   const T *gx = static_cast<const T *>(p.x);
   const T *gdl = static_cast<const T *>(p.delta);
@@ -148,7 +155,19 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
   const float Dv = (ch_ok && p.D) ? p.D[e] : 0.0f;
   float sum_dD = 0.0f, sum_db = 0.0f;
 
-  for (int i = tid; i < TW * 2 * N; i += THREADS) sAcc[i] = 0.0f;
+  // channel-sum passes: this lane sums history row pr, state quad pq, over
+  // the warp's channels j K + pk (j = 0..7), whose slots in the row are the
+  // consecutive warp * 32 + 4 j + (lane & 3)
+  const int pr = lane >> 2, pq = (lane & 3) % NG, pk = (lane & 3) / NG;
+  const float4 *const hrow = sH + pr * RS + warp * 32 + (lane & 3);
+  const bool warp_ok = e0 + warp * CW < E;
+  // add a lane's sum for history row pr of the half at rb into dst [b, L, N]
+  auto red_row = [&](float *dst, int64_t t0, int rb, float2 v01, float2 v23) {
+    const int64_t t = t0 + rb + pr;
+    if (warp_ok && t < L)
+      atomicAdd(reinterpret_cast<float4 *>(dst + (b * L + t) * N + 4 * pq),
+                make_float4(v01.x, v01.y, v23.x, v23.y));
+  };
 
   auto stage = [&](int64_t w, int s) {
     unsigned char *base = smem + s * Cfg::STAGE;
@@ -272,7 +291,7 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
           h[0] = h01.x; h[1] = h01.y; h[2] = h23.x; h[3] = h23.y;
         }
         if (store)
-          sH[(r - r0) * THREADS + tid] = make_float4(h[0], h[1], h[2], h[3]);
+          sH[(r - r0) * RS + tid] = make_float4(h[0], h[1], h[2], h[3]);
       }
     };
 #pragma unroll 1
@@ -285,6 +304,31 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
         float h[4] = {hst[0], hst[1], hst[2], hst[3]};
         recompute(h, rb, true);
       }
+      __syncwarp();
+      // dC[t, n] = sum_e dy h_t[e, n], over this warp's channels
+      {
+        const float *dyr = sDY + (rb + pr) * SP + warp * CW + pk;
+        float dyv[8];
+        if constexpr (K == 1) {
+          const float4 d0 = *reinterpret_cast<const float4 *>(dyr);
+          const float4 d1 = *reinterpret_cast<const float4 *>(dyr + 4);
+          dyv[0] = d0.x; dyv[1] = d0.y; dyv[2] = d0.z; dyv[3] = d0.w;
+          dyv[4] = d1.x; dyv[5] = d1.y; dyv[6] = d1.z; dyv[7] = d1.w;
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) dyv[j] = dyr[j * K];
+        }
+        float2 c01 = make_float2(0.0f, 0.0f), c23 = c01;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float4 hv = hrow[4 * j];
+          const float2 d2 = make_float2(dyv[j], dyv[j]);
+          c01 = fma2(d2, make_float2(hv.x, hv.y), c01);
+          c23 = fma2(d2, make_float2(hv.z, hv.w), c23);
+        }
+        red_row(p.dC, t0, rb, c01, c23);
+      }
+      __syncwarp();
 
       // ---- 4. the reverse sweep over the half, in blocks of NG steps: the
       // per-channel sums (C.h, the dx and d-step partials) are off the
@@ -297,9 +341,9 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
 #pragma unroll
         for (int s = NG - 1; s >= 0; --s) {
           const int r = rb + jb * NG + s;
-          const float4 hc = sH[(r - rb) * THREADS + tid];
+          const float4 hc = sH[(r - rb) * RS + tid];
           const float4 hp4 =
-              r > rb ? sH[(r - rb - 1) * THREADS + tid]
+              r > rb ? sH[(r - rb - 1) * RS + tid]
                      : make_float4(hst[0], hst[1], hst[2], hst[3]);
           const float hcur[4] = {hc.x, hc.y, hc.z, hc.w};
           const float hprev[4] = {hp4.x, hp4.y, hp4.z, hp4.w};
@@ -312,7 +356,7 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
           const float Cv[4] = {Cq.x, Cq.y, Cq.z, Cq.w};
           float &pre = pre_s[s], &dxp = dxp_s[s], &dsp = dsp_s[s];
           pre = dxp = dsp = 0.0f;
-          float v8[8];
+          float4 dBq;  // this step's lam f x, summed into dB after the sweep
           if constexpr (!ZOH) {
             // packed pairs of states; sum_n lam B gives both the dx and the
             // write part of the step-size partial: dx = s sum lam B,
@@ -326,9 +370,8 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
             const float2 C23 = make_float2(Cv[2], Cv[3]);
             const float2 a01 = ex2x2(mul2(s2, make_float2(A2[0], A2[1])));
             const float2 a23 = ex2x2(mul2(s2, make_float2(A2[2], A2[3])));
-            const float2 pr = fma2(C23, hc23, mul2(C01, hc01));
-            pre = pr.x + pr.y;
-            const float2 dC01 = mul2(dy2, hc01), dC23 = mul2(dy2, hc23);
+            const float2 ch = fma2(C23, hc23, mul2(C01, hc01));
+            pre = ch.x + ch.y;
             float2 l01 = fma2(dy2, C01, make_float2(lam[0], lam[1]));
             float2 l23 = fma2(dy2, C23, make_float2(lam[2], lam[3]));
             const float2 lb = fma2(l23, B23, mul2(l01, B01));
@@ -349,59 +392,30 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
             l01 = mul2(l01, a01);
             l23 = mul2(l23, a23);
             lam[0] = l01.x; lam[1] = l01.y; lam[2] = l23.x; lam[3] = l23.y;
-            v8[0] = dB01.x; v8[1] = dB01.y; v8[2] = dB23.x; v8[3] = dB23.y;
-            v8[4] = dC01.x; v8[5] = dC01.y; v8[6] = dC23.x; v8[7] = dC23.y;
+            dBq = make_float4(dB01.x, dB01.y, dB23.x, dB23.y);
           } else {  // zero-order-hold write f = expm1(s A) / A, per state
+            float dBv[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const float zl = sv * A2[i];
               const float a = ex2(zl);
               pre = fmaf(Cv[i], hcur[i], pre);
-              v8[4 + i] = dyv * hcur[i];       // dC
               lam[i] = fmaf(dyv, Cv[i], lam[i]);
               const float da = lam[i] * hprev[i];
               const float f = zoh_factor(sv, zl, a, iA[i]);
               const float lbx = lam[i] * Bv[i] * xv;
               dsp = fmaf(lbx, a, dsp);
-              v8[i] = lam[i] * f * xv;         // dB
+              dBv[i] = lam[i] * f * xv;
               dxp = fmaf(lam[i] * f, Bv[i], dxp);
               dA[i] = fmaf(lbx, (sv * a - f) * iA[i], dA[i]);
               dsp = fmaf(da * a, Av[i], dsp);
               dA[i] = fmaf(da * a, sv, dA[i]);
               lam[i] *= a;
             }
+            dBq = make_float4(dBv[0], dBv[1], dBv[2], dBv[3]);
           }
-          // dB, dC summed over the warp's channels: a transposing butterfly over
-          // lane bits 4, 3, 2 leaves value j = (lane >> 2) & 7 in v8[0]; channel
-          // bits below bit 2 (NG < 4) are summed plainly
-          {
-            bool hi = lane & 16;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float send = hi ? v8[i] : v8[i + 4];
-              const float keep = hi ? v8[i + 4] : v8[i];
-              v8[i] = keep + __shfl_xor_sync(FULL, send, 16);
-            }
-            hi = lane & 8;
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-              const float send = hi ? v8[i] : v8[i + 2];
-              const float keep = hi ? v8[i + 2] : v8[i];
-              v8[i] = keep + __shfl_xor_sync(FULL, send, 8);
-            }
-            hi = lane & 4;
-            {
-              const float send = hi ? v8[0] : v8[1];
-              const float keep = hi ? v8[1] : v8[0];
-              v8[0] = keep + __shfl_xor_sync(FULL, send, 4);
-            }
-            if (NG <= 2) v8[0] += __shfl_xor_sync(FULL, v8[0], 2);
-            if (NG == 1) v8[0] += __shfl_xor_sync(FULL, v8[0], 1);
-            if ((lane & 3 & ~(NG - 1)) == 0) {
-              const int j = (lane >> 2) & 7;
-              atomicAdd(sAcc + r * 2 * N + (j >> 2) * N + 4 * g + (j & 3), v8[0]);
-            }
-          }
+          // step r's history slot is not read again: it takes the dB terms
+          sH[(r - rb) * RS + tid] = dBq;
         }
         const float pre = transpose_reduce<NG, 1>(pre_s, g);
         const float dxp = transpose_reduce<NG, 1>(dxp_s, g);
@@ -423,19 +437,20 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
           sum_db += draw;
         }
       }
-    }
-    __syncthreads();
-    // ---- dB, dC of the window into HBM, once per (t, n) and block
-    for (int idx = tid; idx < TW * 2 * N; idx += THREADS) {
-      const int r = idx / (2 * N), k = idx - r * 2 * N;
-      const int64_t t = t0 + r;
-      if (t < L) {
-        float *dst = (k < N ? p.dB : p.dC) + (b * L + t) * N + (k % N);
-        atomicAdd(dst, sAcc[idx]);
+      __syncwarp();
+      // dB[t, n] = sum_e lam f x, over this warp's channels
+      {
+        float2 b01 = make_float2(0.0f, 0.0f), b23 = b01;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float4 v = hrow[4 * j];
+          b01 = add2(b01, make_float2(v.x, v.y));
+          b23 = add2(b23, make_float2(v.z, v.w));
+        }
+        red_row(p.dB, t0, rb, b01, b23);
       }
-      sAcc[idx] = 0.0f;
+      __syncwarp();
     }
-    __syncthreads();
   }
   cp_async_wait<0>();
   // every lane of a channel finished some of its steps: sum the partials

@@ -620,10 +620,10 @@ int ssm_scan_bwd(ssm_scan_t h, const void *x, const void *delta,
   const void *acts_out[] = {dx, ddelta, dz};
   for (const void *q : acts_out)
     if (q && !aligned(q, esz)) return SSM_ERR_ALIGN;
-  const float *f4[] = {h0, dh_last, dh0, A_log};
+  const float *f4[] = {h0, dh_last, dh0, A_log, dB, dC};
   for (const float *q : f4)
     if (q && !aligned(q, 16)) return SSM_ERR_ALIGN;
-  const float *f1[] = {D, delta_bias, dA_log, dB, dC, dD, ddelta_bias};
+  const float *f1[] = {D, delta_bias, dA_log, dD, ddelta_bias};
   for (const float *q : f1)
     if (q && !aligned(q, 4)) return SSM_ERR_ALIGN;
   int cur = -1;
