@@ -66,7 +66,7 @@ struct BwdCfg {
   static constexpr int BC_BYTES = TW * N * ESZ;
   static constexpr int STAGE = 4 * ACT_BYTES + 2 * BC_BYTES;
   // per-window float arrays: s, x, dy, gate slope, softplus slope [TW][G];
-  // B, C [TW][N]; the states of half a window [TW/2][RS] float4
+  // B, C [TW][N]; the states of half a window [TW/2 + 1][RS] float4
   // row stride of the per-(t, e) arrays: the G channels plus 32 / NG words,
   // so that the NG lanes of a channel, which finish NG consecutive steps,
   // read distinct banks
@@ -75,9 +75,11 @@ struct BwdCfg {
   static constexpr int BCF_BYTES = 2 * TW * N * 4;
   static constexpr int HALF = kCkptSteps;  // rows of state history kept
   // history row stride in float4: 4 past THREADS, so that the two rows a
-  // quarter-warp reads in the channel-sum passes fall on distinct banks
+  // quarter-warp reads in the channel-sum passes fall on distinct banks.
+  // Row 0 is the state before the half, row 1 + i the state after its
+  // step i.
   static constexpr int RS = THREADS + 4;
-  static constexpr int HIST_BYTES = HALF * RS * 16;
+  static constexpr int HIST_BYTES = (HALF + 1) * RS * 16;
   static constexpr int SMEM_BYTES =
       2 * STAGE + SCAL_BYTES + BCF_BYTES + HIST_BYTES;
   // lanes per (history row, quad of states) in the channel-sum passes: a
@@ -159,7 +161,7 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
   // the warp's channels j K + pk (j = 0..7), whose slots in the row are the
   // consecutive warp * 32 + 4 j + (lane & 3)
   const int pr = lane >> 2, pq = (lane & 3) % NG, pk = (lane & 3) / NG;
-  const float4 *const hrow = sH + pr * RS + warp * 32 + (lane & 3);
+  const float4 *const hrow = sH + (1 + pr) * RS + warp * 32 + (lane & 3);
   const bool warp_ok = e0 + warp * CW < E;
   // add a lane's sum for history row pr of the half at rb into dst [b, L, N]
   auto red_row = [&](float *dst, int64_t t0, int rb, float2 v01, float2 v23) {
@@ -265,6 +267,7 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
       hmid[0] = u.x; hmid[1] = u.y; hmid[2] = u.z; hmid[3] = u.w;
     }
     // advance h over rows [r0, r0 + HALF); STORE: keep each state in sH
+    // (row 1 + r - r0)
     auto recompute = [&](float (&h)[4], int r0, bool store) {
 #pragma unroll 4
       for (int r = r0; r < r0 + HALF; ++r) {
@@ -291,7 +294,7 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
           h[0] = h01.x; h[1] = h01.y; h[2] = h23.x; h[3] = h23.y;
         }
         if (store)
-          sH[(r - r0) * RS + tid] = make_float4(h[0], h[1], h[2], h[3]);
+          sH[(1 + r - r0) * RS + tid] = make_float4(h[0], h[1], h[2], h[3]);
       }
     };
 #pragma unroll 1
@@ -300,6 +303,7 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
       float hst[4];  // the state before row rb
 #pragma unroll
       for (int i = 0; i < 4; ++i) hst[i] = half ? hmid[i] : hck[i];
+      sH[tid] = make_float4(hst[0], hst[1], hst[2], hst[3]);
       {
         float h[4] = {hst[0], hst[1], hst[2], hst[3]};
         recompute(h, rb, true);
@@ -335,16 +339,15 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
       // adjoint's critical path, so they are kept per step and summed over
       // the channel's lanes once per block by a transposing butterfly that
       // leaves lane g the totals of the block's step g, which it finishes
+      // the state after step r: carried from the previous (later) step
+      float4 hc = sH[HALF * RS + tid];
 #pragma unroll 1
       for (int jb = HALF / NG - 1; jb >= 0; --jb) {
         float pre_s[NG], dxp_s[NG], dsp_s[NG];
 #pragma unroll
         for (int s = NG - 1; s >= 0; --s) {
           const int r = rb + jb * NG + s;
-          const float4 hc = sH[(r - rb) * RS + tid];
-          const float4 hp4 =
-              r > rb ? sH[(r - rb - 1) * RS + tid]
-                     : make_float4(hst[0], hst[1], hst[2], hst[3]);
+          const float4 hp4 = sH[(r - rb) * RS + tid];
           const float hcur[4] = {hc.x, hc.y, hc.z, hc.w};
           const float hprev[4] = {hp4.x, hp4.y, hp4.z, hp4.w};
           const float sv = sS[r * SP + cl];
@@ -415,7 +418,8 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
             dBq = make_float4(dBv[0], dBv[1], dBv[2], dBv[3]);
           }
           // step r's history slot is not read again: it takes the dB terms
-          sH[(r - rb) * RS + tid] = dBq;
+          sH[(1 + r - rb) * RS + tid] = dBq;
+          hc = hp4;
         }
         const float pre = transpose_reduce<NG, 1>(pre_s, g);
         const float dxp = transpose_reduce<NG, 1>(dxp_s, g);
