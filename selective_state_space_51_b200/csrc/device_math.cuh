@@ -165,14 +165,31 @@ __device__ __forceinline__ float2 silu2_fast(float2 z) {
   return fma2(h, make_float2(tanh_approx(h.x), tanh_approx(h.y)), h);
 }
 
+// sigmoid(v) = 1 / (1 + e^-v) of two values; 0 for v -> -inf, 1 for +inf.
+__device__ __forceinline__ float2 sigmoid2(float2 v) {
+  const float2 e = mul2(v, make_float2(-kLog2e, -kLog2e));
+  const float2 d = add2(make_float2(ex2(e.x), ex2(e.y)), make_float2(1.0f, 1.0f));
+  return make_float2(rcp(d.x), rcp(d.y));
+}
+
 // The step-size softplus and the SiLU the chunked kernel applies to packed
 // pairs: exact-rounding-order forms for float32 activations, the cheaper
-// forms above for bfloat16.
+// forms above for bfloat16. The backward pass takes their derivatives from
+// the same forms: softplus_slope gives softplus(v) and sigmoid(v) (its
+// slope); sigmoid(z) is the gate's, SiLU(z) = z sigmoid(z).
 template <typename T> struct PairMath {
   static __device__ __forceinline__ float2 softplus(float2 v) {
     return softplus2(v);
   }
   static __device__ __forceinline__ float2 silu(float2 z) { return silu2(z); }
+  static __device__ __forceinline__ void softplus_slope(float2 v, float2 &sp,
+                                                        float2 &slope) {
+    sp = softplus2(v);
+    slope = sigmoid2(v);
+  }
+  static __device__ __forceinline__ float2 sigmoid(float2 z) {
+    return sigmoid2(z);
+  }
 };
 template <> struct PairMath<__nv_bfloat16> {
   static __device__ __forceinline__ float2 softplus(float2 v) {
@@ -180,6 +197,26 @@ template <> struct PairMath<__nv_bfloat16> {
   }
   static __device__ __forceinline__ float2 silu(float2 z) {
     return silu2_fast(z);
+  }
+  // softplus2_fast's value, and its slope e^v / (1 + e^v) from the same e^v
+  // (a product, so it keeps relative accuracy where e^v is tiny); above the
+  // threshold the value is v and the slope 1.
+  static __device__ __forceinline__ void softplus_slope(float2 v, float2 &sp,
+                                                        float2 &slope) {
+    const float2 e2 = mul2(v, make_float2(kLog2e, kLog2e));
+    const float2 e = make_float2(ex2(e2.x), ex2(e2.y));
+    const float2 w = add2(e, make_float2(1.0f, 1.0f));
+    const float2 r =
+        mul2(make_float2(lg2(w.x), lg2(w.y)), make_float2(kLn2, kLn2));
+    const float2 sl = mul2(e, make_float2(rcp(w.x), rcp(w.y)));
+    sp = make_float2(v.x > 20.0f ? v.x : r.x, v.y > 20.0f ? v.y : r.y);
+    slope = make_float2(v.x > 20.0f ? 1.0f : sl.x, v.y > 20.0f ? 1.0f : sl.y);
+  }
+  // (1 + tanh(z/2)) / 2, the sigmoid inside silu2_fast
+  static __device__ __forceinline__ float2 sigmoid(float2 z) {
+    const float2 h = mul2(z, make_float2(0.5f, 0.5f));
+    return fma2(make_float2(tanh_approx(h.x), tanh_approx(h.y)),
+                make_float2(0.5f, 0.5f), make_float2(0.5f, 0.5f));
   }
 };
 
@@ -219,12 +256,20 @@ template <typename T> struct Act;
 
 template <> struct Act<float> {
   static __device__ __forceinline__ float load(const float *p) { return *p; }
+  // two adjacent elements (8-byte aligned)
+  static __device__ __forceinline__ float2 load2(const float *p) {
+    return *reinterpret_cast<const float2 *>(p);
+  }
   static __device__ __forceinline__ void store(float *p, float v) { *p = v; }
 };
 
 template <> struct Act<__nv_bfloat16> {
   static __device__ __forceinline__ float load(const __nv_bfloat16 *p) {
     return __bfloat162float(*p);
+  }
+  // two adjacent elements (4-byte aligned)
+  static __device__ __forceinline__ float2 load2(const __nv_bfloat16 *p) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
   }
   static __device__ __forceinline__ void store(__nv_bfloat16 *p, float v) {
     *p = __float2bfloat16_rn(v);

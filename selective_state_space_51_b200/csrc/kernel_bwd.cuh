@@ -149,11 +149,14 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
       lam[0] = v.x; lam[1] = v.y; lam[2] = v.z; lam[3] = v.w;
     }
   }
-  // the pre-pass channel of this thread (THREADS is a multiple of G)
-  const int pc = tid % G;
+  // the pre-pass channel pair of this thread (THREADS is a multiple of G;
+  // E is even, so a pair is wholly inside or wholly past the last channel)
+  const int pc = 2 * (tid % (G / 2));
   const int64_t pe = e0 + pc;
   const bool pe_ok = pe < E;
-  const float pbias = (pe_ok && p.delta_bias) ? p.delta_bias[pe] : 0.0f;
+  const float2 pbias = (pe_ok && p.delta_bias)
+                           ? make_float2(p.delta_bias[pe], p.delta_bias[pe + 1])
+                           : make_float2(0.0f, 0.0f);
   const float Dv = (ch_ok && p.D) ? p.D[e] : 0.0f;
   float sum_dD = 0.0f, sum_db = 0.0f;
 
@@ -209,36 +212,40 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
 
     const int64_t t0 = w * TW;
     const unsigned char *base = smem + par * Cfg::STAGE;
-    // ---- 2. per (t, e) scalars, once
-    for (int idx = tid; idx < TW * G; idx += THREADS) {
-      const int r = idx / G;  // idx % G == pc
-      const bool ok = pe_ok && t0 + r < L;
+    // ---- 2. per (t, e) scalars, once, for two adjacent channels at a time.
+    // The staged tiles are zero past the sequence and past the last channel,
+    // which makes x, dy and the gate slope zero there; the step size is set
+    // to zero past the sequence, so that those steps leave lam unchanged.
+    for (int idx = tid; idx < TW * (G / 2); idx += THREADS) {
+      const int r = idx / (G / 2);  // 2 (idx % (G / 2)) == pc
       const int o = (r * G + pc) * ESZ;
-      const float raw =
-          Act<T>::load(reinterpret_cast<const T *>(base + Cfg::ACT_BYTES + o)) +
-          pbias;
-      const float xv = Act<T>::load(reinterpret_cast<const T *>(base + o));
-      const float gv = Act<T>::load(
+      const float2 raw = add2(
+          Act<T>::load2(reinterpret_cast<const T *>(base + Cfg::ACT_BYTES + o)),
+          pbias);
+      const float2 xv = Act<T>::load2(reinterpret_cast<const T *>(base + o));
+      const float2 gv = Act<T>::load2(
           reinterpret_cast<const T *>(base + 3 * Cfg::ACT_BYTES + o));
-      float dyv = gv, gzv = 0.0f;
+      float2 dyv = gv, gzv = make_float2(0.0f, 0.0f);
       if (has_z) {
-        const float zv = Act<T>::load(
+        // y = pre SiLU(z): dy = g SiLU(z), dz = g pre sg (1 + z (1 - sg))
+        const float2 zv = Act<T>::load2(
             reinterpret_cast<const T *>(base + 2 * Cfg::ACT_BYTES + o));
-        const float sg = rcp(1.0f + ex2(-zv * kLog2e));
-        dyv = gv * zv * sg;
-        gzv = gv * sg * fmaf(zv, 1.0f - sg, 1.0f);
+        const float2 sg = PairMath<T>::sigmoid(zv);
+        const float2 gs = mul2(gv, sg);
+        dyv = mul2(gs, zv);
+        gzv = mul2(gs, fma2(zv, add2(make_float2(1.0f, 1.0f),
+                                     make_float2(-sg.x, -sg.y)),
+                            make_float2(1.0f, 1.0f)));
       }
-      float sv = raw, slope = 1.0f;
-      if (p.softplus) {
-        sv = softplus(raw);
-        slope = rcp(1.0f + ex2(-raw * kLog2e));
-      }
+      float2 sv = raw, slope = make_float2(1.0f, 1.0f);
+      if (p.softplus) PairMath<T>::softplus_slope(raw, sv, slope);
+      const bool ok = t0 + r < L;
       const int so = r * SP + pc;
-      sS[so] = ok ? sv : 0.0f;
-      sX[so] = ok ? xv : 0.0f;
-      sDY[so] = ok ? dyv : 0.0f;
-      sGZ[so] = ok ? gzv : 0.0f;
-      sSG[so] = slope;
+      *reinterpret_cast<float2 *>(sS + so) = ok ? sv : make_float2(0.0f, 0.0f);
+      *reinterpret_cast<float2 *>(sX + so) = xv;
+      *reinterpret_cast<float2 *>(sDY + so) = dyv;
+      *reinterpret_cast<float2 *>(sGZ + so) = gzv;
+      *reinterpret_cast<float2 *>(sSG + so) = slope;
     }
     {
       const unsigned char *bc = base + 4 * Cfg::ACT_BYTES;
