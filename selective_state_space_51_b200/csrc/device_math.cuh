@@ -260,6 +260,10 @@ template <> struct Act<float> {
   static __device__ __forceinline__ float2 load2(const float *p) {
     return *reinterpret_cast<const float2 *>(p);
   }
+  // four adjacent elements (16-byte aligned)
+  static __device__ __forceinline__ float4 load4(const float *p) {
+    return *reinterpret_cast<const float4 *>(p);
+  }
   static __device__ __forceinline__ void store(float *p, float v) { *p = v; }
 };
 
@@ -270,6 +274,15 @@ template <> struct Act<__nv_bfloat16> {
   // two adjacent elements (4-byte aligned)
   static __device__ __forceinline__ float2 load2(const __nv_bfloat16 *p) {
     return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
+  }
+  // four adjacent elements (8-byte aligned) in one 8-byte load; a bfloat16
+  // is the upper half of the float32 with the same value
+  static __device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(p);
+    return make_float4(__uint_as_float(u.x << 16),
+                       __uint_as_float(u.x & 0xffff0000u),
+                       __uint_as_float(u.y << 16),
+                       __uint_as_float(u.y & 0xffff0000u));
   }
   static __device__ __forceinline__ void store(__nv_bfloat16 *p, float v) {
     *p = __float2bfloat16_rn(v);

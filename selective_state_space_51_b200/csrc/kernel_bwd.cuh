@@ -19,7 +19,8 @@
 // as the forward kernel (NG lanes per channel, 4 states per lane). It walks
 // windows of 16 steps from the last to the first. For each window:
 //   1. the x, raw step, z, incoming-gradient, B and C tiles arrive by
-//      cp.async (the previous window's are already in flight);
+//      cp.async (issued at the start of the previous window); B and C are
+//      read from these staged tiles, in the activation type, throughout;
 //   2. a pre-pass forms each (t, e)'s step size, x, dy, gate slope and
 //      softplus slope once, in shared memory;
 //   3. for each half window (one 8-step checkpoint interval), the later
@@ -66,13 +67,12 @@ struct BwdCfg {
   static constexpr int BC_BYTES = TW * N * ESZ;
   static constexpr int STAGE = 4 * ACT_BYTES + 2 * BC_BYTES;
   // per-window float arrays: s, x, dy, gate slope, softplus slope [TW][G];
-  // B, C [TW][N]; the states of half a window [TW/2 + 1][RS] float4
+  // the states of half a window [TW/2 + 1][RS] float4
   // row stride of the per-(t, e) arrays: the G channels plus 32 / NG words,
   // so that the NG lanes of a channel, which finish NG consecutive steps,
   // read distinct banks
   static constexpr int SP = G + (NG > 1 ? 32 / NG : 0);
   static constexpr int SCAL_BYTES = 5 * TW * SP * 4;
-  static constexpr int BCF_BYTES = 2 * TW * N * 4;
   static constexpr int HALF = kCkptSteps;  // rows of state history kept
   // history row stride in float4: 4 past THREADS, so that the two rows a
   // quarter-warp reads in the channel-sum passes fall on distinct banks.
@@ -80,8 +80,7 @@ struct BwdCfg {
   // step i.
   static constexpr int RS = THREADS + 4;
   static constexpr int HIST_BYTES = (HALF + 1) * RS * 16;
-  static constexpr int SMEM_BYTES =
-      2 * STAGE + SCAL_BYTES + BCF_BYTES + HIST_BYTES;
+  static constexpr int SMEM_BYTES = 2 * STAGE + SCAL_BYTES + HIST_BYTES;
   // lanes per (history row, quad of states) in the channel-sum passes: a
   // lane sums 8 channels of its warp
   static constexpr int K = 4 / NG;
@@ -120,9 +119,7 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
   float *const sDY = sX + TW * SP;
   float *const sGZ = sDY + TW * SP;
   float *const sSG = sGZ + TW * SP;
-  float *const sBF = sSG + TW * SP;
-  float *const sCF = sBF + TW * N;
-  float4 *const sH = reinterpret_cast<float4 *>(sCF + TW * N);
+  float4 *const sH = reinterpret_cast<float4 *>(sSG + TW * SP);
 
   const T *gx = static_cast<const T *>(p.x);
   const T *gdl = static_cast<const T *>(p.delta);
@@ -205,13 +202,18 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
   cp_async_commit();
   for (int64_t w = w_last; w >= 0; --w) {
     const int par = int((w_last - w) & 1);
+    // this window's tiles have landed, and every thread is done with the
+    // previous window, whose buffer now takes the next window's tiles
+    cp_async_wait<0>();
+    __syncthreads();
     if (w > 0) stage(w - 1, par ^ 1);
     cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
 
     const int64_t t0 = w * TW;
     const unsigned char *base = smem + par * Cfg::STAGE;
+    const T *const sBr = reinterpret_cast<const T *>(base + 4 * Cfg::ACT_BYTES);
+    const T *const sCr = reinterpret_cast<const T *>(
+        base + 4 * Cfg::ACT_BYTES + Cfg::BC_BYTES);
     // ---- 2. per (t, e) scalars, once, for two adjacent channels at a time.
     // The staged tiles are zero past the sequence and past the last channel,
     // which makes x, dy and the gate slope zero there; the step size is set
@@ -247,14 +249,6 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
       *reinterpret_cast<float2 *>(sGZ + so) = gzv;
       *reinterpret_cast<float2 *>(sSG + so) = slope;
     }
-    {
-      const unsigned char *bc = base + 4 * Cfg::ACT_BYTES;
-      for (int idx = tid; idx < TW * N; idx += THREADS) {
-        sBF[idx] = Act<T>::load(reinterpret_cast<const T *>(bc) + idx);
-        sCF[idx] =
-            Act<T>::load(reinterpret_cast<const T *>(bc + Cfg::BC_BYTES) + idx);
-      }
-    }
     __syncthreads();
 
     // ---- 3. recompute this lane's states from the checkpoints, half a
@@ -280,7 +274,7 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
       for (int r = r0; r < r0 + HALF; ++r) {
         const float sv = sS[r * SP + cl];
         const float xv = sX[r * SP + cl];
-        const float4 Bq = *reinterpret_cast<const float4 *>(sBF + r * N + 4 * g);
+        const float4 Bq = Act<T>::load4(sBr + r * N + 4 * g);
         if constexpr (ZOH) {
           const float Bv[4] = {Bq.x, Bq.y, Bq.z, Bq.w};
 #pragma unroll
@@ -311,9 +305,13 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) hst[i] = half ? hmid[i] : hck[i];
       sH[tid] = make_float4(hst[0], hst[1], hst[2], hst[3]);
+      // the state after step r of the sweep below, carried from the previous
+      // (later) step; the recompute leaves the half's last state
+      float4 hc;
       {
         float h[4] = {hst[0], hst[1], hst[2], hst[3]};
         recompute(h, rb, true);
+        hc = make_float4(h[0], h[1], h[2], h[3]);
       }
       __syncwarp();
       // dC[t, n] = sum_e dy h_t[e, n], over this warp's channels
@@ -346,8 +344,6 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
       // adjoint's critical path, so they are kept per step and summed over
       // the channel's lanes once per block by a transposing butterfly that
       // leaves lane g the totals of the block's step g, which it finishes
-      // the state after step r: carried from the previous (later) step
-      float4 hc = sH[HALF * RS + tid];
 #pragma unroll 1
       for (int jb = HALF / NG - 1; jb >= 0; --jb) {
         float pre_s[NG], dxp_s[NG], dsp_s[NG];
@@ -360,8 +356,8 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
           const float sv = sS[r * SP + cl];
           const float xv = sX[r * SP + cl];
           const float dyv = sDY[r * SP + cl];
-          const float4 Bq = *reinterpret_cast<const float4 *>(sBF + r * N + 4 * g);
-          const float4 Cq = *reinterpret_cast<const float4 *>(sCF + r * N + 4 * g);
+          const float4 Bq = Act<T>::load4(sBr + r * N + 4 * g);
+          const float4 Cq = Act<T>::load4(sCr + r * N + 4 * g);
           const float Bv[4] = {Bq.x, Bq.y, Bq.z, Bq.w};
           const float Cv[4] = {Cq.x, Cq.y, Cq.z, Cq.w};
           float &pre = pre_s[s], &dxp = dxp_s[s], &dsp = dsp_s[s];
