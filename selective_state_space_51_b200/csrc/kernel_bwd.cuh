@@ -270,7 +270,7 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
     // advance h over rows [r0, r0 + HALF); STORE: keep each state in sH
     // (row 1 + r - r0)
     auto recompute = [&](float (&h)[4], int r0, bool store) {
-#pragma unroll 4
+#pragma unroll
       for (int r = r0; r < r0 + HALF; ++r) {
         const float sv = sS[r * SP + cl];
         const float xv = sX[r * SP + cl];
@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
       // adjoint's critical path, so they are kept per step and summed over
       // the channel's lanes once per block by a transposing butterfly that
       // leaves lane g the totals of the block's step g, which it finishes
-#pragma unroll 1
+#pragma unroll
       for (int jb = HALF / NG - 1; jb >= 0; --jb) {
         float pre_s[NG], dxp_s[NG], dsp_s[NG];
 #pragma unroll

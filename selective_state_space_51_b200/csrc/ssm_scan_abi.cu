@@ -360,13 +360,18 @@ int scan_fwd(ssm_scan_s *h, const void *x, const float *conv_weight,
 }
 
 // ---- backward
+// Two warps per block: the 2.8B layer shape's 1280 blocks then fill 148 SMs
+// at 9 blocks each in one wave, with at most 9 blocks where 8.65 is the
+// mean (4-warp blocks: 5 where the mean is 4.3).
+constexpr int kBwdWarps = 2;
+
 template <typename T, int NG, bool ZOH>
 int launch_bwd(const ssm::BwdParams &p, cudaStream_t s) {
-  using Cfg = ssm::BwdCfg<T, NG, 4>;
+  using Cfg = ssm::BwdCfg<T, NG, kBwdWarps>;
   const int64_t tiles = (p.dim + Cfg::G - 1) / Cfg::G;
   const int64_t blocks = p.batch * tiles;
   if (blocks > 0x7fffffff) return SSM_ERR_UNSUPPORTED;
-  auto kern = ssm::scan_bwd_kernel<T, NG, 4, ZOH>;
+  auto kern = ssm::scan_bwd_kernel<T, NG, kBwdWarps, ZOH>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Cfg::SMEM_BYTES) != cudaSuccess) {
     cudaGetLastError();
