@@ -219,7 +219,14 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
     // which makes x, dy and the gate slope zero there; the step size is set
     // to zero past the sequence, so that those steps leave lam unchanged.
     for (int idx = tid; idx < TW * (G / 2); idx += THREADS) {
-      const int r = idx / (G / 2);  // 2 (idx % (G / 2)) == pc
+      int r = idx / (G / 2);  // 2 (idx % (G / 2)) == pc
+      if constexpr (G == 16) {
+        // a warp covers 4 rows, 8 lanes each: let each half-warp store rows
+        // r and r + 2, whose 8-byte stores fall 16 banks apart (rows r and
+        // r + 1 would share 8 of their banks at this row stride)
+        const int q = r & 3;
+        r = (r & ~3) | ((q & 1) << 1) | (q >> 1);
+      }
       const int o = (r * G + pc) * ESZ;
       const float2 raw = add2(
           Act<T>::load2(reinterpret_cast<const T *>(base + Cfg::ACT_BYTES + o)),
