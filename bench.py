@@ -601,8 +601,8 @@ def _finish(args, op, world, rank, local, dev, dist, scan, clocks, total_ms,
     if op.name == "bwd":
         line["roofline"]["peak_note"] += (
             "; one retention exp per element counted (the pass evaluates "
-            "about 3.4: the checkpointing forward, the window recompute, the "
-            "reverse sweep, and the pre-pass slopes)")
+            "about 3.3: one each in the checkpointing forward, the recompute "
+            "and the reverse sweep, plus the pre-pass slopes per (t, e))")
     if op.name != "step":
         line["roofline_min_hbm_sfu"] = {
             "t_hbm_us": t_hbm * 1e6, "t_sfu_us_at_max_clock": t_sfu * 1e6,
