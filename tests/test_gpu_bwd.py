@@ -150,11 +150,11 @@ def test_bwd_argument_errors(scan):
 
     def call(**kw):
         a = dict(x=x, z=None, D=None, dz=None, dD=None, dy=x, dims=dims,
-                 dtype=S.SSM_F32)
+                 dtype=S.SSM_F32, dB=dB)
         a.update(kw)
         return S.ssm_scan_bwd(scan.handle, a["x"], x, A, Bm, Bm, a["D"],
                               a["z"], None, 1, None, a["dy"], None, out, out,
-                              dA, dB, dB.clone(), a["dD"], a["dz"], None,
+                              dA, a["dB"], dB.clone(), a["dD"], a["dz"], None,
                               None, a["dims"], a["dtype"], check=False)
     assert call() == S.SSM_OK
     assert call(dy=None) == S.SSM_ERR_INVALID
@@ -163,4 +163,6 @@ def test_bwd_argument_errors(scan):
     assert call(dims=(b, L, E, 5)) == S.SSM_ERR_UNSUPPORTED
     assert call(dims=(b, L, 6, N)) == S.SSM_ERR_UNSUPPORTED  # 24-byte rows
     assert call(dtype=S.SSM_BF16) == S.SSM_ERR_UNSUPPORTED   # N=4 bf16
+    # dB and dC take 16-byte atomic adds: rejected before any launch
+    assert call(dB=dB.data_ptr() + 4) == S.SSM_ERR_ALIGN
     torch.cuda.synchronize()
