@@ -35,7 +35,8 @@ def _worker(rank, world, port, out):
 def test_two_gloo_ranks():
     world = 2
     port = _free_port()
-    with mp.Manager() as m:
+    # spawn, not fork: earlier tests may have started OpenMP threads
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
