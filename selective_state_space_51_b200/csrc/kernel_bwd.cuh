@@ -86,7 +86,7 @@ struct BwdCfg {
   static constexpr int K = 4 / NG;
   static_assert(HALF == 8 && CW == 8 * K,
                 "channel-sum passes: 8 rows x 4 lanes per warp");
-  static_assert(THREADS % G == 0, "a pre-pass thread keeps one channel");
+  static_assert(THREADS % G == 0, "a pre-pass thread keeps one channel pair");
   static_assert((G * ESZ) % 16 == 0 && (N * ESZ) % 16 == 0,
                 "tile rows are whole 16-byte chunks");
 };
