@@ -14,6 +14,8 @@
 // zeros before the first step.
 #pragma once
 
+#include <float.h>
+
 #include "device_math.cuh"
 #include "scan_params.cuh"
 
@@ -38,7 +40,8 @@ scan_sequential_kernel(const ScanParams p) {
     iA[n] = 0.0f;
     h[n] = 0.0f;
     if (n < N) {
-      A2[n] = -expf(p.A_log[e * N + n]) * kLog2e;
+      // clamp so that a zero step never meets -inf (0 * -inf = NaN)
+      A2[n] = fmaxf(-expf(p.A_log[e * N + n]) * kLog2e, -FLT_MAX);
       iA[n] = -expf(-p.A_log[e * N + n]);
       if (p.h0) h[n] = p.h0[(b * E + e) * N + n];
     }

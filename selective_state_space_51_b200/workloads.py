@@ -25,6 +25,10 @@ Every draw comes from numpy's PCG64 seeded with 51000 + shape index (or an
 explicit seed), in float32, in the fixed order x, raw step, z, B, C, D, dt,
 h0. Sizes may be overridden (batch, seqlen, dim, dstate) to make smaller cases
 with the same distributions for parity tests.
+
+``a_jitter`` (tests only) gives every channel its own A: A_log[e, n] =
+log(n + 1) + a_jitter * N(0, 1), drawn after all the draws above so that
+they stay the same. The stated workloads use a_jitter = 0.
 """
 from __future__ import annotations
 
@@ -108,7 +112,7 @@ def make(index: int, seed: Optional[int] = None, batch: Optional[int] = None,
          seqlen: Optional[int] = None, dim: Optional[int] = None,
          dstate: Optional[int] = None, dtype: Optional[str] = None,
          gated: Optional[bool] = None, with_h0: Optional[bool] = None,
-         with_D: bool = True) -> Workload:
+         with_D: bool = True, a_jitter: float = 0.0) -> Workload:
     """Draw workload ``index`` (0-4), optionally with other sizes or options."""
     name, b0, L0, E0, N0, dt0, gated0, long_memory = SHAPES[index]
     b = b0 if batch is None else int(batch)
@@ -145,6 +149,10 @@ def make(index: int, seed: Optional[int] = None, batch: Optional[int] = None,
     A_log = np.log(np.arange(1, N + 1, dtype=np.float64))
     A_log = np.ascontiguousarray(np.broadcast_to(A_log, (E, N)),
                                  dtype=np.float32)
+    if a_jitter:
+        # per-channel A (A is a learned [E, N] parameter): the last draw
+        A_log = (A_log + np.float32(a_jitter) * normal(E, N)).astype(
+            np.float32)
 
     dev = dict(x=x, delta=raw, z=z, B=Bm, C=Cm)
     if act == BF16:

@@ -57,11 +57,13 @@ VARIANTS = [(S.SSM_VARIANT_AUTO, 0, 0), (S.SSM_VARIANT_SEQUENTIAL, 0, 0),
 VARIANT_IDS = ["auto", "sequential", "chunked", "chunked_split3"]
 
 
+@pytest.mark.parametrize("jitter", [0.0, 0.5], ids=["A_stated",
+                                                    "A_per_channel"])
 @pytest.mark.parametrize("variant", VARIANTS, ids=VARIANT_IDS)
 @pytest.mark.parametrize("name", sorted(CASES))
-def test_conv_parity(scan, name, variant):
+def test_conv_parity(scan, name, variant, jitter):
     idx, size = CASES[name]
-    wl = W.make(idx, **size)
+    wl = W.make(idx, a_jitter=jitter, **size)
     w, cb = W.conv_params(wl.dim, 4)
     _set(scan, *variant)
     try:
@@ -78,7 +80,7 @@ def test_conv_parity(scan, name, variant):
 @pytest.mark.parametrize("idx,dtype", [(1, W.F32), (3, W.BF16), (0, W.F32)],
                          ids=["n16_f32", "n16_bf16", "n4_f32"])
 def test_conv_widths(scan, width, idx, dtype, variant):
-    wl = W.make(idx, batch=2, seqlen=400, dim=64, dtype=dtype)
+    wl = W.make(idx, batch=2, seqlen=400, dim=64, dtype=dtype, a_jitter=0.5)
     w, cb = W.conv_params(wl.dim, width, seed=7 + width)
     _set(scan, *variant)
     try:
@@ -92,7 +94,7 @@ def test_conv_widths(scan, width, idx, dtype, variant):
 
 @pytest.mark.parametrize("variant", VARIANTS, ids=VARIANT_IDS)
 def test_conv_with_zoh_and_no_bias(scan, variant):
-    wl = W.make(3, batch=2, seqlen=1100, dim=40, with_h0=True)
+    wl = W.make(3, batch=2, seqlen=1100, dim=40, with_h0=True, a_jitter=0.5)
     w, _ = W.conv_params(wl.dim, 4, seed=3)
     _set(scan, *variant)
     try:
@@ -108,7 +110,7 @@ def test_conv_with_zoh_and_no_bias(scan, variant):
 def test_conv_split_boundaries(scan, segments):
     """Pieces of a split sequence take their convolution history from the
     piece before; a wide filter with large taps makes any lost halo show."""
-    wl = W.make(4, seqlen=5000, dim=32)
+    wl = W.make(4, seqlen=5000, dim=32, a_jitter=0.5)
     w, cb = W.conv_params(wl.dim, 4, seed=11)
     w *= 4
     _set(scan, S.SSM_VARIANT_CHUNKED, 1, segments)

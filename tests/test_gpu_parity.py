@@ -47,10 +47,17 @@ def _with_variant(scan, variant, segments=0):
     S.library().ssm_scan_set_time_blocks(scan.handle, tb)
 
 
+# a_jitter 0: the stated A_log = log(n + 1) for every channel; 0.5: every
+# channel draws its own A row (A is a learned [E, N] parameter), so a read of
+# the wrong channel's A cannot pass
+JITTER = [0.0, 0.5]
+
+
+@pytest.mark.parametrize("jitter", JITTER, ids=["A_stated", "A_per_channel"])
 @pytest.mark.parametrize("variant", VARIANTS, ids=VARIANT_IDS)
 @pytest.mark.parametrize("idx", sorted(SMALL), ids=lambda i: "shape%d" % i)
-def test_small_parity(scan, idx, variant):
-    wl = W.make(idx, **SMALL[idx])
+def test_small_parity(scan, idx, variant, jitter):
+    wl = W.make(idx, a_jitter=jitter, **SMALL[idx])
     _with_variant(scan, variant)
     try:
         y, h = run(scan, wl)
@@ -91,7 +98,7 @@ def test_full_size_sampled(scan, idx):
 
 @pytest.mark.parametrize("N", [1, 2, 3, 5, 8, 32, 64])
 def test_state_sizes(scan, N):
-    wl = W.make(1, batch=2, seqlen=300, dim=40, dstate=N)
+    wl = W.make(1, batch=2, seqlen=300, dim=40, dstate=N, a_jitter=0.5)
     y, h = run(scan, wl)
     yo, ho = oracle.scan(**oracle_inputs(wl))
     assert_close(y, yo, wl.dtype, "y")
@@ -103,7 +110,7 @@ def test_state_sizes(scan, N):
                                      (16, W.F32), (16, W.BF16)])
 def test_chunked_state_sizes(scan, N, dtype, variant):
     wl = W.make(2, batch=3, seqlen=333, dim=72, dstate=N, dtype=dtype,
-                with_h0=True)
+                with_h0=True, a_jitter=0.5)
     _with_variant(scan, variant)
     try:
         y, h = run(scan, wl)
@@ -206,7 +213,11 @@ def test_forgetting(scan):
 
 
 def test_channel_permutation(scan):
-    wl = W.make(3, batch=2, seqlen=700, dim=48)
+    """Permuting the channels of every per-channel input (x, raw step, z, A
+    rows, D, step bias) permutes the outputs bit for bit. Every channel has
+    its own A row, so a read of another channel's A would show."""
+    wl = W.make(3, batch=2, seqlen=700, dim=48, a_jitter=0.5)
+    assert len({r.tobytes() for r in wl.dev["A_log"]}) == 48
     t = to_device(wl)
     y, h = run(scan, wl, t=t)
     perm = torch.from_numpy(np.random.default_rng(3).permutation(48)).cuda()
@@ -218,6 +229,31 @@ def test_channel_permutation(scan):
     yp, hp = run(scan, wl, t=tp)
     pn = perm.cpu().numpy()
     assert np.array_equal(yp, y[..., pn]) and np.array_equal(hp, h[:, pn])
+
+
+@pytest.mark.parametrize("N", [4, 16])
+def test_sequential_shape_huge_A_freezes_and_forgets(scan, N):
+    """A shape only the sequential variant runs (E * 4 bytes not a multiple
+    of 16) with A_log = 100, so -exp(A_log) overflows float32 to -inf. A zero
+    step must keep the state bitwise (retention 1, not 0 * -inf = NaN); a
+    positive step must forget it (retention 0)."""
+    wl = W.make(1, batch=2, seqlen=90, dim=42, dstate=N, with_h0=True)
+    wl.dev["A_log"] = np.full_like(wl.dev["A_log"], 100.0)
+    wl.dev["A_log"][::3] = 0.5                     # some channels ordinary
+    wl.dev["delta"] = np.zeros_like(wl.dev["delta"])
+    wl.dev["delta_bias"] = None
+    y, h = run(scan, wl, softplus=False)
+    assert scan.last_variant()[0] == S.SSM_VARIANT_SEQUENTIAL
+    assert np.array_equal(h, wl.dev["h0"].astype(np.float64))
+    yo, ho = oracle.scan(**oracle_inputs(wl), delta_softplus=False)
+    assert_close(y, yo, W.F32, "y (zero step)")
+    # positive steps: channels with A_log = 100 forget everything at once
+    wl.dev["delta"] = np.full_like(wl.dev["delta"], 0.05)
+    y, h = run(scan, wl, softplus=False)
+    yo, ho = oracle.scan(**oracle_inputs(wl), delta_softplus=False)
+    assert np.all(np.isfinite(y)) and np.all(np.isfinite(h))
+    assert_close(y, yo, W.F32, "y (forgetting)")
+    assert_close(h, ho, W.F32, "h_last (forgetting)")
 
 
 def test_chunked_unsupported_shapes(scan):

@@ -32,6 +32,8 @@ def _reset(scan):
     S.library().ssm_scan_set_debug(scan.handle, 0, 0)
 
 
+@pytest.mark.parametrize("jitter", [0.0, 0.5], ids=["A_stated",
+                                                    "A_per_channel"])
 @pytest.mark.parametrize("tb", [1, 2])
 @pytest.mark.parametrize("segments", [2, 3, 7])
 @pytest.mark.parametrize("idx,size", [
@@ -39,8 +41,8 @@ def _reset(scan):
     (3, dict(batch=2, seqlen=3000, dim=24, with_h0=True)),
     (1, dict(batch=2, seqlen=2500, dim=40, with_h0=True)),
 ], ids=["long_f32", "layer_bf16", "classifier_f32"])
-def test_split_parity(scan, idx, size, segments, tb):
-    wl = W.make(idx, **size)
+def test_split_parity(scan, idx, size, segments, tb, jitter):
+    wl = W.make(idx, a_jitter=jitter, **size)
     _set(scan, segments, tb)
     try:
         y, h = run(scan, wl)

@@ -37,8 +37,9 @@ def _host(t):
 def test_step_parity(scan, dtype, N, conv, zoh, gate):
     rng = np.random.default_rng(N * 7 + conv)
     b, E, T = 5, 40, 6
+    # every channel has its own A row (A is a learned [E, N] parameter)
     wl = W.make(3, batch=b, seqlen=T, dim=E, dstate=N, dtype=dtype,
-                gated=gate, with_h0=True)
+                gated=gate, with_h0=True, a_jitter=0.5)
     vals = {k: wl.values(k) for k in ("x", "delta", "z", "B", "C")}
     state_h = wl.dev["h0"].astype(np.float64)
     state = torch.from_numpy(wl.dev["h0"].copy()).cuda()
@@ -81,7 +82,7 @@ def test_step_parity(scan, dtype, N, conv, zoh, gate):
 
 def test_decoding_matches_the_scan(scan):
     """Token-by-token decoding (no convolution) equals the chunked scan."""
-    wl = W.make(1, batch=3, seqlen=200, dim=64, with_h0=True)
+    wl = W.make(1, batch=3, seqlen=200, dim=64, with_h0=True, a_jitter=0.5)
     t = to_device(wl)
     y_scan, h_scan = scan(t["x"], t["delta"], t["A_log"], t["B"], t["C"],
                           D=t["D"], z=t["z"], delta_bias=t["delta_bias"],

@@ -37,10 +37,12 @@ CASES = {
                                      (S.SSM_VARIANT_CHUNKED, 1, 1),
                                      (S.SSM_VARIANT_CHUNKED, 1, 3)],
                          ids=["auto", "sequential", "chunked", "chunked_split3"])
+@pytest.mark.parametrize("jitter", [0.0, 0.5], ids=["A_stated",
+                                                    "A_per_channel"])
 @pytest.mark.parametrize("name", sorted(CASES))
-def test_zoh_parity(scan, name, variant):
+def test_zoh_parity(scan, name, variant, jitter):
     idx, size = CASES[name]
-    wl = W.make(idx, **size)
+    wl = W.make(idx, a_jitter=jitter, **size)
     _set(scan, *variant)
     try:
         y, h = run(scan, wl, write_zoh=True)

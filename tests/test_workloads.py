@@ -63,3 +63,20 @@ def test_long_memory_recipe():
     raw = w.dev["delta"]
     assert abs(float(raw.mean()) + 2.0) < 0.02 and abs(float(raw.std()) - 1) < 0.02
     assert abs(float(w.dev["h0"].std()) - 0.1) < 0.01
+
+
+def test_per_channel_A_jitter_keeps_other_draws():
+    """a_jitter draws a distinct A row per channel after every other draw,
+    so the other arrays are unchanged and the rows differ channel to
+    channel."""
+    base = W.make(2, batch=2, seqlen=40, dim=32)
+    jit = W.make(2, batch=2, seqlen=40, dim=32, a_jitter=0.5)
+    for k in base.dev:
+        if k == "A_log" or base.dev[k] is None:
+            continue
+        assert np.array_equal(base.dev[k], jit.dev[k]), k
+    A = jit.dev["A_log"]
+    assert A.dtype == np.float32 and A.shape == (32, 16)
+    assert len({A[e].tobytes() for e in range(32)}) == 32
+    dev = A - base.dev["A_log"]
+    assert 0.35 < float(dev.std()) < 0.65
