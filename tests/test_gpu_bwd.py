@@ -78,11 +78,53 @@ CASES = {
 }
 
 
+@pytest.mark.parametrize("jitter", [0.0, 0.5], ids=["A_stated",
+                                                    "A_per_channel"])
 @pytest.mark.parametrize("zoh", [False, True], ids=["dtBx", "zoh"])
 @pytest.mark.parametrize("name", sorted(CASES))
-def test_bwd_parity(scan, name, zoh):
+def test_bwd_parity(scan, name, zoh, jitter):
     idx, size = CASES[name]
-    _check(scan, W.make(idx, **size), write_zoh=zoh)
+    _check(scan, W.make(idx, a_jitter=jitter, **size), write_zoh=zoh)
+
+
+@pytest.mark.parametrize("idx,size", [
+    (3, dict(batch=2, seqlen=4096, dim=2048)),
+    (1, dict(batch=2, seqlen=2048, dim=2048)),
+], ids=["layer_bf16_E2048_L4096", "classifier_f32_E2048_L2048"])
+def test_bwd_channel_sums_many_tiles(scan, idx, size):
+    """dB and dC sum over every channel, dA_log, dD and the step-bias
+    gradient over every step and sequence: here 128 channel tiles add into
+    each dB/dC row and 2 x L steps into each parameter gradient. All of them,
+    and every per-element gradient, against the oracle at the parity bar."""
+    errs = _check(scan, W.make(idx, a_jitter=0.5, **size), seed=21)
+    for k in ("dB", "dC", "dA_log", "dD", "ddelta_bias"):
+        assert k in errs, k
+
+
+def test_bwd_run_to_run(scan):
+    """The per-element gradients are the same bit for bit on every run. The
+    summed ones (dB, dC, dA_log, dD, step bias) are added with float32
+    atomics, whose order varies from run to run: their spread is bounded
+    far inside the parity bar."""
+    wl = W.make(3, batch=2, seqlen=2048, dim=1024, a_jitter=0.5)
+    t = to_device(wl)
+    b, L, E, N = wl.batch, wl.seqlen, wl.dim, wl.dstate
+    dy_dev, _, dh = _grads(wl.dtype, ((b, L, E), (b, E, N)), 3)
+    dyt, dht = _dev(dy_dev), torch.from_numpy(dh).cuda()
+    runs = []
+    for _ in range(3):
+        g = scan.backward(t["x"], t["delta"], t["A_log"], t["B"], t["C"],
+                          dyt, D=t["D"], z=t["z"], delta_bias=t["delta_bias"],
+                          h0=t["h0"], dh_last=dht)
+        torch.cuda.synchronize()
+        runs.append({k: v.float().cpu().numpy() for k, v in g.items()
+                     if v is not None})
+    for k in runs[0]:
+        for r in runs[1:]:
+            if k in ("dB", "dC", "dA_log", "dD", "ddelta_bias"):
+                assert rel_err(r[k], runs[0][k]) <= 1e-5, k
+            else:
+                assert np.array_equal(r[k], runs[0][k]), k
 
 
 @pytest.mark.parametrize("opts", [dict(gated=False), dict(with_D=False),
@@ -106,7 +148,9 @@ def test_bwd_short_sequences(scan, L):
 def test_bwd_full_size_sampled(scan):
     """The Mamba-2.8B layer at full size: the per-channel gradients of a
     sample of channels against the oracle on those channels (channels are
-    independent); dB and dC (sums over every channel) are finite."""
+    independent). dB and dC, sums over every channel, are finite here; they
+    are compared with the oracle where 128 channel tiles add into them in
+    test_bwd_channel_sums_many_tiles."""
     wl = W.make(3)
     t = to_device(wl)
     b, L, E, N = wl.batch, wl.seqlen, wl.dim, wl.dstate
