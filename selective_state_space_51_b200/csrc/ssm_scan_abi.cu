@@ -109,11 +109,7 @@ int ensure_workspace(ssm_scan_s *h, ssm::ScanParams &p, int64_t tiles,
     h->ws_bytes = bytes;
     h->epoch = 0;
   }
-  if (++h->epoch >= (1u << 30)) {  // tags wrap: clear the flags first
-    if (cudaMemsetAsync(h->ws, 0, off_state, s) != cudaSuccess)
-      return SSM_ERR_CUDA;
-    h->epoch = 1;
-  }
+  if (++h->epoch >= (1u << 30)) h->epoch = 1;
   unsigned char *base = static_cast<unsigned char *>(h->ws);
   const size_t sz = align256(nstate * sizeof(float));
   p.flags = reinterpret_cast<unsigned *>(base);
@@ -125,9 +121,17 @@ int ensure_workspace(ssm_scan_s *h, ssm::ScanParams &p, int64_t tiles,
   p.epoch = h->epoch;
   p.spin_limit = h->spin_limit;
   p.debug = h->debug;
-  return cudaMemsetAsync(p.ticket, 0, sizeof(unsigned), s) == cudaSuccess
-             ? SSM_OK
-             : SSM_ERR_CUDA;
+  // The launch ticket restarts at zero and this call's publication flags are
+  // cleared on the stream before the launch, so a flag left by an earlier
+  // call (or an earlier replay of a captured graph) is never taken for one of
+  // this call's; the per-call tag is a second guard for eager calls.
+  if (cudaMemsetAsync(p.ticket, 0, sizeof(unsigned), s) != cudaSuccess ||
+      cudaMemsetAsync(p.flags, 0, nflags * sizeof(unsigned), s) !=
+          cudaSuccess) {
+    cudaGetLastError();
+    return SSM_ERR_CUDA;
+  }
+  return SSM_OK;
 }
 
 // Pieces per sequence: enough that the blocks fill every resident slot once,

@@ -90,3 +90,47 @@ def test_scan_graph_replay_matches_eager():
         assert scan.sync_status() == S.SSM_OK
     finally:
         scan.close()
+
+
+def test_split_scan_graph_replays_with_new_inputs():
+    """A split call (pieces joined by the look-back over publication flags)
+    captured once and replayed after its input buffers were refilled: every
+    replay must match the oracle on the inputs it saw, so no publication of
+    an earlier replay can be taken for one of the current replay."""
+    import oracle
+    from gpu_helpers import assert_close, oracle_inputs
+    scan = S.SelectiveScan(0)
+    try:
+        scan.set_variant(S.SSM_VARIANT_CHUNKED, 4)
+        wls = [W.make(4, seqlen=6000, dim=32, a_jitter=0.5, seed=s)
+               for s in (101, 202)]
+        ts = [to_device(wl) for wl in wls]
+        buf = {k: (None if v is None else v.clone())
+               for k, v in ts[0].items()}
+        y = torch.empty_like(buf["x"])
+        h = torch.empty((1, 32, 16), dtype=torch.float32, device="cuda")
+
+        def call():
+            scan(buf["x"], buf["delta"], buf["A_log"], buf["B"], buf["C"],
+                 D=buf["D"], z=buf["z"], delta_bias=buf["delta_bias"],
+                 h0=buf["h0"], y=y, h_last=h)
+        call()                       # grows the workspace before capture
+        torch.cuda.synchronize()
+        assert tuple(scan.last_variant()) == (S.SSM_VARIANT_CHUNKED, 4)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            call()
+        for k in (1, 0, 1):
+            for name, v in ts[k].items():
+                if v is not None:
+                    buf[name].copy_(v)
+            graph.replay()
+            torch.cuda.synchronize()
+            assert scan.sync_status() == S.SSM_OK
+            yo, ho = oracle.scan(**oracle_inputs(wls[k]))
+            assert_close(y.cpu().numpy(), yo, W.F32, "y replay (inputs %d)" % k)
+            assert_close(h.cpu().numpy(), ho, W.F32,
+                         "h_last replay (inputs %d)" % k)
+        del graph
+    finally:
+        scan.close()
