@@ -48,10 +48,12 @@
  *     carries at most one in-flight call on any stream at a time when it
  *     needs workspace (long sequences with few channels, and the backward
  *     pass's checkpoints). Different handles are independent.
- *   - CUDA graphs: ssm_scan_step, and ssm_scan_fwd / ssm_scan_fwd_conv when
- *     they do not split sequences, only enqueue kernels, so their calls can
- *     be captured into a graph and replayed. Calls that grow a workspace do
- *     so on their first use: make that call before capturing.
+ *   - CUDA graphs: ssm_scan_step, ssm_scan_fwd and ssm_scan_fwd_conv only
+ *     enqueue memsets and kernels once their workspace exists, so their
+ *     calls can be captured into a graph and replayed, split sequences
+ *     included (each call clears its own publication flags on the stream).
+ *     Calls that grow a workspace do so on their first use with that shape:
+ *     make that call before capturing.
  */
 #ifndef SSM_SCAN_H
 #define SSM_SCAN_H
@@ -316,9 +318,12 @@ SSM_API int ssm_scan_step(ssm_scan_t h, const void *x_new, void *conv_state,
  *   device   : CUDA device of every pointer; it must be current.
  *   segments : pieces per sequence: 0 chooses by shape, 1 never splits, and
  *              a larger value forces that count.
- *   status   : NULL, or a device int the caller has zeroed. It is set to 1
- *              if a bounded wait between thread blocks gave up, and the
- *              outputs are then invalid.
+ *   status   : a device int the caller has zeroed, or NULL. A split call
+ *              sets it to 1 if a bounded wait between thread blocks gave
+ *              up; the outputs are then invalid. With status NULL the call
+ *              never splits (segments 0 then means 1, and segments > 1
+ *              returns SSM_ERR_INVALID), so no such wait can go unreported.
+ *   flags    : SSM_DELTA_SOFTPLUS and SSM_WRITE_ZOH, as for ssm_scan_fwd.
  *   the rest : as for ssm_scan_fwd. Additionally dstate is 4, 8 or 16,
  *              dim * element size is a multiple of 16 bytes, and x, delta,
  *              z, B, C are 16-byte aligned (else SSM_ERR_UNSUPPORTED or
@@ -329,8 +334,9 @@ SSM_API int ssm_scan_step(ssm_scan_t h, const void *x_new, void *conv_state,
  * The first call on a device looks up the array's device address and clears
  * it, which synchronizes that device: make that first call before any stream
  * capture. Every call shares the one array, which keeps the last call's
- * contents. Calls that overlap on the GPU race, so callers on several
- * streams or host threads must serialize them.
+ * contents; a split call clears its launch ticket and publication flags on
+ * the stream before its kernel. Calls that overlap on the GPU race, so
+ * callers on several streams or host threads must serialize them.
  */
 SSM_API int ssm_scan_fwd_static_scratch(
     int device, const void *x, const void *delta, const float *A_log,

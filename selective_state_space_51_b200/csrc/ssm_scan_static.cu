@@ -52,15 +52,18 @@ using S8b = ssm::ChunkCfg<bf16,   2, 1, 2, 32, 4, 32, 0, 0>;
 using S8f = ssm::ChunkCfg<float,  2, 1, 2, 16, 4, 32, 0, 0>;
 using S4f = ssm::ChunkCfg<float,  1, 1, 1, 16, 4,  0, 0, 0>;
 
-template <class Cfg>
+template <class Cfg, bool ZOH>
 int run(DeviceScratch &d, ssm::ScanParams &p, int segments, int *status,
         cudaStream_t s) {
   const int64_t tiles = (p.dim + Cfg::G - 1) / Cfg::G;
   int64_t segs = segments;
+  // Without a caller status word a given-up bounded wait could not be
+  // reported, so such calls never split.
+  if (!status) segs = 1;
   if (segs <= 0) {  // enough pieces to fill every resident block slot once
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-            &per_sm, ssm::scan_chunked_kernel<Cfg, true>, Cfg::THREADS,
+            &per_sm, ssm::scan_chunked_kernel<Cfg, true, ZOH>, Cfg::THREADS,
             Cfg::SMEM_BYTES) != cudaSuccess) {
       cudaGetLastError();
       return SSM_ERR_CUDA;
@@ -80,17 +83,18 @@ int run(DeviceScratch &d, ssm::ScanParams &p, int segments, int *status,
   }
   p.segments = int(segs);
   p.seg_len = seg_len;
-  if (cudaFuncSetAttribute(ssm::scan_chunked_kernel<Cfg, true>,
+  if (cudaFuncSetAttribute(ssm::scan_chunked_kernel<Cfg, true, ZOH>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Cfg::SMEM_BYTES) != cudaSuccess ||
-      cudaFuncSetAttribute(ssm::scan_chunked_kernel<Cfg, false>,
+      cudaFuncSetAttribute(ssm::scan_chunked_kernel<Cfg, false, ZOH>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Cfg::SMEM_BYTES) != cudaSuccess) {
     cudaGetLastError();
     return SSM_ERR_CUDA;
   }
   if (segs <= 1) {
-    ssm::scan_chunked_kernel<Cfg, false>
+    if (p.batch * tiles > 0x7fffffff) return SSM_ERR_UNSUPPORTED;
+    ssm::scan_chunked_kernel<Cfg, false, ZOH>
         <<<unsigned(p.batch * tiles), Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(p);
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
   }
@@ -108,24 +112,37 @@ int run(DeviceScratch &d, ssm::ScanParams &p, int segments, int *status,
   p.agg_decay = reinterpret_cast<float *>(base + off_state + state_bytes);
   p.incl_state = reinterpret_cast<float *>(base + off_state + 2 * state_bytes);
   p.ticket = reinterpret_cast<unsigned *>(base + 4);
-  p.status = status ? status : reinterpret_cast<int *>(base);
+  p.status = status;
   p.spin_limit = kSpinLimit;
   p.debug = 0;
-  // The array keeps the previous call's contents: the ticket must restart
-  // at zero, and flags are told apart by a per-call tag. The array was
-  // cleared when the device was set up; it is cleared again if the tag wraps.
-  if (++d.epoch >= (1u << 30)) {
-    if (cudaMemsetAsync(base, 0, kScratchBytes, s) != cudaSuccess)
-      return SSM_ERR_CUDA;
-    d.epoch = 1;
-  }
+  // The array keeps the previous call's contents: the ticket restarts at
+  // zero and this call's publication flags are cleared on the stream before
+  // the launch (memsets, not allocations), so no flag of an earlier call can
+  // be taken for this one's. The per-call tag is a second guard.
+  if (++d.epoch >= (1u << 30)) d.epoch = 1;
   p.epoch = d.epoch;
-  if (cudaMemsetAsync(p.ticket, 0, sizeof(unsigned), s) != cudaSuccess)
+  if (cudaMemsetAsync(p.ticket, 0, sizeof(unsigned), s) != cudaSuccess ||
+      cudaMemsetAsync(p.flags, 0, nflags * sizeof(unsigned), s) !=
+          cudaSuccess) {
+    cudaGetLastError();
     return SSM_ERR_CUDA;
-  ssm::scan_chunked_kernel<Cfg, true>
+  }
+  ssm::scan_chunked_kernel<Cfg, true, ZOH>
       <<<unsigned(segs * p.batch * tiles), Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(
           p);
   return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+template <bool ZOH>
+int dispatch(DeviceScratch &d, ssm::ScanParams &p, int dtype, int segments,
+             int *status, cudaStream_t s) {
+  if (dtype == SSM_BF16) {
+    if (p.dstate == 16) return run<S16b, ZOH>(d, p, segments, status, s);
+    return run<S8b, ZOH>(d, p, segments, status, s);
+  }
+  if (p.dstate == 16) return run<S16f, ZOH>(d, p, segments, status, s);
+  if (p.dstate == 8) return run<S8f, ZOH>(d, p, segments, status, s);
+  return run<S4f, ZOH>(d, p, segments, status, s);
 }
 
 }  // namespace
@@ -143,8 +160,11 @@ int ssm_scan_fwd_static_scratch(int device, const void *x, const void *delta,
   if (!x || !delta || !A_log || !B || !C || !y) return SSM_ERR_INVALID;
   if (dims.batch <= 0 || dims.seqlen <= 0 || dims.dim <= 0 || dims.dstate <= 0)
     return SSM_ERR_INVALID;
-  if (flags & ~uint32_t(SSM_DELTA_SOFTPLUS)) return SSM_ERR_INVALID;
+  if (flags & ~uint32_t(SSM_DELTA_SOFTPLUS | SSM_WRITE_ZOH))
+    return SSM_ERR_INVALID;
   if (segments < 0) return SSM_ERR_INVALID;
+  // a split call reports a given-up wait through the caller's status word
+  if (segments > 1 && !status) return SSM_ERR_INVALID;
   if (device < 0 || device >= kMaxDevices) return SSM_ERR_INVALID;
   if (dtype != SSM_F32 && dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
   const int esz = dtype == SSM_F32 ? 4 : 2;
@@ -210,16 +230,12 @@ int ssm_scan_fwd_static_scratch(int device, const void *x, const void *delta,
   p.batch = dims.batch; p.seqlen = dims.seqlen; p.dim = dims.dim;
   p.dstate = int(dims.dstate);
   p.softplus = (flags & SSM_DELTA_SOFTPLUS) ? 1 : 0;
+  p.write_zoh = (flags & SSM_WRITE_ZOH) ? 1 : 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
   std::lock_guard<std::mutex> guard(g_lock);  // the epoch and the array
-  if (dtype == SSM_BF16) {
-    if (dims.dstate == 16) return run<S16b>(*d, p, segments, status, s);
-    return run<S8b>(*d, p, segments, status, s);
-  }
-  if (dims.dstate == 16) return run<S16f>(*d, p, segments, status, s);
-  if (dims.dstate == 8) return run<S8f>(*d, p, segments, status, s);
-  return run<S4f>(*d, p, segments, status, s);
+  return p.write_zoh ? dispatch<true>(*d, p, dtype, segments, status, s)
+                     : dispatch<false>(*d, p, dtype, segments, status, s);
 }
 
 }  // extern "C"
