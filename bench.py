@@ -76,12 +76,56 @@ def max_over_ranks(value: float, dist=None, device=None) -> float:
 # ----------------------------------------------------------------- workload
 CONV_WIDTH = 4
 
-# DRAM bytes (read + write) of one launch of the timed kernel, from the ncu
-# capture summarised in profiles/scan_chunked_mamba2p8b_layer.md (current
-# build of the chunked kernel, Mamba-2.8B layer). Workloads without a capture
-# of their current kernel report null.
-NCU_TRAFFIC = {("scan", 3): 1.010016e9 + 0.316603e9}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
+# the timed kernel, from one ncu capture, keyed by (op, workload shape), with
+# the hash of the kernel sources that capture was taken from. A figure whose
+# sources have changed since is stale: the line then reports null.
+NCU_TRAFFIC = {("scan", 3): (1.010016e9 + 0.316603e9, "e2fc272f14a6fc87")}
+KERNEL_SOURCES = ("kernel_chunked.cuh", "device_math.cuh", "scan_params.cuh")
 DECODE_BATCH = 1024
+
+
+def kernel_source_hash() -> str:
+    """sha256 (first 16 hex digits) of the forward kernel's sources."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "selective_state_space_51_b200", "csrc",
+                               name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_record(op: str, shape: int):
+    """(traffic, source description) for the roofline record."""
+    entry = NCU_TRAFFIC.get((op, shape))
+    if entry is None:
+        return None, "no ncu capture of this kernel on this workload"
+    value, src_hash = entry
+    now = kernel_source_hash()
+    if now != src_hash:
+        return None, ("ncu capture of kernel sources %s; the sources are now "
+                      "%s, so the figure is stale" % (src_hash, now))
+    return value, ("ncu dram__bytes_read.sum + dram__bytes_write.sum, one "
+                   "launch, kernel sources %s" % src_hash)
+
+
+def workload_config(wl, op: str, world: int, shape: int) -> dict:
+    """The config record both arms print for the same workload."""
+    from selective_state_space_51_b200 import workloads as W
+    name = W.shape_description(shape)
+    if op == "conv":
+        name += "; causal depthwise conv width %d + SiLU fused in front" % (
+            CONV_WIDTH)
+    elif op == "bwd":
+        name += "; backward"
+    elif op == "step":
+        name = ("decode step, Mamba-2.8B layer shape: %d sequences x E=%d x "
+                "N=%d float32 state, conv width %d, %s activations" % (
+                    wl.batch, wl.dim, wl.dstate, CONV_WIDTH, wl.dtype))
+    return {"workload": name, "op": op, "global_batch": world * wl.batch,
+            "seq_len": wl.seqlen, "dim": wl.dim, "dstate": wl.dstate,
+            "parallelism": "dp%d" % world}
 
 
 def algorithmic_bytes(wl, op: str = "scan") -> int:
@@ -224,34 +268,43 @@ def cpu_oracle_rate(wl, target_s: float = 10.0, inputs=None, k=None):
 
 
 def run_reference(args):
-    """--impl reference: the float64 CPU oracle on the same workload."""
+    """--impl reference: the float64 CPU oracle on the same workload. One
+    step is the oracle over a bounded sample of the workload (every sequence,
+    the first k channels, all L steps), k sized so that the whole run takes
+    about --reference-budget seconds; ms_per_step is that step's wall time
+    and value the sample's scan elements per second."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
+    if args.op != "scan":
+        print(json.dumps({"impl": "reference", "unavailable":
+                          "the oracle arm times the forward scan only"}))
+        return 0
     from selective_state_space_51_b200 import workloads as W
     wl = W.make(args.shape)
-    per_step = []
+    steps_ms, rates = [], []
     sample = None
-    # the whole run stays within about --reference-budget seconds
     target = max(0.05, args.reference_budget / (args.warmup + args.steps))
     inputs = oracle_inputs(wl)
     k = None
     for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
         r = cpu_oracle_rate(wl, target_s=target, inputs=inputs, k=k)
+        dt = time.perf_counter() - t0
         k = r["channels"]
         if i >= args.warmup:
-            per_step.append(r["value"])
+            steps_ms.append(1e3 * dt)
+            rates.append(r["value"])
             sample = r
-    value = statistics.median(per_step)
+    value = statistics.median(rates)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * wl.elements / value,
+        "ms_per_step": statistics.median(steps_ms),
+        "ms_per_step_full_workload_extrapolated": 1e3 * wl.elements / value,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
-        "config": {"workload": W.shape_description(args.shape),
-                   "global_batch": wl.batch, "seq_len": wl.seqlen,
-                   "parallelism": "cpu oracle, rank 0 only"},
+        "config": workload_config(wl, "scan", args.gpus, args.shape),
         "cpu_baseline": dict(sample, value=value),
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -558,6 +611,7 @@ def _finish(args, op, world, rank, local, dev, dist, scan, clocks, total_ms,
               % (wl.batch * wl.dim * wl.dstate * 4 / 1e6))
     else:
         metric, unit = METRIC, UNIT
+        traffic, traffic_source = traffic_record(op.name, args.shape)
         roof = {"bound": "alu", "unit": "Gexp/s",
                 "achieved": achieved_exp / 1e9,
                 "peak": sfu_peak_max / 1e9,
@@ -568,7 +622,7 @@ def _finish(args, op, world, rank, local, dev, dist, scan, clocks, total_ms,
                                              peaks["source"]),
                 "frac_at_sampled_clock": (achieved_exp / sfu_peak_run
                                           if sfu_peak_run else None),
-                "traffic": NCU_TRAFFIC.get((op.name, args.shape)),
+                "traffic": traffic, "traffic_source": traffic_source,
                 "algorithmic_bytes": nbytes}
         l2 = "inputs larger than L2 (%.0f MB read per step)" % (nbytes / 1e6)
     line = {
@@ -576,10 +630,8 @@ def _finish(args, op, world, rank, local, dev, dist, scan, clocks, total_ms,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "io_dtype": wl.dtype, "data": "synthetic",
-        "config": {"workload": op.workload, "op": op.name,
-                   "global_batch": world * wl.batch, "seq_len": wl.seqlen,
-                   "dim": wl.dim, "dstate": wl.dstate,
-                   "parallelism": "dp%d" % world, "l2": l2},
+        "config": workload_config(wl, op.name, world, args.shape),
+        "l2": l2,
         "gb_per_s": gbps,
         "roofline": roof,
         "e2e": (None if e2e_ms is None else
