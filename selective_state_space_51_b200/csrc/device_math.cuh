@@ -220,6 +220,75 @@ template <> struct PairMath<__nv_bfloat16> {
   }
 };
 
+// Retentions close to 1 for float32 activations. The SFU's exp2 errs by up to
+// about 1.4 units in the last place near 1, and a retention that repeats
+// step after step (a held input) compounds that error linearly over the
+// state's memory, about 1/|z| steps. Where |z| = |delta A| < 2^-8 the
+// retention is instead the Taylor polynomial 1 + z + z^2/2 (truncation below
+// |z|^3/6 < 1e-8, a sixth of a unit in the last place), rounded once by its
+// final fused multiply-add. It is written in zl = z log2(e):
+// e^z = 1 + zl (c1 + zl c2), c1 = ln 2, c2 = (ln 2)^2 / 2.
+constexpr float kNear1Zl = 0.0056355275034725f;  // 2^-8 / ln 2
+constexpr float kNear1C1 = 0.6931471805599453f;
+constexpr float kNear1C2 = 0.2402265069591007f;
+
+// The per-lane step-size bound below which all four of a lane's states are
+// in the polynomial's band: kNear1Zl / max_n |A'_n| (A' = A log2 e, <= 0).
+__device__ __forceinline__ float near1_bound(float2 A01, float2 A23) {
+  const float m = fmaxf(fmaxf(-A01.x, -A01.y), fmaxf(-A23.x, -A23.y));
+  return kNear1Zl / m;  // +inf when every A is 0
+}
+
+// For one step of four states (two packed pairs): when |d| < bound, replace
+// the SFU retentions a01, a23 (of arguments zl01, zl23) by the polynomial.
+// One comparison per step and lane; the polynomial runs on packed pairs and
+// only its last multiply-add is predicated.
+__device__ __forceinline__ void near1_retentions(float d, float bound,
+                                                 float2 zl01, float2 zl23,
+                                                 float2 &a01, float2 &a23) {
+  asm("{\n"
+      " .reg .pred p;\n"
+      " .reg .f32 ad;\n"
+      " .reg .b64 z0, z1, t0, t1, r0, r1, c1, c2, one;\n"
+      " abs.f32 ad, %4;\n"
+      " setp.lt.f32 p, ad, %5;\n"
+      " mov.b64 z0, {%6, %7};\n"
+      " mov.b64 z1, {%8, %9};\n"
+      " mov.b64 c2, {%10, %10};\n"
+      " mov.b64 c1, {%11, %11};\n"
+      " mov.b64 one, {%12, %12};\n"
+      " mov.b64 r0, {%0, %1};\n"
+      " mov.b64 r1, {%2, %3};\n"
+      " fma.rn.f32x2 t0, z0, c2, c1;\n"
+      " fma.rn.f32x2 t1, z1, c2, c1;\n"
+      " @p fma.rn.f32x2 r0, z0, t0, one;\n"
+      " @p fma.rn.f32x2 r1, z1, t1, one;\n"
+      " mov.b64 {%0, %1}, r0;\n"
+      " mov.b64 {%2, %3}, r1;\n"
+      "}"
+      : "+f"(a01.x), "+f"(a01.y), "+f"(a23.x), "+f"(a23.y)
+      : "f"(d), "f"(bound), "f"(zl01.x), "f"(zl01.y), "f"(zl23.x),
+        "f"(zl23.y), "f"(kNear1C2), "f"(kNear1C1), "f"(1.0f));
+}
+
+// near1_retentions for a step that the whole warp takes together: the
+// polynomial is skipped, by a branch every lane takes the same way, when no
+// lane of the warp has a step size in the band. Call it with all 32 lanes.
+__device__ __forceinline__ void near1_retentions_warp(float d, float bound,
+                                                      float2 zl01, float2 zl23,
+                                                      float2 &a01,
+                                                      float2 &a23) {
+  if (__any_sync(0xffffffffu, fabsf(d) < bound))
+    near1_retentions(d, bound, zl01, zl23, a01, a23);
+}
+
+// The same for one state (scalar kernels): e^z for zl = z log2 e.
+__device__ __forceinline__ float retention_f32(float zl) {
+  const float a = ex2(zl);
+  const float p = fmaf(zl, fmaf(zl, kNear1C2, kNear1C1), 1.0f);
+  return fabsf(zl) < kNear1Zl ? p : a;
+}
+
 // Exact zero-order-hold write factor expm1(z) / A, z = d A, for one state:
 // given zl = z log2(e) (so a = 2^zl) and invA = 1/A. For |z| < 1/8 it is
 // d phi(z) with phi(z) = (e^z - 1)/z = 1 + z/2 + z^2/6 + z^3/24 + z^4/120 +

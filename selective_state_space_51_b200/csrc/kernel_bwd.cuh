@@ -140,6 +140,13 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
       A2[i] = fmaxf(Av[i] * kLog2e, -FLT_MAX);
       iA[i] = -expf(-al[i]);
     }
+  }
+  // float32: step sizes below this keep the retentions on the near-1
+  // polynomial, as in the forward kernels
+  const float near_bound = near1_bound(make_float2(A2[0], A2[1]),
+                                       make_float2(A2[2], A2[3]));
+  (void)near_bound;
+  if (ch_ok) {
     if (p.dh_last) {
       const float4 v = *reinterpret_cast<const float4 *>(
           p.dh_last + (b * E + e) * N + 4 * g);
@@ -287,14 +294,17 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const float zl = sv * A2[i];
-            const float a = ex2(zl);
+            const float a = sizeof(T) == 4 ? retention_f32(zl) : ex2(zl);
             h[i] = fmaf(a, h[i], zoh_factor(sv, zl, a, iA[i]) * xv * Bv[i]);
           }
         } else {  // packed pairs: a = 2^(s A'), h = a h + (s x) B
           const float2 s2 = make_float2(sv, sv);
           const float2 sx2 = make_float2(sv * xv, sv * xv);
-          const float2 a01 = ex2x2(mul2(s2, make_float2(A2[0], A2[1])));
-          const float2 a23 = ex2x2(mul2(s2, make_float2(A2[2], A2[3])));
+          const float2 zl01 = mul2(s2, make_float2(A2[0], A2[1]));
+          const float2 zl23 = mul2(s2, make_float2(A2[2], A2[3]));
+          float2 a01 = ex2x2(zl01), a23 = ex2x2(zl23);
+          if constexpr (sizeof(T) == 4)
+            near1_retentions(sv, near_bound, zl01, zl23, a01, a23);
           const float2 h01 = fma2(a01, make_float2(h[0], h[1]),
                                   mul2(sx2, make_float2(Bq.x, Bq.y)));
           const float2 h23 = fma2(a23, make_float2(h[2], h[3]),
@@ -381,8 +391,11 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
             const float2 B23 = make_float2(Bv[2], Bv[3]);
             const float2 C01 = make_float2(Cv[0], Cv[1]);
             const float2 C23 = make_float2(Cv[2], Cv[3]);
-            const float2 a01 = ex2x2(mul2(s2, make_float2(A2[0], A2[1])));
-            const float2 a23 = ex2x2(mul2(s2, make_float2(A2[2], A2[3])));
+            const float2 zl01 = mul2(s2, make_float2(A2[0], A2[1]));
+            const float2 zl23 = mul2(s2, make_float2(A2[2], A2[3]));
+            float2 a01 = ex2x2(zl01), a23 = ex2x2(zl23);
+            if constexpr (sizeof(T) == 4)
+              near1_retentions(sv, near_bound, zl01, zl23, a01, a23);
             const float2 ch = fma2(C23, hc23, mul2(C01, hc01));
             pre = ch.x + ch.y;
             float2 l01 = fma2(dy2, C01, make_float2(lam[0], lam[1]));
@@ -411,7 +424,7 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const float zl = sv * A2[i];
-              const float a = ex2(zl);
+              const float a = sizeof(T) == 4 ? retention_f32(zl) : ex2(zl);
               pre = fmaf(Cv[i], hcur[i], pre);
               lam[i] = fmaf(dyv, Cv[i], lam[i]);
               const float da = lam[i] * hprev[i];

@@ -280,6 +280,10 @@ scan_chunked_kernel(const ScanParams p) {
   }
   const float bias = (ch_ok && p.delta_bias) ? p.delta_bias[e] : 0.0f;
   const float Dv = (ch_ok && p.D) ? p.D[e] : 0.0f;
+  // float32: step sizes below this keep all four retentions on the
+  // near-1 polynomial
+  const float near_bound = near1_bound(A01, A23);
+  (void)near_bound;
   // fused convolution weights, right-aligned: cw[kScanConvMaxWidth - 1]
   // multiplies the newest input, leading taps of a narrower filter are zero
   float cw[kScanConvMaxWidth] = {};
@@ -562,8 +566,11 @@ scan_chunked_kernel(const ScanParams p) {
             bc_row(jb * BS + s, Bq, Cq);
             const float2 dA = make_float2(dd[s].x, dd[s].x);
             const float2 zl01 = mul2(dA, A01), zl23 = mul2(dA, A23);
-            const float2 a01 = ex2x2(zl01);
-            const float2 a23 = ex2x2(zl23);
+            float2 a01 = ex2x2(zl01);
+            float2 a23 = ex2x2(zl23);
+            if constexpr (ESZ == 4)  // float32: retentions near 1 exactly
+              near1_retentions_warp(dd[s].x, near_bound, zl01, zl23, a01,
+                                    a23);
             if (MODE == kWalkMain) {
               const float2 dx = make_float2(dd[s].y, dd[s].y);
               float2 w01 = mul2(dx, make_float2(Bq.x, Bq.y));
@@ -618,8 +625,12 @@ scan_chunked_kernel(const ScanParams p) {
               bc_row(r0 + j, Bq, Cq);
               const float2 dA = make_float2(dd.x, dd.x);
               const float2 dx = make_float2(dd.y, dd.y);
-              a01[j] = ex2x2(mul2(dA, A01));
-              a23[j] = ex2x2(mul2(dA, A23));
+              const float2 zl01 = mul2(dA, A01), zl23 = mul2(dA, A23);
+              a01[j] = ex2x2(zl01);
+              a23[j] = ex2x2(zl23);
+              if constexpr (ESZ == 4)
+                near1_retentions(dd.x, near_bound, zl01, zl23, a01[j],
+                                 a23[j]);
               w01[j] = mul2(dx, make_float2(Bq.x, Bq.y));
               w23[j] = mul2(dx, make_float2(Bq.z, Bq.w));
               Bb01 = fma2(a01[j], Bb01, w01[j]);

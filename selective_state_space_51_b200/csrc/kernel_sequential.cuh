@@ -92,7 +92,7 @@ scan_sequential_kernel(const ScanParams p) {
     for (int n = 0; n < NMAX; ++n) {
       if (n < N) {
         const float zl = step * A2[n];
-        const float a = ex2(zl);
+        const float a = sizeof(T) == 4 ? retention_f32(zl) : ex2(zl);
         const float wf = p.write_zoh ? zoh_factor(step, zl, a, iA[n]) * xv : dx;
         h[n] = fmaf(a, h[n], wf * Act<T>::load(Bm + r + n));
         acc = fmaf(Act<T>::load(Cm + r + n), h[n], acc);

@@ -192,7 +192,7 @@ __global__ void __launch_bounds__(128, VEC ? 8 : 1)
           const int k = i0 + i;
           if (n0 + k < N) {
             const float zl = step * Aq[i];
-            const float a = ex2(zl);
+            const float a = sizeof(T) == 4 ? retention_f32(zl) : ex2(zl);
             const float wf =
                 p.write_zoh
                     ? zoh_factor(step, zl, a,
