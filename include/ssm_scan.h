@@ -248,9 +248,12 @@ SSM_API int ssm_scan_set_time_blocks(ssm_scan_t h, int time_blocks);
  * ssm_scan_set_debug: testing hook. `flags` bit 0 makes the first piece of
  * every split sequence skip its publication, so that the bounded wait of its
  * successor runs out: that call then reports SSM_ERR_TIMEOUT through
- * ssm_scan_sync_status and its outputs are invalid. `spin_limit` bounds every
- * wait between thread blocks (in polls of roughly 1 us each; 0 restores the
- * default of 10^6 polls, about one second). Returns SSM_ERR_INVALID for a NULL handle.
+ * ssm_scan_sync_status and its outputs are invalid. Bit 1 makes
+ * ssm_scan_step use its per-thread-load kernel where it would use the
+ * bulk-copy one. `spin_limit` bounds every wait between thread blocks and
+ * every wait for a bulk copy (in polls of roughly 1 us each; 0 restores the
+ * default of 10^6 polls, about one second). Returns SSM_ERR_INVALID for a
+ * NULL handle.
  */
 SSM_API int ssm_scan_set_debug(ssm_scan_t h, unsigned flags,
                                unsigned spin_limit);
@@ -293,6 +296,14 @@ SSM_API int ssm_scan_sync_status(ssm_scan_t h, struct CUstream_st *stream);
  *   dims.seqlen must be 1; dims.dstate is 1..64.
  * state, conv_state and y must not overlap each other or any input. Launches
  * on `stream` without waiting. Errors as for ssm_scan_fwd.
+ * For dstate 4, 8 or 16 (rows of B and C of at least 16 bytes), dim * element
+ * size a multiple of 16 bytes and every buffer 16-byte aligned, each block's
+ * state, inputs, conv buffers and y move as bulk copies between global and
+ * shared memory; its waits for them are bounded, and one that gives up is
+ * reported as SSM_ERR_TIMEOUT by ssm_scan_sync_status (the state is then
+ * partly updated). Other shapes use per-thread loads. The first call on a
+ * handle allocates its 256-byte status block on `stream`: make it before
+ * capturing the step into a CUDA graph.
  */
 SSM_API int ssm_scan_step(ssm_scan_t h, const void *x_new, void *conv_state,
                           const float *conv_weight, const float *conv_bias,

@@ -42,7 +42,18 @@ struct StepParams {
   int64_t batch, dim;
   int dstate;
   int softplus, write_zoh;
+  // bulk-copy variant only: device status word (kStepTimeout on a wait that
+  // gave up) and the polls a wait makes before giving up
+  int *status;
+  unsigned spin_limit;
 };
+
+// Device status written by the bulk-copy decode step (same word as the
+// scan's status; 1 = a bounded wait gave up).
+constexpr int kStepTimeout = 1;
+// Polls of the final wait for copies still in flight after a wait gave up
+// (independent of the caller's limit, which may be tiny in tests).
+constexpr unsigned kStepDrainPolls = 1u << 22;
 
 constexpr int kMaxConvWidth = 8;
 
@@ -223,6 +234,273 @@ __global__ void __launch_bounds__(128, VEC ? 8 : 1)
       if (p.z) out *= silu(Act<T>::load(static_cast<const T *>(p.z) + ch));
       Act<T>::store(static_cast<T *>(p.y) + ch, out);
     }
+  }
+}
+
+
+// ---------------------------------------------------------------------------
+// Decode step with every per-row input and output moved by bulk copies.
+// A block owns 128 consecutive channels and walks batch rows b = blockIdx.y,
+// blockIdx.y + gridDim.y, ... For one row, everything the block reads is a
+// handful of contiguous runs: its channels' [128 x N] float32 state, their
+// x, raw step and z values, their [128 x K] conv buffers, and the row's B and
+// C. Each run arrives in shared memory as one bulk copy (cp.async.bulk from
+// this GPU's own memory; completion counted on an mbarrier), and the updated
+// state, conv buffers and y leave the same way. Three buffers rotate over the
+// rows, so the copies of the next two rows are in flight while one row is
+// updated, and the state moves as whole cache lines.
+// A thread owns one channel (N = 4, 8 or 16 states, N/4 16-byte chunks of
+// its shared row). Its chunks are visited in an order rotated by its place in
+// the quarter warp, so the 16-byte shared accesses of 8 consecutive threads
+// fall in distinct banks. Every wait on an mbarrier is bounded; a wait that
+// gives up sets the status word, and the block stops after draining its
+// copies.
+constexpr int kStepBulkBufs = 3;
+
+template <typename T, int N>
+struct StepBulkLayout {
+  static constexpr int ESZ = sizeof(T);
+  static constexpr int STATE = 0;
+  static constexpr int X = 128 * N * 4;
+  static constexpr int DL = X + 128 * ESZ;
+  static constexpr int Z = DL + 128 * ESZ;
+  static constexpr int Y = Z + 128 * ESZ;
+  static constexpr int CONV = Y + 128 * ESZ;
+  static constexpr int BM = CONV + 128 * kMaxConvWidth * ESZ;
+  static constexpr int CM = BM + (N * ESZ + 15) / 16 * 16;
+  static constexpr int BUF = CM + (N * ESZ + 15) / 16 * 16;  // one buffer
+  static constexpr int BAR = kStepBulkBufs * BUF;            // mbarriers
+  static constexpr int BYTES = BAR + 8 * kStepBulkBufs;
+  static_assert(BUF % 16 == 0 && X % 16 == 0 && CONV % 16 == 0,
+                "bulk copy destinations are 16-byte aligned");
+};
+
+__device__ __forceinline__ unsigned smem_addr(const void *p) {
+  return static_cast<unsigned>(__cvta_generic_to_shared(p));
+}
+
+// Bounded wait for phase `parity` of an mbarrier; false if it gave up.
+__device__ __forceinline__ bool mbar_wait(unsigned bar, unsigned parity,
+                                          unsigned limit) {
+  for (unsigned i = 0; i < limit; ++i) {
+    unsigned done;
+    asm volatile(
+        "{\n .reg .pred p;\n"
+        " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void bulk_load(unsigned dst, const void *src,
+                                          unsigned bytes, unsigned bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_store(void *dst, unsigned src,
+                                           unsigned bytes) {
+  asm volatile(
+      "cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+      "r"(src), "r"(bytes)
+      : "memory");
+}
+
+template <typename T, int N>
+__global__ void __launch_bounds__(128)
+    scan_step_bulk_kernel(const StepParams p) {
+  static_assert(N == 4 || N == 8 || N == 16, "whole 16-byte chunks");
+  using Lay = StepBulkLayout<T, N>;
+  constexpr int R = N / 4;  // 16-byte chunks per channel
+  constexpr int NB = kStepBulkBufs;
+  extern __shared__ __align__(128) unsigned char bulk_smem[];
+  const unsigned sbase = smem_addr(bulk_smem);
+  const unsigned bar0 = sbase + Lay::BAR;
+  const int tid = threadIdx.x;
+  const int64_t E = p.dim;
+  const int64_t e0 = (int64_t)blockIdx.x * 128;
+  const int nch = int(E - e0 < 128 ? E - e0 : 128);
+  const bool live = tid < nch;
+  const int64_t es = live ? e0 + tid : e0;
+  const int K = p.conv_state ? p.conv_width : 0;
+  constexpr int ESZ = Lay::ESZ;
+  // run sizes of one row (all multiples of 16 bytes: checked on the host)
+  const unsigned st_bytes = unsigned(nch) * N * 4;
+  const unsigned act_bytes = unsigned(nch) * ESZ;
+  const unsigned conv_bytes = unsigned(nch) * K * ESZ;
+  constexpr unsigned bc_bytes = N * ESZ;
+  const unsigned row_bytes = st_bytes + (p.z ? 3 : 2) * act_bytes +
+                             conv_bytes + 2 * bc_bytes;
+  // chunk k of this thread's row is visited at position (k - rot) mod R
+  const int rot = ((tid & 7) * R / 8) % R;
+
+  // ---- the channel's constants, in registers
+  float A2[N];
+#pragma unroll
+  for (int i = 0; i < N; ++i)
+    A2[i] = live ? fmaxf(-expf(p.A_log[es * N + i]) * kLog2e, -FLT_MAX) : 0.0f;
+  float cw[kMaxConvWidth];
+#pragma unroll
+  for (int j = 0; j < kMaxConvWidth; ++j)
+    cw[j] = (live && j < K) ? p.conv_weight[es * K + j] : 0.0f;
+  const float cbias = (live && K && p.conv_bias) ? p.conv_bias[es] : 0.0f;
+  const float dbias = (live && p.delta_bias) ? p.delta_bias[es] : 0.0f;
+  const float Dv = (live && p.D) ? p.D[es] : 0.0f;
+
+  if (tid == 0) {
+#pragma unroll
+    for (int i = 0; i < NB; ++i)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0 + 8 * i)
+                   : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  const T *gx = static_cast<const T *>(p.x_new);
+  const T *gdl = static_cast<const T *>(p.delta);
+  const T *gz = static_cast<const T *>(p.z);
+  const T *gB = static_cast<const T *>(p.B);
+  const T *gC = static_cast<const T *>(p.C);
+  T *gy = static_cast<T *>(p.y);
+  T *gconv = static_cast<T *>(p.conv_state);
+
+  // issue the copies of batch row b into buffer `buf` (thread 0)
+  auto load_row = [&](int64_t b, int buf) {
+    const unsigned d = sbase + buf * Lay::BUF;
+    const unsigned bar = bar0 + 8 * buf;
+    const int64_t ch = b * E + e0;
+    asm volatile(
+        "mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
+        "r"(row_bytes)
+        : "memory");
+    bulk_load(d + Lay::STATE, p.state + ch * N, st_bytes, bar);
+    bulk_load(d + Lay::X, gx + ch, act_bytes, bar);
+    bulk_load(d + Lay::DL, gdl + ch, act_bytes, bar);
+    if (gz) bulk_load(d + Lay::Z, gz + ch, act_bytes, bar);
+    if (K) bulk_load(d + Lay::CONV, gconv + ch * K, conv_bytes, bar);
+    bulk_load(d + Lay::BM, gB + b * N, bc_bytes, bar);
+    bulk_load(d + Lay::CM, gC + b * N, bc_bytes, bar);
+  };
+
+  const int64_t first = blockIdx.y, stride = gridDim.y;
+  const int64_t nrows = first < p.batch ? (p.batch - first + stride - 1) / stride
+                                        : 0;
+  if (tid == 0)
+    for (int64_t k = 0; k < NB - 1 && k < nrows; ++k)
+      load_row(first + k * stride, int(k));
+  int64_t k = 0;
+  bool failed = false;
+  for (; k < nrows; ++k) {
+    const int64_t b = first + k * stride;
+    const int buf = int(k % NB);
+    unsigned char *const B0 = bulk_smem + buf * Lay::BUF;
+    // the copies of row k + NB - 1 go into the buffer row k - 1 used, once
+    // the stores that read it have finished reading
+    if (tid == 0 && k + NB - 1 < nrows) {
+      asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+      load_row(b + (NB - 1) * stride, int((k + NB - 1) % NB));
+    }
+    const bool ok =
+        mbar_wait(bar0 + 8 * buf, unsigned(k / NB) & 1u, p.spin_limit);
+    if (__syncthreads_or(!ok)) {
+      failed = true;
+      break;
+    }
+
+    if (live) {
+      // ---- the channel's input, through the causal convolution
+      float xv = Act<T>::load(reinterpret_cast<const T *>(B0 + Lay::X) + tid);
+      if (K) {
+        T *cb = reinterpret_cast<T *>(B0 + Lay::CONV) + tid * K;
+        float hist[kMaxConvWidth];
+#pragma unroll
+        for (int j = 0; j < kMaxConvWidth; ++j)
+          hist[j] = j + 1 < K ? Act<T>::load(cb + j + 1) : xv;
+        float acc = cbias;
+#pragma unroll
+        for (int j = 0; j < kMaxConvWidth; ++j)
+          if (j < K) acc = fmaf(hist[j], cw[j], acc);
+        // shift left by one sample and append
+#pragma unroll
+        for (int j = 0; j < kMaxConvWidth; ++j)
+          if (j < K) Act<T>::store(cb + j, hist[j]);
+        xv = silu(acc);
+      }
+      const float v =
+          Act<T>::load(reinterpret_cast<const T *>(B0 + Lay::DL) + tid) +
+          dbias;
+      const float step = p.softplus ? softplus(v) : v;
+      const float dx = step * xv;
+      const T *Bm = reinterpret_cast<const T *>(B0 + Lay::BM);
+      const T *Cm = reinterpret_cast<const T *>(B0 + Lay::CM);
+      float *const row = reinterpret_cast<float *>(B0 + Lay::STATE) + tid * N;
+      float partial = 0.0f;
+#pragma unroll
+      for (int c = 0; c < R; ++c) {
+        const int j = R == 1 ? 0 : (c + rot) % R;  // this visit's chunk
+        const int i0 = 4 * j;
+        float Bv[4], Cv[4];
+        load4<T>(Bm + i0, Bv);
+        load4<T>(Cm + i0, Cv);
+        const float4 h4 = *reinterpret_cast<const float4 *>(row + i0);
+        float hq[4] = {h4.x, h4.y, h4.z, h4.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          // A2[i0 + i] with i0 a runtime chunk: select from the registers
+          float Ai = A2[i];
+#pragma unroll
+          for (int jj = 1; jj < R; ++jj)
+            if (j == jj) Ai = A2[4 * jj + i];
+          const float zl = step * Ai;
+          const float a = sizeof(T) == 4 ? retention_f32(zl) : ex2(zl);
+          const float wf =
+              p.write_zoh
+                  ? zoh_factor(step, zl, a, -expf(-p.A_log[es * N + i0 + i])) *
+                        xv
+                  : dx;
+          hq[i] = fmaf(a, hq[i], wf * Bv[i]);
+          partial = fmaf(Cv[i], hq[i], partial);
+        }
+        *reinterpret_cast<float4 *>(row + i0) =
+            make_float4(hq[0], hq[1], hq[2], hq[3]);
+      }
+      float out = partial + Dv * xv;
+      if (gz)
+        out *= silu(Act<T>::load(reinterpret_cast<const T *>(B0 + Lay::Z) +
+                                 tid));
+      Act<T>::store(reinterpret_cast<T *>(B0 + Lay::Y) + tid, out);
+    }
+    // this thread's shared writes become visible to the copy engine, then
+    // one thread stores the updated runs
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+    if (tid == 0) {
+      const unsigned d = sbase + buf * Lay::BUF;
+      const int64_t ch = b * E + e0;
+      bulk_store(p.state + ch * N, d + Lay::STATE, st_bytes);
+      bulk_store(gy + ch, d + Lay::Y, act_bytes);
+      if (K) bulk_store(gconv + ch * K, d + Lay::CONV, conv_bytes);
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    }
+  }
+  if (tid == 0) {
+    if (failed) {
+      atomicExch(p.status, kStepTimeout);
+      // copies still in flight (rows k .. k + NB - 1 may have been issued)
+      // land before the block's memory is released; these waits are
+      // bounded too
+      for (int64_t r = k; r < k + NB && r < nrows; ++r)
+        mbar_wait(bar0 + 8 * int(r % NB), unsigned(r / NB) & 1u,
+                  kStepDrainPolls);
+    }
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
 }
 

@@ -60,8 +60,9 @@ enum { kStatusOk = 0, kStatusTimeout = 1 };
 // Publication states (low 2 bits of a flag word; the rest is the epoch).
 enum { kFlagNone = 0, kFlagAggregate = 1, kFlagInclusive = 2 };
 
-// Test hook: the first piece of every sequence never publishes, so its
-// successor's bounded wait must run out and report kStatusTimeout.
-enum { kDebugNoPublish = 1u << 0 };
+// Test hooks: the first piece of every sequence never publishes, so its
+// successor's bounded wait must run out and report kStatusTimeout; the
+// decode step uses its per-thread-load kernel instead of the bulk-copy one.
+enum { kDebugNoPublish = 1u << 0, kDebugStepPerThread = 1u << 1 };
 
 }  // namespace ssm

@@ -82,6 +82,20 @@ using C4f2 = ssm::ChunkCfg<float,  1, 2, 8, 16, 4,  0, 64, 16>;
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
+// The handle's control block ([0] status word, [1] launch ticket), made on
+// first use on `s`.
+int ensure_ctl(ssm_scan_s *h, cudaStream_t s) {
+  if (h->ctl) return SSM_OK;
+  if (cudaMallocAsync(reinterpret_cast<void **>(&h->ctl), 256, s) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    h->ctl = nullptr;
+    return SSM_ERR_NOMEM;
+  }
+  return cudaMemsetAsync(h->ctl, 0, 256, s) == cudaSuccess ? SSM_OK
+                                                          : SSM_ERR_CUDA;
+}
+
 // Grow the split workspace for `segs` pieces; fills the ScanParams pointers.
 int ensure_workspace(ssm_scan_s *h, ssm::ScanParams &p, int64_t tiles,
                      int64_t segs, cudaStream_t s) {
@@ -89,13 +103,9 @@ int ensure_workspace(ssm_scan_s *h, ssm::ScanParams &p, int64_t tiles,
   const size_t nstate = size_t(p.batch) * segs * p.dim * p.dstate;
   const size_t off_state = align256(nflags * sizeof(unsigned));
   const size_t bytes = off_state + 3 * align256(nstate * sizeof(float));
-  if (!h->ctl) {
-    if (cudaMallocAsync(reinterpret_cast<void **>(&h->ctl), 256, s) !=
-        cudaSuccess) {
-      cudaGetLastError();
-      return SSM_ERR_NOMEM;
-    }
-    if (cudaMemsetAsync(h->ctl, 0, 256, s) != cudaSuccess) return SSM_ERR_CUDA;
+  {
+    const int rc = ensure_ctl(h, s);
+    if (rc != SSM_OK) return rc;
   }
   if (bytes > h->ws_bytes) {
     if (h->ws) cudaFreeAsync(h->ws, s);
@@ -277,6 +287,39 @@ int launch_step_cfg(const ssm::StepParams &p, bool vec, int sm_count,
   return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
+// The bulk-copy decode step (N = 4, 8 or 16): one 128-channel block per
+// state run, grid.y batch-row strides sized so every block is resident.
+template <typename T, int N>
+int launch_step_bulk(const ssm::StepParams &p, int sm_count, cudaStream_t s) {
+  const int64_t bx = (p.dim + 127) / 128;
+  if (bx > 0x7fffffff) return SSM_ERR_UNSUPPORTED;
+  auto kern = ssm::scan_step_bulk_kernel<T, N>;
+  constexpr int smem = ssm::StepBulkLayout<T, N>::BYTES;
+  static int per_sm = 0;  // resident blocks per SM
+  if (per_sm < 1) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess) {
+      cudaGetLastError();
+      return SSM_ERR_CUDA;
+    }
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 128, smem) !=
+            cudaSuccess ||
+        n < 1) {
+      cudaGetLastError();
+      n = 1;
+    }
+    per_sm = n;
+  }
+  int64_t by = int64_t(sm_count) * per_sm / bx;
+  if (by > p.batch) by = p.batch;
+  if (by > 65535) by = 65535;
+  if (by < 1) by = 1;
+  const dim3 grid{static_cast<unsigned>(bx), static_cast<unsigned>(by), 1u};
+  kern<<<grid, 128, smem, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
 // States per thread: the whole channel up to 16, else 16 per thread and 2 or
 // 4 threads per channel.
 template <typename T>
@@ -450,6 +493,31 @@ int ssm_scan_step(ssm_scan_t h, const void *x_new, void *conv_state,
   const bool vec = (dims.dstate % 4 == 0) && aligned(state, 16) &&
                    aligned(B, 4 * esz) && aligned(C, 4 * esz);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // The bulk-copy kernel: N = 4, 8 or 16 with rows of B and C at least 16
+  // bytes, channel runs of whole 16-byte chunks, every buffer 16-byte
+  // aligned and a conv buffer of at most 8 samples.
+  bool bulk = !(h->debug & ssm::kDebugStepPerThread) &&
+              (dims.dstate == 4 || dims.dstate == 8 || dims.dstate == 16) &&
+              dims.dstate * esz >= 16 && (dims.dim * esz) % 16 == 0;
+  {
+    const void *runs[] = {x_new, delta, z, B, C, y, state, conv_state};
+    for (const void *q : runs)
+      if (q && !aligned(q, 16)) bulk = false;
+  }
+  if (bulk) {
+    const int rc = ensure_ctl(h, s);
+    if (rc != SSM_OK) return rc;
+    p.status = h->ctl;
+    p.spin_limit = h->spin_limit;
+    const int n = int(dims.dstate);
+    if (dtype == SSM_F32)
+      return n == 4    ? launch_step_bulk<float, 4>(p, h->sm_count, s)
+             : n == 8 ? launch_step_bulk<float, 8>(p, h->sm_count, s)
+                      : launch_step_bulk<float, 16>(p, h->sm_count, s);
+    return n == 4    ? launch_step_bulk<__nv_bfloat16, 4>(p, h->sm_count, s)
+           : n == 8 ? launch_step_bulk<__nv_bfloat16, 8>(p, h->sm_count, s)
+                    : launch_step_bulk<__nv_bfloat16, 16>(p, h->sm_count, s);
+  }
   return dtype == SSM_F32
              ? launch_step<float>(p, vec, h->sm_count, s)
              : launch_step<__nv_bfloat16>(p, vec, h->sm_count, s);

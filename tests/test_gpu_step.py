@@ -29,12 +29,28 @@ def _host(t):
     return t.float().cpu().numpy().astype(np.float64)
 
 
+# N = 4, 8, 16 run the bulk-copy kernel unless the per-thread-load kernel is
+# asked for (debug flag 2); the other N always run the per-thread kernel.
+KERNELS = {"bulk": 0, "per_thread": 2}
+
+
+@pytest.mark.parametrize("kernel", sorted(KERNELS))
 @pytest.mark.parametrize("dtype", [W.F32, W.BF16])
 @pytest.mark.parametrize("N", [1, 3, 4, 8, 16, 32, 64])
 @pytest.mark.parametrize("conv,zoh,gate", [(4, False, True), (0, False, True),
                                            (3, True, False), (1, False, False)],
                          ids=["conv4", "noconv", "conv3_zoh", "conv1_nogate"])
-def test_step_parity(scan, dtype, N, conv, zoh, gate):
+def test_step_parity(scan, dtype, N, conv, zoh, gate, kernel):
+    if kernel == "per_thread" and N not in (4, 8, 16):
+        pytest.skip("only one kernel runs this state size")
+    S.library().ssm_scan_set_debug(scan.handle, KERNELS[kernel], 0)
+    try:
+        _step_parity(scan, dtype, N, conv, zoh, gate)
+    finally:
+        S.library().ssm_scan_set_debug(scan.handle, 0, 0)
+
+
+def _step_parity(scan, dtype, N, conv, zoh, gate):
     rng = np.random.default_rng(N * 7 + conv)
     b, E, T = 5, 40, 6
     # every channel has its own A row (A is a learned [E, N] parameter)
@@ -137,3 +153,82 @@ def test_step_argument_errors(scan):
     assert call(state=st.data_ptr() + 2) == S.SSM_ERR_ALIGN
     torch.cuda.synchronize()
     assert scan.sync_status() == S.SSM_OK
+
+
+@pytest.mark.parametrize("dtype", [W.F32, W.BF16])
+def test_step_bulk_many_rows_and_ragged_channels(scan, dtype):
+    """The bulk-copy kernel over more batch rows than resident blocks (each
+    block walks several rows through its two buffers) and a ragged last
+    block of channels (E not a multiple of 128): two tokens against the
+    oracle, and against the per-thread-load kernel (the state bit for bit;
+    y differs only in the order of the readout sum)."""
+    b, E, N = 300, 200, 16
+    wl = W.make(3, batch=b, seqlen=2, dim=E, dstate=N, dtype=dtype,
+                with_h0=True, a_jitter=0.5)
+    vals = {k: wl.values(k) for k in ("x", "delta", "z", "B", "C")}
+    A_log = torch.from_numpy(wl.dev["A_log"]).cuda()
+    D = torch.from_numpy(wl.dev["D"]).cuda()
+    bias = torch.from_numpy(wl.dev["delta_bias"]).cuda()
+    outs = {}
+    for kernel, flag in KERNELS.items():
+        S.library().ssm_scan_set_debug(scan.handle, flag, 0)
+        try:
+            state = torch.from_numpy(wl.dev["h0"].copy()).cuda()
+            state_h = wl.dev["h0"].astype(np.float64)
+            ys = []
+            for t in range(2):
+                y = scan.step(_dev(vals["x"][:, t], dtype),
+                              _dev(vals["delta"][:, t], dtype), A_log,
+                              _dev(vals["B"][:, t], dtype),
+                              _dev(vals["C"][:, t], dtype), state, D=D,
+                              z=_dev(vals["z"][:, t], dtype), delta_bias=bias)
+                torch.cuda.synchronize()
+                assert scan.sync_status() == S.SSM_OK
+                yo, state_h, _ = oracle.step(
+                    vals["x"][:, t], vals["delta"][:, t], wl.dev["A_log"],
+                    vals["B"][:, t], vals["C"][:, t], state_h, D=wl.dev["D"],
+                    z=vals["z"][:, t], delta_bias=wl.dev["delta_bias"])
+                assert_close(_host(y), yo, dtype, "%s y token %d" % (kernel, t))
+                assert_close(state.cpu().numpy(), state_h, dtype,
+                             "%s state token %d" % (kernel, t))
+                ys.append(_host(y))
+            outs[kernel] = (ys, state.cpu().numpy())
+        finally:
+            S.library().ssm_scan_set_debug(scan.handle, 0, 0)
+    for t in range(2):
+        assert rel_err(outs["bulk"][0][t], outs["per_thread"][0][t]) <= \
+            TOL[dtype]
+    assert np.array_equal(outs["bulk"][1], outs["per_thread"][1])
+
+
+def test_step_bulk_short_wait_limit_reports_and_recovers(scan):
+    """With the bounded wait cut to a single poll, a wait for a state copy
+    may give up: the call then reports SSM_ERR_TIMEOUT through the status
+    word (the block drains its copies before it exits) and the context stays
+    usable: the next call with the normal limit is correct."""
+    b, E, N = 512, 1024, 16
+    wl = W.make(3, batch=b, seqlen=1, dim=E, dstate=N, with_h0=True)
+    t = {k: (None if v is None else v) for k, v in to_device(wl).items()}
+    flat = {k: t[k][:, 0].contiguous() for k in ("x", "delta", "z", "B", "C")}
+    state = t["h0"].clone()
+    S.library().ssm_scan_set_debug(scan.handle, 0, 1)
+    try:
+        scan.step(flat["x"], flat["delta"], t["A_log"], flat["B"], flat["C"],
+                  state, D=t["D"], z=flat["z"], delta_bias=t["delta_bias"])
+        rc = scan.sync_status()
+        assert rc in (S.SSM_OK, S.SSM_ERR_TIMEOUT)
+    finally:
+        S.library().ssm_scan_set_debug(scan.handle, 0, 0)
+    assert scan.sync_status() == S.SSM_OK
+    state = t["h0"].clone()
+    y = scan.step(flat["x"], flat["delta"], t["A_log"], flat["B"], flat["C"],
+                  state, D=t["D"], z=flat["z"], delta_bias=t["delta_bias"])
+    torch.cuda.synchronize()
+    assert scan.sync_status() == S.SSM_OK
+    vals = {k: wl.values(k)[:, 0] for k in ("x", "delta", "z", "B", "C")}
+    yo, so, _ = oracle.step(vals["x"], vals["delta"], wl.dev["A_log"],
+                            vals["B"], vals["C"],
+                            wl.dev["h0"].astype(np.float64), D=wl.dev["D"],
+                            z=vals["z"], delta_bias=wl.dev["delta_bias"])
+    assert_close(_host(y), yo, wl.dtype, "y after recovery")
+    assert_close(state.cpu().numpy(), so, wl.dtype, "state after recovery")
