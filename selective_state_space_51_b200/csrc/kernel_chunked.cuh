@@ -203,11 +203,17 @@ __device__ __forceinline__ float2 transpose_reduce2(const float (&p)[2 * NG],
 
 enum { kWalkMain = 0, kWalkCorrect = 1 };
 
-template <class Cfg, bool SPLIT, bool ZOH = false, bool CONV = false>
+// FAST: the launch guarantees whole channel tiles (E a multiple of G), whole
+// windows (L a multiple of TW), a gate, the softplus step and no checkpoints,
+// so none of those is tested at run time.
+template <class Cfg, bool SPLIT, bool ZOH = false, bool CONV = false,
+          bool FAST = false>
 __global__ void __launch_bounds__(Cfg::THREADS)
 scan_chunked_kernel(const ScanParams p) {
   static_assert(!ZOH || Cfg::TB == 1,
                 "the zero-order-hold write runs with one time block");
+  static_assert(!FAST || (Cfg::TB == 1 && !SPLIT && !ZOH && !CONV),
+                "the specialised path is the plain one-time-block scan");
   static_assert(!CONV || Cfg::TB == 1,
                 "the fused convolution runs with one time block");
   using T = typename Cfg::T;
@@ -245,7 +251,7 @@ scan_chunked_kernel(const ScanParams p) {
   const int64_t tile = rem - b * tiles;
   const int64_t e0 = tile * G;
   const int64_t e = e0 + cl;
-  const bool ch_ok = e < E;
+  const bool ch_ok = FAST || e < E;
   const int64_t t_begin = SPLIT ? seg * p.seg_len : 0;
   const int64_t t_end = SPLIT ? min(L, t_begin + p.seg_len) : L;
 
@@ -255,8 +261,9 @@ scan_chunked_kernel(const ScanParams p) {
   const T *gB = static_cast<const T *>(p.B);
   const T *gC = static_cast<const T *>(p.C);
   T *gy = static_cast<T *>(p.y);
-  const bool has_z = gz != nullptr;
-  const bool store_y = gy != nullptr;
+  const bool has_z = FAST || gz != nullptr;
+  const bool store_y = FAST || gy != nullptr;
+  const bool use_softplus = FAST || p.softplus;
 
   float2 A01 = make_float2(0.0f, 0.0f), A23 = A01;  // A * log2(e)
   float2 iA01 = A01, iA23 = A01;  // 1 / A (zero-order-hold write only)
@@ -312,11 +319,14 @@ scan_chunked_kernel(const ScanParams p) {
     const int64_t t0 = w * TW;
     constexpr int CPR = Cfg::RAW_ROW / 16;  // 16-byte chunks per tile row
     constexpr int EPC = 16 / ESZ;           // elements per chunk
-    for (int idx = tid; idx < TW * CPR; idx += THREADS) {
+#pragma unroll
+    for (int it = 0; it < (TW * CPR + THREADS - 1) / THREADS; ++it) {
+      const int idx = tid + it * THREADS;
+      if ((TW * CPR) % THREADS != 0 && idx >= TW * CPR) break;
       const int r = idx / CPR, k = idx - (idx / CPR) * CPR;
       const int64_t t = t0 + r;
       const int64_t ec = e0 + k * EPC;
-      const bool ok = t < t_end && ec < E;
+      const bool ok = FAST || (t < t_end && ec < E);
       const int64_t go = ok ? (b * L + t) * E + ec : 0;
       const int so = Cfg::raw_off(r) + k * 16;
       cp_async16(base + so, gx + go, ok);
@@ -327,9 +337,12 @@ scan_chunked_kernel(const ScanParams p) {
     if constexpr (ESZ == 2) {
       // dense [TW][N] bfloat16 rows, contiguous in memory
       constexpr int CH = TW * N * 2 / 16;
-      for (int idx = tid; idx < CH; idx += THREADS) {
+#pragma unroll
+      for (int it = 0; it < (CH + THREADS - 1) / THREADS; ++it) {
+        const int idx = tid + it * THREADS;
+        if (CH % THREADS != 0 && idx >= CH) break;
         const int r = idx * 16 / (N * 2);
-        const bool ok = t0 + r < t_end;
+        const bool ok = FAST || t0 + r < t_end;
         const int64_t go = ok ? (b * L + t0) * N + (int64_t)idx * 8 : 0;
         cp_async16(bc + idx * 16, gB + go, ok);
         cp_async16(bc + Cfg::BCRAW_BYTES + idx * 16, gC + go, ok);
@@ -337,9 +350,12 @@ scan_chunked_kernel(const ScanParams p) {
     } else {
       // float rows of N*4 bytes straight into the padded float layout
       constexpr int CPRB = N * 4 / 16;
-      for (int idx = tid; idx < TW * CPRB; idx += THREADS) {
+#pragma unroll
+      for (int it = 0; it < (TW * CPRB + THREADS - 1) / THREADS; ++it) {
+        const int idx = tid + it * THREADS;
+        if ((TW * CPRB) % THREADS != 0 && idx >= TW * CPRB) break;
         const int r = idx / CPRB, k = idx - (idx / CPRB) * CPRB;
-        const bool ok = t0 + r < t_end;
+        const bool ok = FAST || t0 + r < t_end;
         const int64_t go = ok ? (b * L + t0 + r) * N + k * 4 : 0;
         const int so = Cfg::bf_off(r) + k * 16;
         cp_async16(bc + so, gB + go, ok);
@@ -391,7 +407,10 @@ scan_chunked_kernel(const ScanParams p) {
         float *fb = bf_conv;
         float *fc = reinterpret_cast<float *>(
             reinterpret_cast<unsigned char *>(bf_conv) + Cfg::BF_BYTES);
-        for (int idx = tid; idx < TW * N / 2; idx += THREADS) {
+#pragma unroll
+        for (int it = 0; it < (TW * N / 2 + THREADS - 1) / THREADS; ++it) {
+          const int idx = tid + it * THREADS;
+          if ((TW * N / 2) % THREADS != 0 && idx >= TW * N / 2) break;
           const int r = idx * 2 / N, n = idx * 2 - r * N;
           const int o = (Cfg::bf_off(r) >> 2) + n;
           *reinterpret_cast<float2 *>(fb + o) = __bfloat1622float2(rb[idx]);
@@ -416,7 +435,7 @@ scan_chunked_kernel(const ScanParams p) {
         const float dv = Act<T>::load(reinterpret_cast<const T *>(sDL + o));
         zm = has_z ? Act<T>::load(reinterpret_cast<const T *>(sZ + o)) : 0.0f;
         const float v = dv + bias;
-        float dm = p.softplus ? softplus(v) : v;
+        float dm = use_softplus ? softplus(v) : v;
         if (t0 + r >= t_end) dm = 0.0f;
         const float dxm = MODE == kWalkMain ? dm * xm : 0.0f;
         xch[slot_par * 32 + (c * TB + q) * NG + g] = make_float2(dm, dxm);
@@ -456,7 +475,8 @@ scan_chunked_kernel(const ScanParams p) {
         (void)xlo;
         (void)xhi;
         (void)xst;
-        const bool full = t0 + TW <= t_end;  // no step of the window is past
+        // no step of the window is past the end
+        const bool full = FAST || t0 + TW <= t_end;
         T *const yw = gy + ybase;
 
         // input of row r of the window; EDGE: r may be before the window
@@ -494,7 +514,7 @@ scan_chunked_kernel(const ScanParams p) {
                            Act<T>::load(reinterpret_cast<const T *>(sZ + o0)),
                            Act<T>::load(reinterpret_cast<const T *>(sZ + o1)))
                      : make_float2(0.0f, 0.0f);
-          float2 d2 = p.softplus ? PairMath<T>::softplus(v2) : v2;
+          float2 d2 = use_softplus ? PairMath<T>::softplus(v2) : v2;
           if (!full) {
             if (t0 + r0 >= t_end) d2.x = 0.0f;
             if (t0 + r0 + 1 >= t_end) d2.y = 0.0f;
@@ -533,7 +553,7 @@ scan_chunked_kernel(const ScanParams p) {
 #pragma unroll 4
         for (int jb = 0; jb < NBW; ++jb) {
           const int par = jb & 1;
-          if constexpr (!SPLIT) {
+          if constexpr (!SPLIT && !FAST) {
             // training forward: the state before every kCkptSteps-th step
             if (MODE == kWalkMain && p.ckpt && (jb * BS) % kCkptSteps == 0 &&
                 ch_ok && t0 + jb * BS < t_end) {

@@ -170,10 +170,10 @@ int64_t auto_segments(const ssm::ScanParams &p, int sm_count) {
   return segs < 2 ? 1 : segs;
 }
 
-template <class Cfg, bool SPLIT, bool ZOH, bool CONV>
+template <class Cfg, bool SPLIT, bool ZOH, bool CONV, bool FAST = false>
 int launch_kernel(const ssm::ScanParams &p, int64_t blocks, cudaStream_t s) {
   if (blocks > 0x7fffffff) return SSM_ERR_UNSUPPORTED;
-  auto kern = ssm::scan_chunked_kernel<Cfg, SPLIT, ZOH, CONV>;
+  auto kern = ssm::scan_chunked_kernel<Cfg, SPLIT, ZOH, CONV, FAST>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Cfg::SMEM_BYTES) != cudaSuccess) {
     cudaGetLastError();
@@ -199,6 +199,14 @@ int launch_chunked(ssm_scan_s *h, ssm::ScanParams &p, int64_t segs_req,
   p.segments = int(segs);
   p.seg_len = seg_len;
   h->last_segments = int(segs);
+  if constexpr (!ZOH && !CONV && Cfg::TB == 1) {
+    // whole tiles and windows, gated, softplus, no checkpoints: the
+    // specialised kernel tests none of these at run time
+    if (segs <= 1 && p.z && p.softplus && !p.ckpt && p.y &&
+        p.dim % Cfg::G == 0 && p.seqlen % Cfg::TW == 0)
+      return launch_kernel<Cfg, false, false, false, true>(
+          p, p.batch * tiles, s);
+  }
   if (segs <= 1)
     return launch_kernel<Cfg, false, ZOH, CONV>(p, p.batch * tiles, s);
   const int rc = ensure_workspace(h, p, tiles, segs, s);

@@ -305,3 +305,22 @@ def test_argument_errors(scan):
     assert call(h0=t["A_log"].data_ptr() + 1) == S.SSM_ERR_ALIGN
     torch.cuda.synchronize()
     assert scan.sync_status() == S.SSM_OK
+
+
+@pytest.mark.parametrize("idx,size", [
+    (3, dict(batch=2, seqlen=1024, dim=64)),
+    (2, dict(batch=3, seqlen=640, dim=96, dstate=8)),
+    (1, dict(batch=2, seqlen=512, dim=64)),
+    (0, dict(batch=2, seqlen=256, dim=32)),
+], ids=["bf16_n16", "bf16_n8", "f32_n16", "f32_n4"])
+@pytest.mark.parametrize("h0", [False, True], ids=["zero_state", "h0"])
+def test_whole_tiles_and_windows(scan, idx, size, h0):
+    """Shapes of whole channel tiles and whole windows with a gate and the
+    softplus step: the launch takes the specialised kernel that tests none
+    of those at run time. Per-channel A; against the oracle."""
+    wl = W.make(idx, a_jitter=0.5, with_h0=h0, **size)
+    y, h = run(scan, wl)
+    assert tuple(scan.last_variant()) == (S.SSM_VARIANT_CHUNKED, 1)
+    yo, ho = oracle.scan(**oracle_inputs(wl))
+    assert_close(y, yo, wl.dtype, "y")
+    assert_close(h, ho, wl.dtype, "h_last")
