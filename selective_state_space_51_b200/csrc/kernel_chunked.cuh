@@ -388,18 +388,36 @@ scan_chunked_kernel(const ScanParams p) {
       const int par = int((w - w_begin) & 1);
       const int wpar = par;  // window parity (selects the halo)
       (void)wpar;
-      if (w + 1 < w_end) stage(w + 1, par ^ 1);
-      cp_async_commit();
-      cp_async_wait<1>();
-      __syncthreads();
+      if constexpr (FAST) {
+        // this window's copies have landed and every thread is done with
+        // the previous window's buffer: refill it with the next window
+        cp_async_wait<0>();
+        __syncthreads();
+        if (w + 1 < w_end) stage(w + 1, par ^ 1);
+        cp_async_commit();
+      } else {
+        if (w + 1 < w_end) stage(w + 1, par ^ 1);
+        cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();
+      }
 
       const unsigned char *base = smem + par * Cfg::STAGE_BYTES;
       const unsigned char *sX = base;
       const unsigned char *sDL = base + Cfg::RAW_BYTES;
       const unsigned char *sZ = base + 2 * Cfg::RAW_BYTES;
-      const float *sB;
-      const float *sC;
-      if constexpr (ESZ == 2) {
+      const float *sB = nullptr;
+      const float *sC = nullptr;
+      // bfloat16 B and C as staged (the specialised path reads them with
+      // 8-byte loads widened in registers; the others from float copies)
+      const T *const rawB =
+          reinterpret_cast<const T *>(base + 3 * Cfg::RAW_BYTES);
+      const T *const rawC = reinterpret_cast<const T *>(
+          base + 3 * Cfg::RAW_BYTES + Cfg::BCRAW_BYTES);
+      (void)rawB;
+      (void)rawC;
+      if constexpr (ESZ == 2 && FAST) {
+      } else if constexpr (ESZ == 2) {
         const __nv_bfloat162 *rb = reinterpret_cast<const __nv_bfloat162 *>(
             base + 3 * Cfg::RAW_BYTES);
         const __nv_bfloat162 *rc = reinterpret_cast<const __nv_bfloat162 *>(
@@ -452,9 +470,14 @@ scan_chunked_kernel(const ScanParams p) {
       };
       // one step of the 4 states: a = 2^(d A'), h = a h + d x B, partial C.h
       auto bc_row = [&](int r, float4 &Bq, float4 &Cq) {
-        const int o = (Cfg::bf_off(r) >> 2) + 4 * g;
-        Bq = *reinterpret_cast<const float4 *>(sB + o);
-        Cq = *reinterpret_cast<const float4 *>(sC + o);
+        if constexpr (ESZ == 2 && FAST) {
+          Bq = Act<T>::load4(rawB + r * N + 4 * g);
+          Cq = Act<T>::load4(rawC + r * N + 4 * g);
+        } else {
+          const int o = (Cfg::bf_off(r) >> 2) + 4 * g;
+          Bq = *reinterpret_cast<const float4 *>(sB + o);
+          Cq = *reinterpret_cast<const float4 *>(sC + o);
+        }
       };
 
       if constexpr (TB == 1) {
@@ -746,7 +769,7 @@ scan_chunked_kernel(const ScanParams p) {
         const int alive = (h01.x != 0.0f) | (h01.y != 0.0f) |
                           (h23.x != 0.0f) | (h23.y != 0.0f);
         if (!__syncthreads_or(alive)) break;
-      } else {
+      } else if constexpr (!FAST) {
         __syncthreads();
       }
     }

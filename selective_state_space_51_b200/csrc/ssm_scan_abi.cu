@@ -79,6 +79,9 @@ using C8b2 = ssm::ChunkCfg<bf16,   2, 2, 8, 32, 4,  0, 16, 32>;
 using C8f2 = ssm::ChunkCfg<float,  2, 2, 8, 16, 4, 32, 64, 32>;
 using C4f1 = ssm::ChunkCfg<float,  1, 1, 1, 16, 4,  0,  0,  0>;
 using C4f2 = ssm::ChunkCfg<float,  1, 2, 8, 16, 4,  0, 64, 16>;
+// 16-channel tiles for the specialised bfloat16 path: twice the blocks, so
+// the last wave's imbalance over the SMs is about half as large
+using C16b1h = ssm::ChunkCfg<bf16, 4, 1, 4, 32, 2, 16,  0,  0>;
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
@@ -253,6 +256,11 @@ int pick(ssm_scan_s *h, ssm::ScanParams &p, int tb, int64_t segs,
 int dispatch_chunked(ssm_scan_s *h, ssm::ScanParams &p, int dtype, int tb,
                      int64_t segs, cudaStream_t s) {
   if (dtype == SSM_BF16) {
+    if (p.dstate == 16 && tb == 1 && segs <= 1 && !p.conv_weight &&
+        !p.write_zoh && p.z && p.softplus && !p.ckpt &&
+        p.dim % C16b1h::G == 0 && p.seqlen % C16b1h::TW == 0 &&
+        p.batch * (p.dim / C16b1h::G) >= 2 * int64_t(h->sm_count) * 4)
+      return launch_chunked<C16b1h>(h, p, 1, s);
     if (p.dstate == 16) return pick<C16b1, C16b2>(h, p, tb, segs, s);
     if (p.dstate == 8) return pick<C8b1, C8b2>(h, p, tb, segs, s);
     return SSM_ERR_UNSUPPORTED;

@@ -309,10 +309,11 @@ def test_argument_errors(scan):
 
 @pytest.mark.parametrize("idx,size", [
     (3, dict(batch=2, seqlen=1024, dim=64)),
+    (3, dict(batch=4, seqlen=96, dim=4736)),   # enough tiles for 16-ch ones
     (2, dict(batch=3, seqlen=640, dim=96, dstate=8)),
     (1, dict(batch=2, seqlen=512, dim=64)),
     (0, dict(batch=2, seqlen=256, dim=32)),
-], ids=["bf16_n16", "bf16_n8", "f32_n16", "f32_n4"])
+], ids=["bf16_n16", "bf16_n16_many_tiles", "bf16_n8", "f32_n16", "f32_n4"])
 @pytest.mark.parametrize("h0", [False, True], ids=["zero_state", "h0"])
 def test_whole_tiles_and_windows(scan, idx, size, h0):
     """Shapes of whole channel tiles and whole windows with a gate and the
