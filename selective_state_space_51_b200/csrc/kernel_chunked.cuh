@@ -205,15 +205,16 @@ enum { kWalkMain = 0, kWalkCorrect = 1 };
 
 // FAST: the launch guarantees whole channel tiles (E a multiple of G), whole
 // windows (L a multiple of TW), a gate, the softplus step and no checkpoints,
-// so none of those is tested at run time.
+// so none of those is tested at run time (with or without the fused
+// convolution).
 template <class Cfg, bool SPLIT, bool ZOH = false, bool CONV = false,
           bool FAST = false>
 __global__ void __launch_bounds__(Cfg::THREADS)
 scan_chunked_kernel(const ScanParams p) {
   static_assert(!ZOH || Cfg::TB == 1,
                 "the zero-order-hold write runs with one time block");
-  static_assert(!FAST || (Cfg::TB == 1 && !SPLIT && !ZOH && !CONV),
-                "the specialised path is the plain one-time-block scan");
+  static_assert(!FAST || (Cfg::TB == 1 && !SPLIT && !ZOH),
+                "the specialised path is the one-time-block, unsplit scan");
   static_assert(!CONV || Cfg::TB == 1,
                 "the fused convolution runs with one time block");
   using T = typename Cfg::T;

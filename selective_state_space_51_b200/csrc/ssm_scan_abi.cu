@@ -202,12 +202,12 @@ int launch_chunked(ssm_scan_s *h, ssm::ScanParams &p, int64_t segs_req,
   p.segments = int(segs);
   p.seg_len = seg_len;
   h->last_segments = int(segs);
-  if constexpr (!ZOH && !CONV && Cfg::TB == 1) {
+  if constexpr (!ZOH && Cfg::TB == 1) {
     // whole tiles and windows, gated, softplus, no checkpoints: the
     // specialised kernel tests none of these at run time
     if (segs <= 1 && p.z && p.softplus && !p.ckpt && p.y &&
         p.dim % Cfg::G == 0 && p.seqlen % Cfg::TW == 0)
-      return launch_kernel<Cfg, false, false, false, true>(
+      return launch_kernel<Cfg, false, false, CONV, true>(
           p, p.batch * tiles, s);
   }
   if (segs <= 1)
@@ -256,11 +256,12 @@ int pick(ssm_scan_s *h, ssm::ScanParams &p, int tb, int64_t segs,
 int dispatch_chunked(ssm_scan_s *h, ssm::ScanParams &p, int dtype, int tb,
                      int64_t segs, cudaStream_t s) {
   if (dtype == SSM_BF16) {
-    if (p.dstate == 16 && tb == 1 && segs <= 1 && !p.conv_weight &&
-        !p.write_zoh && p.z && p.softplus && !p.ckpt &&
-        p.dim % C16b1h::G == 0 && p.seqlen % C16b1h::TW == 0 &&
+    if (p.dstate == 16 && tb == 1 && segs <= 1 && !p.write_zoh && p.z &&
+        p.softplus && !p.ckpt && p.dim % C16b1h::G == 0 &&
+        p.seqlen % C16b1h::TW == 0 &&
         p.batch * (p.dim / C16b1h::G) >= 2 * int64_t(h->sm_count) * 4)
-      return launch_chunked<C16b1h>(h, p, 1, s);
+      return p.conv_weight ? launch_chunked<C16b1h, false, true>(h, p, 1, s)
+                           : launch_chunked<C16b1h>(h, p, 1, s);
     if (p.dstate == 16) return pick<C16b1, C16b2>(h, p, tb, segs, s);
     if (p.dstate == 8) return pick<C8b1, C8b2>(h, p, tb, segs, s);
     return SSM_ERR_UNSUPPORTED;

@@ -181,3 +181,21 @@ def test_conv_argument_errors(scan):
     assert call(None, 4) == S.SSM_ERR_INVALID
     assert call(w4, 4) == S.SSM_OK
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("width", [4, 2])
+@pytest.mark.parametrize("idx,size", [
+    (3, dict(batch=2, seqlen=1024, dim=64)),
+    (3, dict(batch=4, seqlen=96, dim=4736)),   # enough tiles for 16-ch ones
+    (1, dict(batch=2, seqlen=512, dim=64)),
+], ids=["bf16", "bf16_many_tiles", "f32"])
+def test_conv_whole_tiles_and_windows(scan, idx, size, width):
+    """Shapes of whole channel tiles and windows, gated, softplus: the fused
+    convolution on the specialised kernel (halo carried across windows with
+    one barrier per window). Per-channel A; against the oracle."""
+    wl = W.make(idx, a_jitter=0.5, **size)
+    w, cb = W.conv_params(wl.dim, width, seed=5 + width)
+    y, h = _run(scan, wl, w, cb)
+    yo, ho = _oracle(wl, w, cb)
+    assert_close(y, yo, wl.dtype, "y")
+    assert_close(h, ho, wl.dtype, "h_last")
