@@ -207,8 +207,12 @@ enum { kWalkMain = 0, kWalkCorrect = 1 };
 // windows (L a multiple of TW), a gate, the softplus step and no checkpoints,
 // so none of those is tested at run time (with or without the fused
 // convolution).
+// CKPT: the training forward of the backward pass. It writes the state
+// before every kCkptSteps-th step and nothing else: no readout, no gate, no
+// y, so C and z are neither staged nor read. With FAST it also needs only
+// whole tiles and windows and the softplus step.
 template <class Cfg, bool SPLIT, bool ZOH = false, bool CONV = false,
-          bool FAST = false>
+          bool FAST = false, bool CKPT = false>
 __global__ void __launch_bounds__(Cfg::THREADS)
 scan_chunked_kernel(const ScanParams p) {
   static_assert(!ZOH || Cfg::TB == 1,
@@ -217,6 +221,8 @@ scan_chunked_kernel(const ScanParams p) {
                 "the specialised path is the one-time-block, unsplit scan");
   static_assert(!CONV || Cfg::TB == 1,
                 "the fused convolution runs with one time block");
+  static_assert(!CKPT || (Cfg::TB == 1 && !SPLIT && !CONV),
+                "checkpoints are written by the unsplit one-time-block scan");
   using T = typename Cfg::T;
   constexpr int NG = Cfg::NG, TB = Cfg::TB, K = Cfg::K, TW = Cfg::TW;
   constexpr int CW = Cfg::CW, G = Cfg::G, N = Cfg::N, ESZ = Cfg::ESZ;
@@ -262,8 +268,8 @@ scan_chunked_kernel(const ScanParams p) {
   const T *gB = static_cast<const T *>(p.B);
   const T *gC = static_cast<const T *>(p.C);
   T *gy = static_cast<T *>(p.y);
-  const bool has_z = FAST || gz != nullptr;
-  const bool store_y = FAST || gy != nullptr;
+  const bool has_z = !CKPT && (FAST || gz != nullptr);
+  const bool store_y = !CKPT && (FAST || gy != nullptr);
   const bool use_softplus = FAST || p.softplus;
 
   float2 A01 = make_float2(0.0f, 0.0f), A23 = A01;  // A * log2(e)
@@ -346,7 +352,8 @@ scan_chunked_kernel(const ScanParams p) {
         const bool ok = FAST || t0 + r < t_end;
         const int64_t go = ok ? (b * L + t0) * N + (int64_t)idx * 8 : 0;
         cp_async16(bc + idx * 16, gB + go, ok);
-        cp_async16(bc + Cfg::BCRAW_BYTES + idx * 16, gC + go, ok);
+        if constexpr (!CKPT)
+          cp_async16(bc + Cfg::BCRAW_BYTES + idx * 16, gC + go, ok);
       }
     } else {
       // float rows of N*4 bytes straight into the padded float layout
@@ -360,7 +367,7 @@ scan_chunked_kernel(const ScanParams p) {
         const int64_t go = ok ? (b * L + t0 + r) * N + k * 4 : 0;
         const int so = Cfg::bf_off(r) + k * 16;
         cp_async16(bc + so, gB + go, ok);
-        cp_async16(bc + Cfg::BF_BYTES + so, gC + go, ok);
+        if constexpr (!CKPT) cp_async16(bc + Cfg::BF_BYTES + so, gC + go, ok);
       }
     }
   };
@@ -433,7 +440,8 @@ scan_chunked_kernel(const ScanParams p) {
           const int r = idx * 2 / N, n = idx * 2 - r * N;
           const int o = (Cfg::bf_off(r) >> 2) + n;
           *reinterpret_cast<float2 *>(fb + o) = __bfloat1622float2(rb[idx]);
-          *reinterpret_cast<float2 *>(fc + o) = __bfloat1622float2(rc[idx]);
+          if constexpr (!CKPT)
+            *reinterpret_cast<float2 *>(fc + o) = __bfloat1622float2(rc[idx]);
         }
         __syncthreads();
         sB = fb;
@@ -470,6 +478,16 @@ scan_chunked_kernel(const ScanParams p) {
         }
       };
       // one step of the 4 states: a = 2^(d A'), h = a h + d x B, partial C.h
+      // B alone (the checkpointing forward reads no C)
+      auto b_row = [&](int r, float4 &Bq) {
+        if constexpr (ESZ == 2 && FAST) {
+          Bq = Act<T>::load4(rawB + r * N + 4 * g);
+        } else {
+          Bq = *reinterpret_cast<const float4 *>(sB + (Cfg::bf_off(r) >> 2) +
+                                                 4 * g);
+        }
+      };
+      (void)b_row;
       auto bc_row = [&](int r, float4 &Bq, float4 &Cq) {
         if constexpr (ESZ == 2 && FAST) {
           Bq = Act<T>::load4(rawB + r * N + 4 * g);
@@ -577,10 +595,11 @@ scan_chunked_kernel(const ScanParams p) {
 #pragma unroll 4
         for (int jb = 0; jb < NBW; ++jb) {
           const int par = jb & 1;
-          if constexpr (!SPLIT && !FAST) {
+          if constexpr (!SPLIT && (!FAST || CKPT)) {
             // training forward: the state before every kCkptSteps-th step
-            if (MODE == kWalkMain && p.ckpt && (jb * BS) % kCkptSteps == 0 &&
-                ch_ok && t0 + jb * BS < t_end) {
+            if (MODE == kWalkMain && (CKPT || p.ckpt) &&
+                (jb * BS) % kCkptSteps == 0 && ch_ok &&
+                t0 + jb * BS < t_end) {
               const int64_t k = (t0 + jb * BS) / kCkptSteps;
               const int64_t nck = (L + kCkptSteps - 1) / kCkptSteps;
               *reinterpret_cast<float4 *>(
@@ -607,7 +626,10 @@ scan_chunked_kernel(const ScanParams p) {
 #pragma unroll
           for (int s = 0; s < BS; ++s) {
             float4 Bq, Cq;
-            bc_row(jb * BS + s, Bq, Cq);
+            if constexpr (CKPT)
+              b_row(jb * BS + s, Bq);
+            else
+              bc_row(jb * BS + s, Bq, Cq);
             const float2 dA = make_float2(dd[s].x, dd[s].x);
             const float2 zl01 = mul2(dA, A01), zl23 = mul2(dA, A23);
             float2 a01 = ex2x2(zl01);
@@ -633,12 +655,15 @@ scan_chunked_kernel(const ScanParams p) {
               h01 = mul2(a01, h01);
               h23 = mul2(a23, h23);
             }
-            const float2 acc =
-                fma2(make_float2(Cq.z, Cq.w), h23,
-                     mul2(make_float2(Cq.x, Cq.y), h01));
-            ps[s] = acc.x + acc.y;
+            if constexpr (!CKPT) {
+              const float2 acc =
+                  fma2(make_float2(Cq.z, Cq.w), h23,
+                       mul2(make_float2(Cq.x, Cq.y), h01));
+              ps[s] = acc.x + acc.y;
+            }
           }
-          finish2(jb, transpose_reduce2<NG, TB>(ps, g), x2, z2);
+          if constexpr (!CKPT)
+            finish2(jb, transpose_reduce2<NG, TB>(ps, g), x2, z2);
           x2 = xn;
           z2 = zn;
           e0 = n0;

@@ -173,10 +173,11 @@ int64_t auto_segments(const ssm::ScanParams &p, int sm_count) {
   return segs < 2 ? 1 : segs;
 }
 
-template <class Cfg, bool SPLIT, bool ZOH, bool CONV, bool FAST = false>
+template <class Cfg, bool SPLIT, bool ZOH, bool CONV, bool FAST = false,
+          bool CKPT = false>
 int launch_kernel(const ssm::ScanParams &p, int64_t blocks, cudaStream_t s) {
   if (blocks > 0x7fffffff) return SSM_ERR_UNSUPPORTED;
-  auto kern = ssm::scan_chunked_kernel<Cfg, SPLIT, ZOH, CONV, FAST>;
+  auto kern = ssm::scan_chunked_kernel<Cfg, SPLIT, ZOH, CONV, FAST, CKPT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Cfg::SMEM_BYTES) != cudaSuccess) {
     cudaGetLastError();
@@ -450,9 +451,19 @@ int launch_bwd(const ssm::BwdParams &p, cudaStream_t s) {
 template <class Cf, typename T, int NG>
 int run_bwd(ssm::ScanParams &fp, const ssm::BwdParams &bp, cudaStream_t s) {
   const int64_t tiles = (fp.dim + Cf::G - 1) / Cf::G;
+  const int64_t blocks = fp.batch * tiles;
+  // the checkpoint-only forward: no readout, C and z not read; with whole
+  // tiles and windows and the softplus step, the specialised instantiation
+  const bool fast = !fp.write_zoh && fp.softplus && fp.dim % Cf::G == 0 &&
+                    fp.seqlen % Cf::TW == 0;
   int rc = fp.write_zoh
-               ? launch_kernel<Cf, false, true, false>(fp, fp.batch * tiles, s)
-               : launch_kernel<Cf, false, false, false>(fp, fp.batch * tiles, s);
+               ? launch_kernel<Cf, false, true, false, false, true>(fp, blocks,
+                                                                   s)
+           : fast
+               ? launch_kernel<Cf, false, false, false, true, true>(fp, blocks,
+                                                                   s)
+               : launch_kernel<Cf, false, false, false, false, true>(fp, blocks,
+                                                                    s);
   if (rc != SSM_OK) return rc;
   return fp.write_zoh ? launch_bwd<T, NG, true>(bp, s)
                       : launch_bwd<T, NG, false>(bp, s);
