@@ -436,7 +436,11 @@ int launch_bwd(const ssm::BwdParams &p, cudaStream_t s) {
   const int64_t tiles = (p.dim + Cfg::G - 1) / Cfg::G;
   const int64_t blocks = p.batch * tiles;
   if (blocks > 0x7fffffff) return SSM_ERR_UNSUPPORTED;
-  auto kern = ssm::scan_bwd_kernel<T, NG, kBwdWarps, ZOH>;
+  // whole tiles and windows, gated, softplus: the specialised instantiation
+  const bool fast = p.dim % Cfg::G == 0 && p.seqlen % Cfg::TW == 0 && p.z &&
+                    p.softplus;
+  auto kern = fast ? ssm::scan_bwd_kernel<T, NG, kBwdWarps, ZOH, true>
+                   : ssm::scan_bwd_kernel<T, NG, kBwdWarps, ZOH, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Cfg::SMEM_BYTES) != cudaSuccess) {
     cudaGetLastError();
