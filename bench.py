@@ -80,17 +80,27 @@ CONV_WIDTH = 4
 # the timed kernel, from one ncu capture, keyed by (op, workload shape), with
 # the hash of the kernel sources that capture was taken from. A figure whose
 # sources have changed since is stale: the line then reports null.
-NCU_TRAFFIC = {("scan", 3): (1.033237248e9 + 0.314034042e9, "f8f3614b19836357")}
-KERNEL_SOURCES = ("kernel_chunked.cuh", "device_math.cuh", "scan_params.cuh",
-                  "ssm_scan_abi.cu")
+NCU_TRAFFIC = {
+    ("scan", 3): (1.029873920e9 + 0.316743168e9, "0ccbbc6f7ed60c4b"),
+    ("step", 3): (0.409515520e9 + 0.330249984e9, "b881e3539ef9b0e4"),
+}
+KERNEL_SOURCES = {
+    "scan": ("kernel_chunked.cuh", "device_math.cuh", "scan_params.cuh",
+             "ssm_scan_abi.cu"),
+    "conv": ("kernel_chunked.cuh", "device_math.cuh", "scan_params.cuh",
+             "ssm_scan_abi.cu"),
+    "step": ("kernel_step.cuh", "device_math.cuh", "ssm_scan_abi.cu"),
+    "bwd": ("kernel_bwd.cuh", "kernel_chunked.cuh", "device_math.cuh",
+            "scan_params.cuh", "ssm_scan_abi.cu"),
+}
 DECODE_BATCH = 1024
 
 
-def kernel_source_hash() -> str:
-    """sha256 (first 16 hex digits) of the forward kernel's sources."""
+def kernel_source_hash(op: str = "scan") -> str:
+    """sha256 (first 16 hex digits) of the sources of an op's kernel."""
     import hashlib
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
+    for name in KERNEL_SOURCES[op]:
         with open(os.path.join(ROOT, "selective_state_space_51_b200", "csrc",
                                name), "rb") as f:
             h.update(f.read())
@@ -103,7 +113,7 @@ def traffic_record(op: str, shape: int):
     if entry is None:
         return None, "no ncu capture of this kernel on this workload"
     value, src_hash = entry
-    now = kernel_source_hash()
+    now = kernel_source_hash(op)
     if now != src_hash:
         return None, ("ncu capture of kernel sources %s; the sources are now "
                       "%s, so the figure is stale" % (src_hash, now))

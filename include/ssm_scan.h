@@ -301,8 +301,11 @@ SSM_API int ssm_scan_sync_status(ssm_scan_t h, struct CUstream_st *stream);
  * state, inputs, conv buffers and y move as bulk copies between global and
  * shared memory; its waits for them are bounded, and one that gives up is
  * reported as SSM_ERR_TIMEOUT by ssm_scan_sync_status (the state is then
- * partly updated). Other shapes use per-thread loads. The first call on a
- * handle allocates its 256-byte status block on `stream`: make it before
+ * partly updated). The blocks of each 128-channel column take batch rows from
+ * a counter in the handle's control block, cleared on `stream` before each
+ * launch, so a handle runs one step at a time (one stream, or calls ordered
+ * between streams). Other shapes use per-thread loads. The first call on a
+ * handle allocates its 4 KiB control block on `stream`: make it before
  * capturing the step into a CUDA graph.
  */
 SSM_API int ssm_scan_step(ssm_scan_t h, const void *x_new, void *conv_state,

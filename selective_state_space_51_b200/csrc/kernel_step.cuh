@@ -46,6 +46,11 @@ struct StepParams {
   // gave up) and the polls a wait makes before giving up
   int *status;
   unsigned spin_limit;
+  // bulk-copy variant: per 128-channel column, a counter of the batch rows
+  // handed out so far (zero before the launch); blocks of a column take rows
+  // from it as they go, so the ones that run faster take more rows. nullptr:
+  // block y takes rows y, y + gridDim.y, ...
+  unsigned *row_counter;
 };
 
 // Device status written by the bulk-copy decode step (same word as the
@@ -389,23 +394,44 @@ __global__ void __launch_bounds__(128)
     bulk_load(d + Lay::CM, gC + b * N, bc_bytes, bar);
   };
 
+  // The batch row of each of this block's rows in flight, by buffer: taken
+  // from the column's counter (or the fixed stride) when its copies are
+  // issued; a row past the batch means there are no more.
+  __shared__ long long s_row[NB];
   const int64_t first = blockIdx.y, stride = gridDim.y;
-  const int64_t nrows = first < p.batch ? (p.batch - first + stride - 1) / stride
-                                        : 0;
+  unsigned *const counter =
+      p.row_counter ? p.row_counter + blockIdx.x : nullptr;
+  int64_t next_static = first;
+  auto take_row = [&]() -> int64_t {
+    if (counter) return int64_t(atomicAdd(counter, 1u));
+    const int64_t r = next_static;
+    next_static += stride;
+    return r;
+  };
   if (tid == 0)
-    for (int64_t k = 0; k < NB - 1 && k < nrows; ++k)
-      load_row(first + k * stride, int(k));
+    for (int i = 0; i < NB - 1; ++i) {
+      const int64_t r = take_row();
+      s_row[i] = r;
+      if (r < p.batch) load_row(r, i);
+    }
+  __syncthreads();
   int64_t k = 0;
   bool failed = false;
-  for (; k < nrows; ++k) {
-    const int64_t b = first + k * stride;
+  for (;; ++k) {
     const int buf = int(k % NB);
+    const int64_t b = s_row[buf];
+    if (b >= p.batch) break;  // the same value for every thread
     unsigned char *const B0 = bulk_smem + buf * Lay::BUF;
-    // the copies of row k + NB - 1 go into the buffer row k - 1 used, once
-    // the stores that read it have finished reading
-    if (tid == 0 && k + NB - 1 < nrows) {
-      asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-      load_row(b + (NB - 1) * stride, int((k + NB - 1) % NB));
+    // the copies of the row after next go into the buffer the previous row
+    // used, once the stores that read it have finished reading
+    if (tid == 0) {
+      const int nb = int((k + NB - 1) % NB);
+      const int64_t r = take_row();
+      s_row[nb] = r;
+      if (r < p.batch) {
+        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+        load_row(r, nb);
+      }
     }
     const bool ok =
         mbar_wait(bar0 + 8 * buf, unsigned(k / NB) & 1u, p.spin_limit);
@@ -496,9 +522,10 @@ __global__ void __launch_bounds__(128)
       // copies still in flight (rows k .. k + NB - 1 may have been issued)
       // land before the block's memory is released; these waits are
       // bounded too
-      for (int64_t r = k; r < k + NB && r < nrows; ++r)
-        mbar_wait(bar0 + 8 * int(r % NB), unsigned(r / NB) & 1u,
-                  kStepDrainPolls);
+      for (int64_t r = k; r < k + NB; ++r)
+        if (s_row[r % NB] < p.batch)
+          mbar_wait(bar0 + 8 * int(r % NB), unsigned(r / NB) & 1u,
+                    kStepDrainPolls);
     }
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }

@@ -25,7 +25,8 @@ struct ssm_scan_s {
   unsigned epoch = 0;
   unsigned debug = 0;
   unsigned spin_limit = kDefaultSpinLimit;
-  // control block: [0] status word, [1] launch ticket (device, 256 bytes)
+  // control block (device, kCtlBytes): [0] status word, [1] launch ticket,
+  // from [kCtlRowCounters] the decode step's per-column row counters
   int *ctl = nullptr;
   // split-sequence workspace: flags, then three state arrays
   void *ws = nullptr;
@@ -85,18 +86,25 @@ using C16b1h = ssm::ChunkCfg<bf16, 4, 1, 4, 32, 2, 16,  0,  0>;
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-// The handle's control block ([0] status word, [1] launch ticket), made on
-// first use on `s`.
+// Size of the handle's control block, and the word where the decode step's
+// row counters (one per 128-channel column) start.
+constexpr int kCtlBytes = 4096;
+constexpr int kCtlRowCounters = 4;
+constexpr int kMaxRowCounters = kCtlBytes / 4 - kCtlRowCounters;
+
+// The handle's control block ([0] status word, [1] launch ticket, then the
+// decode step's row counters), made on first use on `s`.
 int ensure_ctl(ssm_scan_s *h, cudaStream_t s) {
   if (h->ctl) return SSM_OK;
-  if (cudaMallocAsync(reinterpret_cast<void **>(&h->ctl), 256, s) !=
+  if (cudaMallocAsync(reinterpret_cast<void **>(&h->ctl), kCtlBytes, s) !=
       cudaSuccess) {
     cudaGetLastError();
     h->ctl = nullptr;
     return SSM_ERR_NOMEM;
   }
-  return cudaMemsetAsync(h->ctl, 0, 256, s) == cudaSuccess ? SSM_OK
-                                                          : SSM_ERR_CUDA;
+  return cudaMemsetAsync(h->ctl, 0, kCtlBytes, s) == cudaSuccess
+             ? SSM_OK
+             : SSM_ERR_CUDA;
 }
 
 // Grow the split workspace for `segs` pieces; fills the ScanParams pointers.
@@ -333,6 +341,14 @@ int launch_step_bulk(const ssm::StepParams &p, int sm_count, cudaStream_t s) {
   if (by > p.batch) by = p.batch;
   if (by > 65535) by = 65535;
   if (by < 1) by = 1;
+  // rows are handed out by the column's counter when there is one (cleared
+  // here, on the launch's stream), else by a fixed stride
+  if (p.row_counter &&
+      cudaMemsetAsync(p.row_counter, 0, size_t(bx) * sizeof(unsigned), s) !=
+          cudaSuccess) {
+    cudaGetLastError();
+    return SSM_ERR_CUDA;
+  }
   const dim3 grid{static_cast<unsigned>(bx), static_cast<unsigned>(by), 1u};
   kern<<<grid, 128, smem, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
@@ -541,6 +557,9 @@ int ssm_scan_step(ssm_scan_t h, const void *x_new, void *conv_state,
     if (rc != SSM_OK) return rc;
     p.status = h->ctl;
     p.spin_limit = h->spin_limit;
+    // counters run to 2^32 rows; with more columns or rows, fixed strides
+    if ((dims.dim + 127) / 128 <= kMaxRowCounters && dims.batch < (1ll << 31))
+      p.row_counter = reinterpret_cast<unsigned *>(h->ctl + kCtlRowCounters);
     const int n = int(dims.dstate);
     if (dtype == SSM_F32)
       return n == 4    ? launch_step_bulk<float, 4>(p, h->sm_count, s)
