@@ -94,8 +94,11 @@ struct BwdCfg {
 // FAST: the launch guarantees whole channel tiles (E a multiple of G), whole
 // windows (L a multiple of TW), a gate and the softplus step, so none of
 // those is tested at run time.
+// Held to 18 warps per SM (9 two-warp blocks: the shared-memory limit), so
+// that the Mamba-2.8B layer's 1280 blocks are resident in one wave.
 template <typename T, int NG, int NW, bool ZOH, bool FAST = false>
-__global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(32 * NW, 18 / NW)
+    scan_bwd_kernel(const BwdParams p) {
   using Cfg = BwdCfg<T, NG, NW>;
   constexpr int N = Cfg::N, CW = Cfg::CW, G = Cfg::G, TW = Cfg::TW;
   constexpr int THREADS = Cfg::THREADS, ESZ = Cfg::ESZ, HALF = Cfg::HALF;
@@ -207,9 +210,25 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
     }
   };
 
+  // the checkpoints that start window w's two halves, loaded one window
+  // ahead so that their latency is hidden behind a window of work
+  float4 ck_lo = make_float4(0.0f, 0.0f, 0.0f, 0.0f), ck_hi = ck_lo;
+  auto load_ckpts = [&](int64_t w) {
+    if (ch_ok) {
+      ck_lo = *reinterpret_cast<const float4 *>(
+          p.ckpt + ((b * nck + 2 * w) * E + e) * N + 4 * g);
+      // the later half may lie wholly past the sequence (no checkpoint, and
+      // its steps change nothing): start it from the first one then
+      const int64_t k2 = 2 * w + 1 < nck ? 2 * w + 1 : 2 * w;
+      ck_hi = *reinterpret_cast<const float4 *>(
+          p.ckpt + ((b * nck + k2) * E + e) * N + 4 * g);
+    }
+  };
+
   const int64_t w_last = nwin - 1;
   stage(w_last, 0);
   cp_async_commit();
+  load_ckpts(w_last);
   for (int64_t w = w_last; w >= 0; --w) {
     const int par = int((w_last - w) & 1);
     // this window's tiles have landed, and every thread is done with the
@@ -272,18 +291,10 @@ __global__ void __launch_bounds__(32 * NW) scan_bwd_kernel(const BwdParams p) {
     // window (one checkpoint interval) at a time, the later half first: the
     // state history of the half being reversed is kept in shared memory.
     // Both halves start from a stored state, so each step is recomputed once.
-    float hck[4] = {}, hmid[4] = {};
-    if (ch_ok) {
-      const float4 v = *reinterpret_cast<const float4 *>(
-          p.ckpt + ((b * nck + 2 * w) * E + e) * N + 4 * g);
-      hck[0] = v.x; hck[1] = v.y; hck[2] = v.z; hck[3] = v.w;
-      // the later half may lie wholly past the sequence (no checkpoint, and
-      // its steps change nothing): start it from the first one then
-      const int64_t k2 = 2 * w + 1 < nck ? 2 * w + 1 : 2 * w;
-      const float4 u = *reinterpret_cast<const float4 *>(
-          p.ckpt + ((b * nck + k2) * E + e) * N + 4 * g);
-      hmid[0] = u.x; hmid[1] = u.y; hmid[2] = u.z; hmid[3] = u.w;
-    }
+    // (this window's checkpoints were loaded during the previous window)
+    const float hck[4] = {ck_lo.x, ck_lo.y, ck_lo.z, ck_lo.w};
+    const float hmid[4] = {ck_hi.x, ck_hi.y, ck_hi.z, ck_hi.w};
+    if (w > 0) load_ckpts(w - 1);
     // advance h over rows [r0, r0 + HALF); STORE: keep each state in sH
     // (row 1 + r - r0)
     auto recompute = [&](float (&h)[4], int r0, bool store) {
