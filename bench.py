@@ -8,7 +8,7 @@ SiLU gate, y and h_last stores). Default workload: the Mamba-2.8B-shaped layer
 seeded inputs (selective_state_space_51_b200.workloads, shape 3).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--shape I]
-                    [--impl reference] [--op scan|conv|step]
+                    [--impl reference] [--op scan|conv|step|bwd|train]
 
 Prints ONE JSON line (rank 0). Multi-GPU runs are launched by torchrun with
 one process per GPU; each rank scans its own batch of sequences (weak
@@ -21,7 +21,10 @@ T_roof = max(bytes / HBM peak, exps / SFU peak), fraction = T_roof / T.
 
 `--op bwd` times the backward pass (ssm_scan_bwd: a forward that writes a
 state checkpoint every 8 steps, then the reverse sweep) on the same
-workload. Two more operations print a line of the same form: `--op conv` times the scan
+workload, and `--op train` a training step (ssm_scan_fwd with
+SSM_SAVE_CHECKPOINTS, whose forward keeps those checkpoints, then
+ssm_scan_bwd with SSM_REUSE_CHECKPOINTS, the reverse sweep alone). Two more
+operations print a line of the same form: `--op conv` times the scan
 with the causal depthwise convolution (width 4) + SiLU fused in front
 (ssm_scan_fwd_conv, same workload and roofline), and `--op step` times one
 batched decode step (ssm_scan_step: conv buffer shift, conv + SiLU, state
@@ -92,6 +95,8 @@ KERNEL_SOURCES = {
     "step": ("kernel_step.cuh", "device_math.cuh", "ssm_scan_abi.cu"),
     "bwd": ("kernel_bwd.cuh", "kernel_chunked.cuh", "device_math.cuh",
             "scan_params.cuh", "ssm_scan_abi.cu"),
+    "train": ("kernel_bwd.cuh", "kernel_chunked.cuh", "device_math.cuh",
+              "scan_params.cuh", "ssm_scan_abi.cu"),
 }
 DECODE_BATCH = 1024
 
@@ -130,6 +135,9 @@ def workload_config(wl, op: str, world: int, shape: int) -> dict:
             CONV_WIDTH)
     elif op == "bwd":
         name += "; backward"
+    elif op == "train":
+        name += ("; training step: forward keeping its checkpoints + "
+                 "backward from them")
     elif op == "step":
         name = ("decode step, Mamba-2.8B layer shape: %d sequences x E=%d x "
                 "N=%d float32 state, conv width %d, %s activations" % (
@@ -459,6 +467,39 @@ class BwdOp:
         return tuple(v for v in self.grads.values() if v is not None)
 
 
+class TrainOp(BwdOp):
+    """One training step per step: the forward that keeps the backward's
+    state checkpoints (y and h_last out), then the backward that starts from
+    them (its reverse sweep alone)."""
+
+    def __init__(self, args, plan, dev, scan):
+        import torch
+        from selective_state_space_51_b200 import workloads as W
+        super().__init__(args, plan, dev, scan)
+        self.name = "train"
+        self.launches_per_step = 2   # forward with checkpoints, reverse sweep
+        wl = self.wl
+        self.y = torch.empty_like(self.t["x"])
+        self.h_last = torch.empty((wl.batch, wl.dim, wl.dstate),
+                                  dtype=torch.float32, device=dev)
+        self.nbytes += algorithmic_bytes(wl, "scan")
+        self.workload = W.shape_description(args.shape) + (
+            "; training step: forward keeping its checkpoints + backward "
+            "from them")
+
+    def run(self, t, stream):
+        self.scan(t["x"], t["delta"], t["A_log"], t["B"], t["C"], D=t["D"],
+                  z=t["z"], delta_bias=t["delta_bias"], h0=t["h0"], y=self.y,
+                  h_last=self.h_last, stream=stream, save_checkpoints=True)
+        self.grads = self.scan.backward(
+            t["x"], t["delta"], t["A_log"], t["B"], t["C"], t["dy"],
+            D=t["D"], z=t["z"], delta_bias=t["delta_bias"], h0=t["h0"],
+            stream=stream, reuse_checkpoints=True)
+
+    def outputs(self):
+        return (self.y, self.h_last) + super().outputs()
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -478,7 +519,8 @@ def run_gpu(args):
 
     plan = shard_for_rank(rank, world, args.shape)
     scan = S.SelectiveScan(local)
-    op = {"step": StepOp, "bwd": BwdOp}.get(args.op, ScanOp)(args, plan, dev,
+    op = {"step": StepOp, "bwd": BwdOp, "train": TrainOp}.get(
+        args.op, ScanOp)(args, plan, dev,
                                                               scan)
     t = op.t
     stream = torch.cuda.current_stream(dev)
@@ -661,11 +703,13 @@ def _finish(args, op, world, rank, local, dev, dist, scan, clocks, total_ms,
             line["roofline"]["frac_of_measured_ex2"] = achieved_exp / rate
         except Exception as exc:  # reported, never fatal to the bench line
             line["roofline"]["ex2_measured_error"] = str(exc)[:200]
-    if op.name == "bwd":
+    if op.name in ("bwd", "train"):
         line["roofline"]["peak_note"] += (
-            "; one retention exp per element counted (the pass evaluates "
-            "about 3.3: one each in the checkpointing forward, the recompute "
-            "and the reverse sweep, plus the pre-pass slopes per (t, e))")
+            "; one retention exp per element counted (the %s evaluates "
+            "about 3.3: one each in the %sforward, the recompute and the "
+            "reverse sweep, plus the softplus and gate per (t, e))" % (
+                ("pass", "checkpointing ") if op.name == "bwd"
+                else ("step", "")))
     if op.name != "step":
         line["roofline_min_hbm_sfu"] = {
             "t_hbm_us": t_hbm * 1e6, "t_sfu_us_at_max_clock": t_sfu * 1e6,
@@ -674,7 +718,7 @@ def _finish(args, op, world, rank, local, dev, dist, scan, clocks, total_ms,
             "hbm_peak_gbs": peaks["hbm_gbs"], "hbm_source": peaks["source"],
             "frac_at_8tbs_hbm": max(nbytes / (HBM_NOMINAL_GBS * 1e9), t_sfu)
             / (kernel_ms * 1e-3)}
-        if op.name != "bwd":
+        if op.name not in ("bwd", "train"):
             line["kernel"] = {"variant": variant[0], "segments": variant[1]}
     if (rank == 0 and world == 1 and not args.no_cpu_baseline
             and op.name == "scan"):
@@ -696,11 +740,12 @@ def main(argv=None):
     ap.add_argument("--shape", type=int, default=3,
                     help="workload shape index (default 3: Mamba-2.8B layer)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--op", choices=["scan", "conv", "step", "bwd"],
+    ap.add_argument("--op", choices=["scan", "conv", "step", "bwd", "train"],
                     default="scan",
                     help="scan (default), the scan with the fused "
-                         "convolution, the batched decode step, or the "
-                         "backward pass")
+                         "convolution, the batched decode step, the "
+                         "backward pass, or a training step (forward "
+                         "keeping checkpoints + backward from them)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--reference-seconds", type=float, default=10.0,
                     help="CPU seconds of the oracle sample in cpu_baseline")

@@ -97,6 +97,32 @@ enum { SSM_F32 = 0, SSM_BF16 = 1 };
  */
 enum { SSM_DELTA_SOFTPLUS = 1u << 0, SSM_WRITE_ZOH = 1u << 1 };
 
+/*
+ * Training pair (the states are still recomputed on the way back, as section
+ * "Compose the updates instead of waiting for every state" of the abhik page
+ * describes; only the sparse checkpoints the backward starts from are kept):
+ *   SSM_SAVE_CHECKPOINTS (ssm_scan_fwd only): the forward also writes the
+ *     state before every 8th step into the handle's checkpoint workspace,
+ *     which it grows on first use (b * ceil(L / 8) * dim * dstate floats;
+ *     SSM_ERR_NOMEM if it cannot: make that call before capturing a graph).
+ *     The call then runs unsplit (one block per sequence and channel tile),
+ *     needs the chunked variant's shapes (dstate 4, 8 or 16, 8 or 16 for
+ *     bfloat16; dim * element size a multiple of 16 bytes; 16-byte aligned
+ *     x, delta, z, B, C: SSM_ERR_UNSUPPORTED otherwise) and does not combine
+ *     with ssm_scan_fwd_conv (SSM_ERR_INVALID). The handle remembers the
+ *     shape, dtype and flags the checkpoints belong to.
+ *   SSM_REUSE_CHECKPOINTS (ssm_scan_bwd only): skip the backward's own
+ *     checkpointing forward and start from the checkpoints the last
+ *     SSM_SAVE_CHECKPOINTS forward on this handle wrote. Its shape, dtype and
+ *     SSM_DELTA_SOFTPLUS / SSM_WRITE_ZOH flags must match this call's
+ *     (SSM_ERR_INVALID otherwise, also when there are none, or when a
+ *     backward without this flag has overwritten them since); its inputs
+ *     (x, delta, A_log, B, h0, delta_bias) must be this call's, which the
+ *     library cannot check. The gradients are the ones the same call without
+ *     the flag returns.
+ */
+enum { SSM_SAVE_CHECKPOINTS = 1u << 2, SSM_REUSE_CHECKPOINTS = 1u << 3 };
+
 /* Status codes. */
 enum {
     SSM_OK = 0,
@@ -194,7 +220,8 @@ SSM_API int ssm_scan_fwd_conv(ssm_scan_t h, const void *v,
  * waiting for every state" describes). Two launches on `stream`: the forward
  * with a state checkpoint every 8 steps into a workspace the handle grows
  * (b * ceil(L / 8) * dim * dstate floats; SSM_ERR_NOMEM if it cannot), then
- * a reverse sweep from those checkpoints.
+ * a reverse sweep from those checkpoints. With SSM_REUSE_CHECKPOINTS (see
+ * above), only the reverse sweep, from the training forward's checkpoints.
  *   inputs     : as ssm_scan_fwd (x, delta, A_log, B, C, D, z, delta_bias,
  *                flags, h0); dy [batch, seqlen, dim] activation dtype,
  *                required; dh_last [batch, dim, dstate] float32 or NULL (0).

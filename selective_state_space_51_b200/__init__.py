@@ -17,6 +17,11 @@ importing works but the first call raises: there is no fallback path.
     # gradients of sum(dy * y) + sum(dh_last * h_last)
     grads = scan.backward(x, delta, A_log, B, C, dy, D=D, z=z,
                           delta_bias=bias)
+    # a training step: the forward keeps the backward's checkpoints
+    y, h_last = scan(x, delta, A_log, B, C, D=D, z=z, delta_bias=bias,
+                     save_checkpoints=True)
+    grads = scan.backward(x, delta, A_log, B, C, dy, D=D, z=z,
+                          delta_bias=bias, reuse_checkpoints=True)
 """
 from __future__ import annotations
 
@@ -31,6 +36,8 @@ SSM_F32 = 0
 SSM_BF16 = 1
 SSM_DELTA_SOFTPLUS = 1
 SSM_WRITE_ZOH = 2
+SSM_SAVE_CHECKPOINTS = 4
+SSM_REUSE_CHECKPOINTS = 8
 
 SSM_OK = 0
 SSM_ERR_INVALID = -1
@@ -295,11 +302,13 @@ class SelectiveScan:
 
     def backward(self, x, delta, A_log, B, C, dy, D=None, z=None,
                  delta_bias=None, delta_softplus=True, h0=None, dh_last=None,
-                 write_zoh=False, stream=None):
+                 write_zoh=False, stream=None, reuse_checkpoints=False):
         """Gradients of sum(dy * y) + sum(dh_last * h_last) for the scan of
         these inputs. Returns a dict: dx, ddelta, dz (activation dtype; dz
         None without z), dB, dC, dA_log, dD, ddelta_bias, dh0 (float32; dD /
-        ddelta_bias None without D / delta_bias)."""
+        ddelta_bias None without D / delta_bias). reuse_checkpoints: start
+        from the checkpoints of this handle's last forward called with
+        save_checkpoints=True on these same inputs."""
         import torch
         if x.dtype == torch.float32:
             dtype = SSM_F32
@@ -322,7 +331,8 @@ class SelectiveScan:
         if stream is None:
             stream = torch.cuda.current_stream(self.device)
         flags = (SSM_DELTA_SOFTPLUS if delta_softplus else 0) | \
-            (SSM_WRITE_ZOH if write_zoh else 0)
+            (SSM_WRITE_ZOH if write_zoh else 0) | \
+            (SSM_REUSE_CHECKPOINTS if reuse_checkpoints else 0)
         ssm_scan_bwd(self.handle, x, delta, A_log, B, C, D, z, delta_bias,
                      flags, h0, dy, dh_last, g["dx"], g["ddelta"], g["dA_log"],
                      g["dB"], g["dC"], g["dD"], g["dz"], g["ddelta_bias"],
@@ -354,9 +364,11 @@ class SelectiveScan:
     def __call__(self, x, delta, A_log, B, C, D=None, z=None, delta_bias=None,
                  delta_softplus=True, h0=None, y=None, h_last=None,
                  return_last_state=True, stream=None, write_zoh=False,
-                 conv_weight=None, conv_bias=None):
+                 conv_weight=None, conv_bias=None, save_checkpoints=False):
         """The forward scan. With conv_weight ([E, K] float32) x is the input
-        of the causal depthwise convolution + SiLU fused in front."""
+        of the causal depthwise convolution + SiLU fused in front. With
+        save_checkpoints the handle keeps the state checkpoints a following
+        backward(..., reuse_checkpoints=True) starts from."""
         import torch
         if x.dtype == torch.float32:
             dtype = SSM_F32
@@ -389,7 +401,8 @@ class SelectiveScan:
         if stream is None:
             stream = torch.cuda.current_stream(self.device)
         flags = (SSM_DELTA_SOFTPLUS if delta_softplus else 0) | \
-            (SSM_WRITE_ZOH if write_zoh else 0)
+            (SSM_WRITE_ZOH if write_zoh else 0) | \
+            (SSM_SAVE_CHECKPOINTS if save_checkpoints else 0)
         if conv_weight is not None:
             ssm_scan_fwd_conv(self.handle, x, conv_weight, conv_bias,
                               conv_weight.shape[-1], delta, A_log, B, C, D, z,

@@ -211,8 +211,10 @@ enum { kWalkMain = 0, kWalkCorrect = 1 };
 // before every kCkptSteps-th step and nothing else: no readout, no gate, no
 // y, so C and z are neither staged nor read. With FAST it also needs only
 // whole tiles and windows and the softplus step.
+// SAVE: the specialised path's forward that also writes those checkpoints
+// (y and all), for a backward that reuses them.
 template <class Cfg, bool SPLIT, bool ZOH = false, bool CONV = false,
-          bool FAST = false, bool CKPT = false>
+          bool FAST = false, bool CKPT = false, bool SAVE = false>
 __global__ void __launch_bounds__(Cfg::THREADS)
 scan_chunked_kernel(const ScanParams p) {
   static_assert(!ZOH || Cfg::TB == 1,
@@ -223,6 +225,8 @@ scan_chunked_kernel(const ScanParams p) {
                 "the fused convolution runs with one time block");
   static_assert(!CKPT || (Cfg::TB == 1 && !SPLIT && !CONV),
                 "checkpoints are written by the unsplit one-time-block scan");
+  static_assert(!SAVE || (FAST && !CKPT && !CONV),
+                "SAVE is the specialised forward that keeps its checkpoints");
   using T = typename Cfg::T;
   constexpr int NG = Cfg::NG, TB = Cfg::TB, K = Cfg::K, TW = Cfg::TW;
   constexpr int CW = Cfg::CW, G = Cfg::G, N = Cfg::N, ESZ = Cfg::ESZ;
@@ -595,9 +599,9 @@ scan_chunked_kernel(const ScanParams p) {
 #pragma unroll 4
         for (int jb = 0; jb < NBW; ++jb) {
           const int par = jb & 1;
-          if constexpr (!SPLIT && (!FAST || CKPT)) {
+          if constexpr (!SPLIT && (!FAST || CKPT || SAVE)) {
             // training forward: the state before every kCkptSteps-th step
-            if (MODE == kWalkMain && (CKPT || p.ckpt) &&
+            if (MODE == kWalkMain && (CKPT || SAVE || p.ckpt) &&
                 (jb * BS) % kCkptSteps == 0 && ch_ok &&
                 t0 + jb * BS < t_end) {
               const int64_t k = (t0 + jb * BS) / kCkptSteps;

@@ -34,6 +34,12 @@ struct ssm_scan_s {
   // backward: the forward's state checkpoints
   float *ckpt = nullptr;
   size_t ckpt_bytes = 0;
+  // what ckpt holds, when ckpt_saved: the checkpoints of the last forward
+  // with SSM_SAVE_CHECKPOINTS, for this shape, dtype and flags
+  bool ckpt_saved = false;
+  ssm_scan_dims ckpt_dims{};
+  int ckpt_dtype = 0;
+  uint32_t ckpt_flags = 0;
 };
 
 namespace {
@@ -91,6 +97,31 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 constexpr int kCtlBytes = 4096;
 constexpr int kCtlRowCounters = 4;
 constexpr int kMaxRowCounters = kCtlBytes / 4 - kCtlRowCounters;
+
+// The checkpoint workspace, grown on `s` to at least `need` bytes.
+int ensure_ckpt(ssm_scan_s *h, size_t need, cudaStream_t s) {
+  if (need <= h->ckpt_bytes) return SSM_OK;
+  if (h->ckpt) cudaFreeAsync(h->ckpt, s);
+  h->ckpt = nullptr;
+  h->ckpt_bytes = 0;
+  h->ckpt_saved = false;
+  if (cudaMallocAsync(reinterpret_cast<void **>(&h->ckpt), need, s) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return SSM_ERR_NOMEM;
+  }
+  h->ckpt_bytes = need;
+  return SSM_OK;
+}
+
+// Checkpoint floats of a (batch, seqlen, dim, dstate) scan: one state every
+// kCkptSteps steps; false on overflow.
+bool ckpt_floats(const ssm_scan_dims &d, int64_t *out) {
+  int64_t bd = 0, st = 0;
+  const int64_t nck = (d.seqlen + ssm::kCkptSteps - 1) / ssm::kCkptSteps;
+  return mul_ok(d.batch, d.dim, &bd) && mul_ok(bd, d.dstate, &st) &&
+         mul_ok(st, nck, out) && *out <= (int64_t(1) << 56);
+}
 
 // The handle's control block ([0] status word, [1] launch ticket, then the
 // decode step's row counters), made on first use on `s`.
@@ -182,10 +213,10 @@ int64_t auto_segments(const ssm::ScanParams &p, int sm_count) {
 }
 
 template <class Cfg, bool SPLIT, bool ZOH, bool CONV, bool FAST = false,
-          bool CKPT = false>
+          bool CKPT = false, bool SAVE = false>
 int launch_kernel(const ssm::ScanParams &p, int64_t blocks, cudaStream_t s) {
   if (blocks > 0x7fffffff) return SSM_ERR_UNSUPPORTED;
-  auto kern = ssm::scan_chunked_kernel<Cfg, SPLIT, ZOH, CONV, FAST, CKPT>;
+  auto kern = ssm::scan_chunked_kernel<Cfg, SPLIT, ZOH, CONV, FAST, CKPT, SAVE>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Cfg::SMEM_BYTES) != cudaSuccess) {
     cudaGetLastError();
@@ -278,6 +309,41 @@ int dispatch_chunked(ssm_scan_s *h, ssm::ScanParams &p, int dtype, int tb,
   if (p.dstate == 16) return pick<C16f1, C16f2>(h, p, tb, segs, s);
   if (p.dstate == 8) return pick<C8f1, C8f2>(h, p, tb, segs, s);
   if (p.dstate == 4) return pick<C4f1, C4f2>(h, p, tb, segs, s);
+  return SSM_ERR_UNSUPPORTED;
+}
+
+// The forward with SSM_SAVE_CHECKPOINTS: unsplit, one time block, the
+// checkpoints written into p.ckpt; the specialised instantiation where the
+// scan path would take it.
+template <class Cfg>
+int launch_save(ssm_scan_s *h, ssm::ScanParams &p, cudaStream_t s) {
+  const int64_t blocks = p.batch * ((p.dim + Cfg::G - 1) / Cfg::G);
+  p.segments = 1;
+  p.seg_len = p.seqlen;
+  h->last_segments = 1;
+  if (p.write_zoh) return launch_kernel<Cfg, false, true, false>(p, blocks, s);
+  if (p.z && p.softplus && p.y && p.dim % Cfg::G == 0 &&
+      p.seqlen % Cfg::TW == 0)
+    return launch_kernel<Cfg, false, false, false, true, false, true>(
+        p, blocks, s);
+  return launch_kernel<Cfg, false, false, false>(p, blocks, s);
+}
+
+int dispatch_save(ssm_scan_s *h, ssm::ScanParams &p, int dtype,
+                  cudaStream_t s) {
+  if (dtype == SSM_BF16) {
+    if (p.dstate == 16) {
+      if (p.dim % C16b1h::G == 0 && p.seqlen % C16b1h::TW == 0 &&
+          p.batch * (p.dim / C16b1h::G) >= 2 * int64_t(h->sm_count) * 4)
+        return launch_save<C16b1h>(h, p, s);
+      return launch_save<C16b1>(h, p, s);
+    }
+    if (p.dstate == 8) return launch_save<C8b1>(h, p, s);
+    return SSM_ERR_UNSUPPORTED;
+  }
+  if (p.dstate == 16) return launch_save<C16f1>(h, p, s);
+  if (p.dstate == 8) return launch_save<C8f1>(h, p, s);
+  if (p.dstate == 4) return launch_save<C4f1>(h, p, s);
   return SSM_ERR_UNSUPPORTED;
 }
 
@@ -377,7 +443,8 @@ int scan_fwd(ssm_scan_s *h, const void *x, const float *conv_weight,
   if (!h || !x || !delta || !A_log || !B || !C || !y) return SSM_ERR_INVALID;
   if (dims.batch <= 0 || dims.seqlen <= 0 || dims.dim <= 0 || dims.dstate <= 0)
     return SSM_ERR_INVALID;
-  if (flags & ~uint32_t(SSM_DELTA_SOFTPLUS | SSM_WRITE_ZOH))
+  if (flags & ~uint32_t(SSM_DELTA_SOFTPLUS | SSM_WRITE_ZOH |
+                        (conv_weight ? 0u : unsigned(SSM_SAVE_CHECKPOINTS))))
     return SSM_ERR_INVALID;
   if (conv_weight &&
       (conv_width < 1 || conv_width > ssm::kScanConvMaxWidth))
@@ -418,8 +485,28 @@ int scan_fwd(ssm_scan_s *h, const void *x, const float *conv_weight,
   p.conv_width = conv_weight ? conv_width : 0;
   p.segments = 1;
 
-  int variant = h->variant;
   const bool chunk_ok = chunked_supported(p, dtype);
+  if (flags & SSM_SAVE_CHECKPOINTS) {
+    // the training forward: unsplit chunked scan, checkpoints kept
+    if (!chunk_ok || h->variant == SSM_VARIANT_SEQUENTIAL ||
+        h->time_blocks > 1)
+      return SSM_ERR_UNSUPPORTED;
+    int64_t ck = 0;
+    if (!ckpt_floats(dims, &ck)) return SSM_ERR_INVALID;
+    int rc = ensure_ckpt(h, size_t(ck) * sizeof(float), s);
+    if (rc != SSM_OK) return rc;
+    h->ckpt_saved = false;
+    p.ckpt = h->ckpt;
+    rc = dispatch_save(h, p, dtype, s);
+    if (rc != SSM_OK) return rc;
+    h->ckpt_saved = true;
+    h->ckpt_dims = dims;
+    h->ckpt_dtype = dtype;
+    h->ckpt_flags = flags & (SSM_DELTA_SOFTPLUS | SSM_WRITE_ZOH);
+    h->last_variant = SSM_VARIANT_CHUNKED;
+    return SSM_OK;
+  }
+  int variant = h->variant;
   if (variant == SSM_VARIANT_AUTO)
     variant = chunk_ok ? SSM_VARIANT_CHUNKED : SSM_VARIANT_SEQUENTIAL;
   int rc;
@@ -467,9 +554,15 @@ int launch_bwd(const ssm::BwdParams &p, cudaStream_t s) {
 }
 
 // The training forward (checkpoints, no y) and the reverse sweep for one
-// (forward config, activation type, states per lane).
+// (forward config, activation type, states per lane); with `reuse`, the
+// reverse sweep alone, from the checkpoints a SSM_SAVE_CHECKPOINTS forward
+// left.
 template <class Cf, typename T, int NG>
-int run_bwd(ssm::ScanParams &fp, const ssm::BwdParams &bp, cudaStream_t s) {
+int run_bwd(ssm::ScanParams &fp, const ssm::BwdParams &bp, bool reuse,
+            cudaStream_t s) {
+  if (reuse)  // the training forward left the checkpoints
+    return fp.write_zoh ? launch_bwd<T, NG, true>(bp, s)
+                        : launch_bwd<T, NG, false>(bp, s);
   const int64_t tiles = (fp.dim + Cf::G - 1) / Cf::G;
   const int64_t blocks = fp.batch * tiles;
   // the checkpoint-only forward: no readout, C and z not read; with whole
@@ -727,8 +820,11 @@ int ssm_scan_bwd(ssm_scan_t h, const void *x, const void *delta,
     return SSM_ERR_INVALID;
   if (dims.batch <= 0 || dims.seqlen <= 0 || dims.dim <= 0 || dims.dstate <= 0)
     return SSM_ERR_INVALID;
-  if (flags & ~uint32_t(SSM_DELTA_SOFTPLUS | SSM_WRITE_ZOH))
+  if (flags & ~uint32_t(SSM_DELTA_SOFTPLUS | SSM_WRITE_ZOH |
+                        SSM_REUSE_CHECKPOINTS))
     return SSM_ERR_INVALID;
+  const bool reuse = (flags & SSM_REUSE_CHECKPOINTS) != 0;
+  flags &= ~uint32_t(SSM_REUSE_CHECKPOINTS);
   if (dtype != SSM_F32 && dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
   const int64_t N = dims.dstate;
   const size_t esz = dtype == SSM_F32 ? 4 : 2;
@@ -762,19 +858,19 @@ int ssm_scan_bwd(ssm_scan_t h, const void *x, const void *delta,
   if (cur != h->device) return SSM_ERR_INVALID;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
-  // ---- checkpoint workspace, and the summed outputs cleared
-  const size_t need = size_t(ck) * sizeof(float);
-  if (need > h->ckpt_bytes) {
-    if (h->ckpt) cudaFreeAsync(h->ckpt, s);
-    h->ckpt = nullptr;
-    h->ckpt_bytes = 0;
-    if (cudaMallocAsync(reinterpret_cast<void **>(&h->ckpt), need, s) !=
-        cudaSuccess) {
-      cudaGetLastError();
-      return SSM_ERR_NOMEM;
-    }
-    h->ckpt_bytes = need;
+  // ---- checkpoints: the training forward's, or a workspace for our own
+  if (reuse) {
+    const ssm_scan_dims &k = h->ckpt_dims;
+    if (!h->ckpt_saved || k.batch != dims.batch || k.seqlen != dims.seqlen ||
+        k.dim != dims.dim || k.dstate != dims.dstate ||
+        h->ckpt_dtype != dtype || h->ckpt_flags != flags)
+      return SSM_ERR_INVALID;
+  } else {
+    const int rc = ensure_ckpt(h, size_t(ck) * sizeof(float), s);
+    if (rc != SSM_OK) return rc;
+    h->ckpt_saved = false;  // this call's forward overwrites them
   }
+  // ---- the summed outputs cleared
   const size_t bcn = size_t(rows) * N * sizeof(float);
   if (cudaMemsetAsync(dB, 0, bcn, s) != cudaSuccess ||
       cudaMemsetAsync(dC, 0, bcn, s) != cudaSuccess ||
@@ -809,12 +905,12 @@ int ssm_scan_bwd(ssm_scan_t h, const void *x, const void *delta,
   bp.dstate = int(N); bp.softplus = fp.softplus;
 
   if (dtype == SSM_BF16) {
-    if (N == 16) return run_bwd<C16b1, __nv_bfloat16, 4>(fp, bp, s);
-    return run_bwd<C8b1, __nv_bfloat16, 2>(fp, bp, s);
+    if (N == 16) return run_bwd<C16b1, __nv_bfloat16, 4>(fp, bp, reuse, s);
+    return run_bwd<C8b1, __nv_bfloat16, 2>(fp, bp, reuse, s);
   }
-  if (N == 16) return run_bwd<C16f1, float, 4>(fp, bp, s);
-  if (N == 8) return run_bwd<C8f1, float, 2>(fp, bp, s);
-  return run_bwd<C4f1, float, 1>(fp, bp, s);
+  if (N == 16) return run_bwd<C16f1, float, 4>(fp, bp, reuse, s);
+  if (N == 8) return run_bwd<C8f1, float, 2>(fp, bp, reuse, s);
+  return run_bwd<C4f1, float, 1>(fp, bp, reuse, s);
 }
 
 }  // extern "C"
