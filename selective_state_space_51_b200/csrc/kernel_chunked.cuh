@@ -64,6 +64,12 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem,
                "l"(gmem), "r"(src_size)
                : "memory");
 }
+__device__ __forceinline__ void cp_async8(void *smem, const void *gmem) {
+  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(s),
+               "l"(gmem)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;\n" ::: "memory");
 }
@@ -114,8 +120,8 @@ struct ChunkCfg {
   // (delta, delta * x) pairs of a block, one row of BS pairs per channel.
   // Channels whose bit XRB is set keep their row's halves swapped (pair s at
   // s ^ BS/2), which makes both the 16-byte stores (8 lanes: 2 channels x 4
-  // groups at N = 16) and the 8-byte loads (16 lanes: 4 channels) free of
-  // bank conflicts.
+  // groups at N = 16) and the 16-byte loads of two steps' pairs free of bank
+  // conflicts.
   static constexpr int BS = 2 * NG;
   static constexpr int SLOT = BS;
   static constexpr int XRB = NG == 4 ? 1 : 2;
@@ -136,6 +142,8 @@ struct ChunkCfg {
   static_assert(K % NG == 0, "a time block holds whole NG-step blocks");
   static_assert(RAW_P % 16 == 0 && RAW_PB % 16 == 0 && BF_PB % 16 == 0,
                 "cp.async destinations are 16-byte aligned");
+  static_assert(TB > 1 || NG == 1 || (NG % 2 == 0 && SLOT * 8 % 16 == 0),
+                "a half row of exchange pairs is whole 16-byte units");
   static_assert((TB > 1 ? K / NG : TW / (2 * NG)) % 2 == 0,
                 "exchange slots alternate parity from block to block");
   static_assert(TW % kCkptSteps == 0 && kCkptSteps % (2 * NG) == 0,
@@ -232,6 +240,10 @@ scan_chunked_kernel(const ScanParams p) {
   constexpr int CW = Cfg::CW, G = Cfg::G, N = Cfg::N, ESZ = Cfg::ESZ;
   constexpr int THREADS = Cfg::THREADS;
   constexpr unsigned FULL = 0xffffffffu;
+  // the specialised bfloat16 scan stages B and C interleaved per state group
+  // (with the fused convolution this measured slower, so that keeps them
+  // apart)
+  constexpr bool BC_PAIRED = ESZ == 2 && FAST && !CKPT && !CONV;
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ unsigned s_word;
   // fused convolution: the last KH inputs of the previous window, per channel
@@ -345,7 +357,20 @@ scan_chunked_kernel(const ScanParams p) {
       if (has_z) cp_async16(base + 2 * Cfg::RAW_BYTES + so, gz + go, ok);
     }
     unsigned char *bc = base + 3 * Cfg::RAW_BYTES;
-    if constexpr (ESZ == 2) {
+    if constexpr (BC_PAIRED) {
+      // the specialised path's B and C interleaved per state group: 16-byte
+      // unit (r, g) holds B[r, 4g .. 4g+3] then C[r, 4g .. 4g+3], so a lane
+      // reads both with one 16-byte load
+      constexpr int U = TW * N / 4;  // 8-byte units per matrix
+#pragma unroll
+      for (int it = 0; it < (2 * U + THREADS - 1) / THREADS; ++it) {
+        const int idx = tid + it * THREADS;
+        if ((2 * U) % THREADS != 0 && idx >= 2 * U) break;
+        const int q = idx >> 1, m = idx & 1;
+        cp_async8(bc + q * 16 + m * 8,
+                  (m ? gC : gB) + (b * L + t0) * N + int64_t(q) * 4);
+      }
+    } else if constexpr (ESZ == 2) {
       // dense [TW][N] bfloat16 rows, contiguous in memory
       constexpr int CH = TW * N * 2 / 16;
 #pragma unroll
@@ -420,8 +445,10 @@ scan_chunked_kernel(const ScanParams p) {
       const unsigned char *sZ = base + 2 * Cfg::RAW_BYTES;
       const float *sB = nullptr;
       const float *sC = nullptr;
-      // bfloat16 B and C as staged (the specialised path reads them with
-      // 8-byte loads widened in registers; the others from float copies)
+      // bfloat16 B and C as staged (the specialised path reads them widened
+      // in registers: B and C of a state group paired in one 16-byte load,
+      // or, with the fused convolution, 8-byte loads of each; the others
+      // from float copies)
       const T *const rawB =
           reinterpret_cast<const T *>(base + 3 * Cfg::RAW_BYTES);
       const T *const rawC = reinterpret_cast<const T *>(
@@ -493,7 +520,19 @@ scan_chunked_kernel(const ScanParams p) {
       };
       (void)b_row;
       auto bc_row = [&](int r, float4 &Bq, float4 &Cq) {
-        if constexpr (ESZ == 2 && FAST) {
+        if constexpr (BC_PAIRED) {
+          const uint4 v = *reinterpret_cast<const uint4 *>(
+              reinterpret_cast<const unsigned char *>(rawB) +
+              (r * (N / 4) + g) * 16);
+          Bq = make_float4(__uint_as_float(v.x << 16),
+                           __uint_as_float(v.x & 0xffff0000u),
+                           __uint_as_float(v.y << 16),
+                           __uint_as_float(v.y & 0xffff0000u));
+          Cq = make_float4(__uint_as_float(v.z << 16),
+                           __uint_as_float(v.z & 0xffff0000u),
+                           __uint_as_float(v.w << 16),
+                           __uint_as_float(v.w & 0xffff0000u));
+        } else if constexpr (ESZ == 2 && FAST) {
           Bq = Act<T>::load4(rawB + r * N + 4 * g);
           Cq = Act<T>::load4(rawC + r * N + 4 * g);
         } else {
@@ -613,10 +652,17 @@ scan_chunked_kernel(const ScanParams p) {
           }
           float2 dd[BS];
           if constexpr (NG > 1) {
+            // two steps' pairs per 16-byte load (each half of the row is
+            // whole 16-byte units: BS / 2 is even and rows start 16-byte
+            // aligned)
 #pragma unroll
-            for (int s = 0; s < BS; ++s)
-              dd[s] = xch[par * CW * SLOT +
-                          (s < BS / 2 ? xlo + s : xhi + s - BS / 2)];
+            for (int s = 0; s < BS; s += 2) {
+              const float4 v = *reinterpret_cast<const float4 *>(
+                  xch + par * CW * SLOT +
+                  (s < BS / 2 ? xlo + s : xhi + s - BS / 2));
+              dd[s] = make_float2(v.x, v.y);
+              dd[s + 1] = make_float2(v.z, v.w);
+            }
           } else {
             dd[0] = e0;
             dd[1] = e1;

@@ -300,7 +300,8 @@ def test_argument_errors(scan):
     assert call(dims=(1, 0, 16, 4)) == S.SSM_ERR_INVALID
     assert call(dims=(1, 64, 16, 65)) == S.SSM_ERR_UNSUPPORTED
     assert call(dtype=7) == S.SSM_ERR_UNSUPPORTED
-    assert call(flags=4) == S.SSM_ERR_INVALID
+    assert call(flags=1 << 6) == S.SSM_ERR_INVALID            # unknown flag
+    assert call(flags=S.SSM_REUSE_CHECKPOINTS) == S.SSM_ERR_INVALID  # bwd's
     assert call(x=t["x"].data_ptr() + 2) == S.SSM_ERR_ALIGN
     assert call(h0=t["A_log"].data_ptr() + 1) == S.SSM_ERR_ALIGN
     torch.cuda.synchronize()
