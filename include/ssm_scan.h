@@ -364,7 +364,8 @@ SSM_API int ssm_scan_step(ssm_scan_t h, const void *x_new, void *conv_state,
  *              up; the outputs are then invalid. With status NULL the call
  *              never splits (segments 0 then means 1, and segments > 1
  *              returns SSM_ERR_INVALID), so no such wait can go unreported.
- *   flags    : SSM_DELTA_SOFTPLUS and SSM_WRITE_ZOH, as for ssm_scan_fwd.
+ *   flags    : SSM_DELTA_SOFTPLUS and SSM_WRITE_ZOH, as for ssm_scan_fwd
+ *              (SSM_SAVE_CHECKPOINTS: SSM_ERR_INVALID, there is no handle).
  *   the rest : as for ssm_scan_fwd. Additionally dstate is 4, 8 or 16,
  *              dim * element size is a multiple of 16 bytes, and x, delta,
  *              z, B, C are 16-byte aligned (else SSM_ERR_UNSUPPORTED or

@@ -90,8 +90,8 @@ def test_static_scratch_matches_fwd_and_oracle_twice(name):
 def test_static_scratch_rejects_what_does_not_fit():
     """Asking for more pieces than the fixed array can hold is refused on the
     host with SSM_ERR_UNSUPPORTED (buffers are full size all the same); a
-    forced split with no status word to report a given-up wait is refused
-    with SSM_ERR_INVALID."""
+    forced split with no status word to report a given-up wait, and the
+    checkpoint-saving flag, are refused with SSM_ERR_INVALID."""
     b, L, E, N = 1, 16 * 16 * 64, 4096, 16        # 16 pieces need ~12.6 MB
     x = torch.zeros((b, L, E), dtype=torch.float32, device="cuda")
     dl = torch.zeros_like(x)
@@ -108,5 +108,11 @@ def test_static_scratch_rejects_what_does_not_fit():
         0, x, dl, A_log, Bm, Bm, None, None, None, S.SSM_DELTA_SOFTPLUS,
         None, y, None, (b, L, E, N), S.SSM_F32, segments=2, status=None,
         check=False)
+    assert rc == S.SSM_ERR_INVALID
+    # no handle to keep checkpoints in
+    rc = S.ssm_scan_fwd_static_scratch(
+        0, x, dl, A_log, Bm, Bm, None, None, None,
+        S.SSM_DELTA_SOFTPLUS | S.SSM_SAVE_CHECKPOINTS, None, y, None,
+        (b, L, E, N), S.SSM_F32, segments=1, status=status, check=False)
     assert rc == S.SSM_ERR_INVALID
     torch.cuda.synchronize()
