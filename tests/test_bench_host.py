@@ -98,3 +98,45 @@ def test_reference_arm_line(capsys):
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"],
                         "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert "b=1" in d["config"]["workload"]
+
+
+def test_every_op_has_kernel_sources_and_a_config():
+    """Each --op choice names the sources its traffic figure is tied to, and
+    its config record names the operation."""
+    ops = ("scan", "conv", "step", "bwd", "train")
+    wl = _wl(4, 8192, 5120, 16, "bf16")
+    for op in ops:
+        assert op in bench.KERNEL_SOURCES
+        assert len(bench.kernel_source_hash(op)) == 16
+        cfg = bench.workload_config(wl, op, 1, 3)
+        assert cfg["op"] == op and cfg["parallelism"] == "dp1"
+    assert "backward" in bench.workload_config(wl, "bwd", 1, 3)["workload"]
+    assert "training step" in bench.workload_config(wl, "train", 1,
+                                                    3)["workload"]
+    # a world of 2 doubles the global batch (weak scaling)
+    assert bench.workload_config(wl, "scan", 2, 3)["global_batch"] == 8
+
+
+def test_traffic_record_goes_stale_with_its_sources(monkeypatch):
+    """A recorded ncu traffic figure is reported only while the sources it
+    was captured from are unchanged; otherwise the line carries null and
+    says why."""
+    now = bench.kernel_source_hash("scan")
+    monkeypatch.setattr(bench, "NCU_TRAFFIC", {("scan", 3): (1.5e9, now)})
+    value, why = bench.traffic_record("scan", 3)
+    assert value == 1.5e9 and now in why
+    monkeypatch.setattr(bench, "NCU_TRAFFIC",
+                        {("scan", 3): (1.5e9, "0" * 16)})
+    value, why = bench.traffic_record("scan", 3)
+    assert value is None and "stale" in why
+    value, why = bench.traffic_record("bwd", 3)
+    assert value is None and "no ncu capture" in why
+
+
+@pytest.mark.parametrize("op", ["step", "bwd", "train", "conv"])
+def test_reference_arm_times_the_forward_only(capsys, op):
+    rc = bench.main(["--impl", "reference", "--op", op, "--steps", "2",
+                     "--warmup", "3"])
+    assert rc == 0
+    d = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert d["impl"] == "reference" and "unavailable" in d
