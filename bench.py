@@ -205,6 +205,29 @@ class ClockSampler:
         self.proc = None
         self.lines = []
         self.thread = None
+        self.span = None   # (first, last) sample index of the timed region
+
+    def wait_first(self, timeout: float = 3.0):
+        """Block until the sampler has produced a line (nvidia-smi takes a
+        moment to start), at most `timeout` seconds."""
+        t0 = time.time()
+        while self.proc is not None and not self.lines and \
+                time.time() - t0 < timeout:
+            time.sleep(0.01)
+
+    def mark(self, end: bool = False):
+        """Note where the timed region starts (end=False) or ends in the
+        sample stream; the summary then uses the samples taken inside it,
+        plus the first one after it."""
+        if not end:
+            self.span = (len(self.lines), None)
+        elif self.span is not None:
+            t0 = time.time()
+            # the sample that covers the region's last moments
+            while self.proc is not None and len(self.lines) <= self.span[0] \
+                    and time.time() - t0 < 0.5:
+                time.sleep(0.01)
+            self.span = (self.span[0], len(self.lines))
 
     def __enter__(self):
         try:
@@ -236,7 +259,10 @@ class ClockSampler:
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
                  "sw_power_cap"]
-        for ln in self.lines:
+        lines = self.lines
+        if self.span is not None and self.span[1] is not None:
+            lines = self.lines[self.span[0]:self.span[1]] or self.lines
+        for ln in lines:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -538,9 +564,10 @@ def run_gpu(args):
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     with ClockSampler(local) as clocks:
-        time.sleep(0.3)
+        clocks.wait_first()
         barrier()
         torch.cuda.synchronize(dev)
+        clocks.mark()
         t_begin = torch.cuda.Event(enable_timing=True)
         t_end = torch.cuda.Event(enable_timing=True)
         t_begin.record(stream)
@@ -550,8 +577,8 @@ def run_gpu(args):
             ends[i].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize(dev)
+        clocks.mark(end=True)
         barrier()
-        time.sleep(0.2)
     status = scan.sync_status(stream)
     if status != S.SSM_OK:
         raise SystemExit("device status %d in the timed region" % status)

@@ -140,3 +140,20 @@ def test_reference_arm_times_the_forward_only(capsys, op):
     assert rc == 0
     d = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert d["impl"] == "reference" and "unavailable" in d
+
+
+def test_clock_summary_keeps_the_timed_region():
+    """Samples taken before the timed region started are left out; the
+    first sample after it (which covers its last moments) is kept."""
+    c = bench.ClockSampler(0)
+    idle = "0, 600, 1965, 90.0, 0x0, Not Active, Not Active, Not Active, " \
+           "Not Active"
+    busy = "0, 1965, 1965, 900.0, 0x0, Not Active, Not Active, Not Active, " \
+           "Not Active"
+    c.lines = [idle, idle]
+    c.mark()
+    c.lines += [busy, busy]
+    c.mark(end=True)
+    c.lines += [idle]
+    s = c.summary()
+    assert s["sm_mhz"] == 1965.0 and s["samples"] == 2
