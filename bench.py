@@ -86,6 +86,7 @@ CONV_WIDTH = 4
 NCU_TRAFFIC = {
     ("scan", 3): (1.030579456e9 + 0.316773120e9, "8eeadd9c24a3577c"),
     ("step", 3): (0.409518848e9 + 0.330304512e9, "25f3d5fb59a178e8"),
+    ("conv", 3): (1.029994e9 + 0.317378816e9, "8eeadd9c24a3577c"),
     # the reverse sweep, the dominant kernel of both (mean of 7 launches)
     ("bwd", 3): (2.826236635e9 + 0.994677357e9, "f30039c1609bc49d"),
     ("train", 3): (2.826236635e9 + 0.994677357e9, "f30039c1609bc49d"),
