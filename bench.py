@@ -485,13 +485,14 @@ class BwdOp:
                        + (2 + gated) * b * L * E * act + 2 * b * L * N * 4
                        + 2 * E * N * 4 + 4 * E * 4)
         self.grads = None
+        self.det = bool(getattr(args, "deterministic", False))
         self.workload = W.shape_description(args.shape) + "; backward"
 
     def run(self, t, stream):
         self.grads = self.scan.backward(
             t["x"], t["delta"], t["A_log"], t["B"], t["C"], t["dy"],
             D=t["D"], z=t["z"], delta_bias=t["delta_bias"], h0=t["h0"],
-            stream=stream)
+            stream=stream, deterministic=self.det)
 
     def outputs(self):
         return tuple(v for v in self.grads.values() if v is not None)
@@ -524,7 +525,7 @@ class TrainOp(BwdOp):
         self.grads = self.scan.backward(
             t["x"], t["delta"], t["A_log"], t["B"], t["C"], t["dy"],
             D=t["D"], z=t["z"], delta_bias=t["delta_bias"], h0=t["h0"],
-            stream=stream, reuse_checkpoints=True)
+            stream=stream, reuse_checkpoints=True, deterministic=self.det)
 
     def outputs(self):
         return (self.y, self.h_last) + super().outputs()
@@ -714,7 +715,9 @@ def _finish(args, op, world, rank, local, dev, dist, scan, clocks, total_ms,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "io_dtype": wl.dtype, "data": "synthetic",
-        "config": workload_config(wl, op.name, world, args.shape),
+        "config": dict(workload_config(wl, op.name, world, args.shape),
+                       **({"deterministic_sums": True}
+                          if getattr(op, "det", False) else {})),
         "l2": l2,
         "gb_per_s": gbps,
         "roofline": roof,
@@ -778,6 +781,9 @@ def main(argv=None):
                          "backward pass, or a training step (forward "
                          "keeping checkpoints + backward from them)")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--deterministic", action="store_true",
+                    help="--op bwd / train: bitwise reproducible summed "
+                         "gradients (SSM_DETERMINISTIC)")
     ap.add_argument("--reference-seconds", type=float, default=10.0,
                     help="CPU seconds of the oracle sample in cpu_baseline")
     ap.add_argument("--reference-budget", type=float, default=120.0,

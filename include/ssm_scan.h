@@ -123,6 +123,20 @@ enum { SSM_DELTA_SOFTPLUS = 1u << 0, SSM_WRITE_ZOH = 1u << 1 };
  */
 enum { SSM_SAVE_CHECKPOINTS = 1u << 2, SSM_REUSE_CHECKPOINTS = 1u << 3 };
 
+/*
+ * SSM_DETERMINISTIC (ssm_scan_bwd only): the gradients summed over channels
+ * or steps (dB, dC, dA_log, dD, ddelta_bias) are bitwise the same on every
+ * run. Without it they are added with float32 atomics, whose order varies
+ * (a relative run-to-run spread far below the float32 rounding of the
+ * oracle comparison). With it, each thread block writes its share to a
+ * partial array the handle grows (2 * ceil(dim / G) * batch * seqlen *
+ * dstate + batch * dim * (dstate + 2) floats, G = 16, 32 or 64 channels for
+ * dstate 16, 8 or 4; SSM_ERR_NOMEM if it cannot) and fixed-order sums of
+ * those arrays follow on `stream`. The per-element gradients are
+ * deterministic either way.
+ */
+enum { SSM_DETERMINISTIC = 1u << 4 };
+
 /* Status codes. */
 enum {
     SSM_OK = 0,

@@ -38,6 +38,7 @@ SSM_DELTA_SOFTPLUS = 1
 SSM_WRITE_ZOH = 2
 SSM_SAVE_CHECKPOINTS = 4
 SSM_REUSE_CHECKPOINTS = 8
+SSM_DETERMINISTIC = 16
 
 SSM_OK = 0
 SSM_ERR_INVALID = -1
@@ -302,13 +303,16 @@ class SelectiveScan:
 
     def backward(self, x, delta, A_log, B, C, dy, D=None, z=None,
                  delta_bias=None, delta_softplus=True, h0=None, dh_last=None,
-                 write_zoh=False, stream=None, reuse_checkpoints=False):
+                 write_zoh=False, stream=None, reuse_checkpoints=False,
+                 deterministic=False):
         """Gradients of sum(dy * y) + sum(dh_last * h_last) for the scan of
         these inputs. Returns a dict: dx, ddelta, dz (activation dtype; dz
         None without z), dB, dC, dA_log, dD, ddelta_bias, dh0 (float32; dD /
         ddelta_bias None without D / delta_bias). reuse_checkpoints: start
         from the checkpoints of this handle's last forward called with
-        save_checkpoints=True on these same inputs."""
+        save_checkpoints=True on these same inputs. deterministic: the summed
+        gradients bitwise reproducible (fixed-order sums of per-block
+        partials instead of atomics)."""
         import torch
         if x.dtype == torch.float32:
             dtype = SSM_F32
@@ -332,7 +336,8 @@ class SelectiveScan:
             stream = torch.cuda.current_stream(self.device)
         flags = (SSM_DELTA_SOFTPLUS if delta_softplus else 0) | \
             (SSM_WRITE_ZOH if write_zoh else 0) | \
-            (SSM_REUSE_CHECKPOINTS if reuse_checkpoints else 0)
+            (SSM_REUSE_CHECKPOINTS if reuse_checkpoints else 0) | \
+            (SSM_DETERMINISTIC if deterministic else 0)
         ssm_scan_bwd(self.handle, x, delta, A_log, B, C, D, z, delta_bias,
                      flags, h0, dy, dh_last, g["dx"], g["ddelta"], g["dA_log"],
                      g["dB"], g["dC"], g["dD"], g["dz"], g["ddelta_bias"],

@@ -45,6 +45,11 @@ struct BwdParams {
   const void *x, *delta, *z, *dy, *B, *C;  // activation dtype
   const float *A_log, *D, *delta_bias, *h0, *dh_last;
   const float *ckpt;  // [b, ceil(L / 8), E, N]: state before step 8 k
+  // deterministic sums (DET): each block's share of the summed gradients,
+  // added up afterwards in a fixed order instead of by atomics:
+  // part_dB, part_dC [tiles][b, L, N]; part_dA [b][E, N]; part_dD, part_db
+  // [b][E] (written only with D / delta_bias)
+  float *part_dB, *part_dC, *part_dA, *part_dD, *part_db;
   void *dx, *ddelta, *dz;  // [b, L, E] activation dtype (dz: with z only)
   float *dB, *dC;          // [b, L, N], summed into (zero before the launch)
   float *dA_log;           // [E, N], summed into
@@ -96,7 +101,12 @@ struct BwdCfg {
 // those is tested at run time.
 // Held to 18 warps per SM (9 two-warp blocks: the shared-memory limit), so
 // that the Mamba-2.8B layer's 1280 blocks are resident in one wave.
-template <typename T, int NG, int NW, bool ZOH, bool FAST = false>
+// DET: the summed gradients go to per-block partial slices (see BwdParams)
+// instead of float32 atomics, so that a fixed-order reduction makes them
+// bitwise reproducible; the NW warps of a block combine their channel sums
+// through shared memory first, in warp order.
+template <typename T, int NG, int NW, bool ZOH, bool FAST = false,
+          bool DET = false>
 __global__ void __launch_bounds__(32 * NW, 18 / NW)
     scan_bwd_kernel(const BwdParams p) {
   using Cfg = BwdCfg<T, NG, NW>;
@@ -177,11 +187,47 @@ __global__ void __launch_bounds__(32 * NW, 18 / NW)
   const float4 *const hrow = sH + (1 + pr) * RS + warp * 32 + (lane & 3);
   const bool warp_ok = e0 + warp * CW < E;
   // add a lane's sum for history row pr of the half at rb into dst [b, L, N]
-  auto red_row = [&](float *dst, int64_t t0, int rb, float2 v01, float2 v23) {
+  // (DET: the block's sum into its slice of the partial array `part`; slot
+  // 0 or 1 picks the exchange buffer of the pass)
+  const int64_t tile = blockIdx.x - b * tiles;
+  float4 *const sRed = reinterpret_cast<float4 *>(smem + Cfg::SMEM_BYTES);
+  (void)tile;
+  (void)sRed;
+  auto red_row = [&](float *dst, float *part, int slot, int64_t t0, int rb,
+                     float2 v01, float2 v23) {
     const int64_t t = t0 + rb + pr;
-    if (FAST || (warp_ok && t < L))
-      atomicAdd(reinterpret_cast<float4 *>(dst + (b * L + t) * N + 4 * pq),
-                make_float4(v01.x, v01.y, v23.x, v23.y));
+    float4 v = make_float4(v01.x, v01.y, v23.x, v23.y);
+    if constexpr (DET) {
+      (void)dst;
+      // with fewer than 4 state quads, K lanes (bits of lane & 3 above NG)
+      // summed different channels of the same row and quad: add theirs
+#pragma unroll
+      for (int m = NG; m < 4; m <<= 1)
+        v = make_float4(v.x + __shfl_xor_sync(FULL, v.x, m),
+                        v.y + __shfl_xor_sync(FULL, v.y, m),
+                        v.z + __shfl_xor_sync(FULL, v.z, m),
+                        v.w + __shfl_xor_sync(FULL, v.w, m));
+      // warps 1.. hand their sums to warp 0, which adds them in warp order
+      float4 *const sr = sRed + slot * (NW - 1) * 32;
+      if (warp > 0) sr[(warp - 1) * 32 + lane] = v;
+      __syncthreads();
+      if (warp == 0) {
+#pragma unroll
+        for (int k = 0; k < NW - 1; ++k) {
+          const float4 u = sr[k * 32 + lane];
+          v = make_float4(v.x + u.x, v.y + u.y, v.z + u.z, v.w + u.w);
+        }
+        if ((FAST || t < L) && (lane & 3) < NG)
+          *reinterpret_cast<float4 *>(
+              part + ((tile * p.batch + b) * L + t) * N + 4 * pq) = v;
+      }
+    } else {
+      (void)part;
+      (void)slot;
+      if (FAST || (warp_ok && t < L))
+        atomicAdd(reinterpret_cast<float4 *>(dst + (b * L + t) * N + 4 * pq),
+                  v);
+    }
   };
 
   auto stage = [&](int64_t w, int s) {
@@ -366,7 +412,7 @@ __global__ void __launch_bounds__(32 * NW, 18 / NW)
           c01 = fma2(d2, make_float2(hv.x, hv.y), c01);
           c23 = fma2(d2, make_float2(hv.z, hv.w), c23);
         }
-        red_row(p.dC, t0, rb, c01, c23);
+        red_row(p.dC, p.part_dC, 0, t0, rb, c01, c23);
       }
       __syncwarp();
 
@@ -488,7 +534,7 @@ __global__ void __launch_bounds__(32 * NW, 18 / NW)
           b01 = add2(b01, make_float2(v.x, v.y));
           b23 = add2(b23, make_float2(v.z, v.w));
         }
-        red_row(p.dB, t0, rb, b01, b23);
+        red_row(p.dB, p.part_dB, 1, t0, rb, b01, b23);
       }
       __syncwarp();
     }
@@ -505,13 +551,41 @@ __global__ void __launch_bounds__(32 * NW, 18 / NW)
     if (p.dh0)
       *reinterpret_cast<float4 *>(p.dh0 + (b * E + e) * N + 4 * g) =
           make_float4(lam[0], lam[1], lam[2], lam[3]);
+    if constexpr (DET) {  // this batch row's share, summed afterwards
+      *reinterpret_cast<float4 *>(p.part_dA + (b * E + e) * N + 4 * g) =
+          make_float4(dA[0] * Av[0], dA[1] * Av[1], dA[2] * Av[2],
+                      dA[3] * Av[3]);
+      if (g == 0) {
+        if (p.dD) p.part_dD[b * E + e] = sum_dD;
+        if (p.ddelta_bias) p.part_db[b * E + e] = sum_db;
+      }
+    } else {
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      atomicAdd(p.dA_log + e * N + 4 * g + i, dA[i] * Av[i]);
-    if (g == 0) {
-      if (p.dD) atomicAdd(p.dD + e, sum_dD);
-      if (p.ddelta_bias) atomicAdd(p.ddelta_bias + e, sum_db);
+      for (int i = 0; i < 4; ++i)
+        atomicAdd(p.dA_log + e * N + 4 * g + i, dA[i] * Av[i]);
+      if (g == 0) {
+        if (p.dD) atomicAdd(p.dD + e, sum_dD);
+        if (p.ddelta_bias) atomicAdd(p.ddelta_bias + e, sum_db);
+      }
     }
+  }
+}
+
+// out[i] = sum over k = 0 .. slices-1, in that order, of part[k n + i]; n a
+// multiple of 4. The deterministic backward's last step.
+constexpr int kBwdRedBytes = 2 * 32 * 16;  // DET exchange, per extra warp
+__global__ void __launch_bounds__(256)
+    sum_slices_kernel(const float *part, int64_t slices, int64_t n,
+                      float *out) {
+  const int64_t n4 = n / 4;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int64_t k = 0; k < slices; ++k) {
+      const float4 v = __ldcs(reinterpret_cast<const float4 *>(part + k * n) + i);
+      acc = make_float4(acc.x + v.x, acc.y + v.y, acc.z + v.z, acc.w + v.w);
+    }
+    reinterpret_cast<float4 *>(out)[i] = acc;
   }
 }
 

@@ -4,6 +4,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <new>
 
 #include "../../include/ssm_scan.h"
@@ -37,6 +38,9 @@ struct ssm_scan_s {
   // what ckpt holds, when ckpt_saved: the checkpoints of the last forward
   // with SSM_SAVE_CHECKPOINTS, for this shape, dtype and flags
   bool ckpt_saved = false;
+  // deterministic backward: the per-block partial sums
+  float *det = nullptr;
+  size_t det_bytes = 0;
   ssm_scan_dims ckpt_dims{};
   int ckpt_dtype = 0;
   uint32_t ckpt_flags = 0;
@@ -528,6 +532,17 @@ int scan_fwd(ssm_scan_s *h, const void *x, const float *conv_weight,
 }
 
 // ---- backward
+// out = the fixed-order sum of `slices` arrays of n floats (n a multiple of
+// 4), on `s`.
+int sum_slices(const float *part, int64_t slices, int64_t n, float *out,
+               cudaStream_t s) {
+  const int64_t n4 = n / 4;
+  const int64_t grid = std::min<int64_t>((n4 + 255) / 256, 4096);
+  ssm::sum_slices_kernel<<<unsigned(grid < 1 ? 1 : grid), 256, 0, s>>>(
+      part, slices, n, out);
+  return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
 // Two warps per block: the 2.8B layer shape's 1280 blocks then fill 148 SMs
 // at 9 blocks each in one wave, with at most 9 blocks where 8.65 is the
 // mean (4-warp blocks: 5 where the mean is 4.3).
@@ -539,18 +554,36 @@ int launch_bwd(const ssm::BwdParams &p, cudaStream_t s) {
   const int64_t tiles = (p.dim + Cfg::G - 1) / Cfg::G;
   const int64_t blocks = p.batch * tiles;
   if (blocks > 0x7fffffff) return SSM_ERR_UNSUPPORTED;
-  // whole tiles and windows, gated, softplus: the specialised instantiation
+  // whole tiles and windows, gated, softplus: the specialised instantiation;
+  // deterministic sums: per-block partials, then fixed-order reductions
   const bool fast = p.dim % Cfg::G == 0 && p.seqlen % Cfg::TW == 0 && p.z &&
                     p.softplus;
-  auto kern = fast ? ssm::scan_bwd_kernel<T, NG, kBwdWarps, ZOH, true>
-                   : ssm::scan_bwd_kernel<T, NG, kBwdWarps, ZOH, false>;
+  const bool det = p.part_dB != nullptr;
+  auto kern =
+      det ? (fast ? ssm::scan_bwd_kernel<T, NG, kBwdWarps, ZOH, true, true>
+                  : ssm::scan_bwd_kernel<T, NG, kBwdWarps, ZOH, false, true>)
+          : (fast ? ssm::scan_bwd_kernel<T, NG, kBwdWarps, ZOH, true, false>
+                  : ssm::scan_bwd_kernel<T, NG, kBwdWarps, ZOH, false, false>);
+  const int smem =
+      Cfg::SMEM_BYTES + (det ? (kBwdWarps - 1) * ssm::kBwdRedBytes : 0);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           Cfg::SMEM_BYTES) != cudaSuccess) {
+                           smem) != cudaSuccess) {
     cudaGetLastError();
     return SSM_ERR_CUDA;
   }
-  kern<<<unsigned(blocks), Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(p);
-  return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+  kern<<<unsigned(blocks), Cfg::THREADS, smem, s>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return SSM_ERR_CUDA;
+  if (!det) return SSM_OK;
+  const int64_t bln = p.batch * p.seqlen * p.dstate;
+  const int64_t en = p.dim * p.dstate;
+  int rc = sum_slices(p.part_dB, tiles, bln, p.dB, s);
+  if (rc == SSM_OK) rc = sum_slices(p.part_dC, tiles, bln, p.dC, s);
+  if (rc == SSM_OK) rc = sum_slices(p.part_dA, p.batch, en, p.dA_log, s);
+  if (rc == SSM_OK && p.dD)
+    rc = sum_slices(p.part_dD, p.batch, p.dim, p.dD, s);
+  if (rc == SSM_OK && p.ddelta_bias)
+    rc = sum_slices(p.part_db, p.batch, p.dim, p.ddelta_bias, s);
+  return rc;
 }
 
 // The training forward (checkpoints, no y) and the reverse sweep for one
@@ -698,13 +731,14 @@ int ssm_scan_create(ssm_scan_t *out, int device) {
 int ssm_scan_destroy(ssm_scan_t h) {
   if (!h) return SSM_OK;
   int rc = SSM_OK;
-  if (h->ws || h->ctl || h->ckpt) {
+  if (h->ws || h->ctl || h->ckpt || h->det) {
     int prev = 0;
     cudaGetDevice(&prev);
     cudaSetDevice(h->device);
     if (h->ws && cudaFree(h->ws) != cudaSuccess) rc = SSM_ERR_CUDA;
     if (h->ctl && cudaFree(h->ctl) != cudaSuccess) rc = SSM_ERR_CUDA;
     if (h->ckpt && cudaFree(h->ckpt) != cudaSuccess) rc = SSM_ERR_CUDA;
+    if (h->det && cudaFree(h->det) != cudaSuccess) rc = SSM_ERR_CUDA;
     cudaSetDevice(prev);
   }
   delete h;
@@ -821,10 +855,11 @@ int ssm_scan_bwd(ssm_scan_t h, const void *x, const void *delta,
   if (dims.batch <= 0 || dims.seqlen <= 0 || dims.dim <= 0 || dims.dstate <= 0)
     return SSM_ERR_INVALID;
   if (flags & ~uint32_t(SSM_DELTA_SOFTPLUS | SSM_WRITE_ZOH |
-                        SSM_REUSE_CHECKPOINTS))
+                        SSM_REUSE_CHECKPOINTS | SSM_DETERMINISTIC))
     return SSM_ERR_INVALID;
   const bool reuse = (flags & SSM_REUSE_CHECKPOINTS) != 0;
-  flags &= ~uint32_t(SSM_REUSE_CHECKPOINTS);
+  const bool det = (flags & SSM_DETERMINISTIC) != 0;
+  flags &= ~uint32_t(SSM_REUSE_CHECKPOINTS | SSM_DETERMINISTIC);
   if (dtype != SSM_F32 && dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
   const int64_t N = dims.dstate;
   const size_t esz = dtype == SSM_F32 ? 4 : 2;
@@ -870,9 +905,37 @@ int ssm_scan_bwd(ssm_scan_t h, const void *x, const void *delta,
     if (rc != SSM_OK) return rc;
     h->ckpt_saved = false;  // this call's forward overwrites them
   }
-  // ---- the summed outputs cleared
+  // ---- deterministic sums: the partial slices (every element written by
+  // exactly one block, so nothing is cleared); else the summed outputs are
+  // cleared for the atomics
+  size_t det_parts[5] = {0, 0, 0, 0, 0};  // float offsets: dB dC dA dD db
+  if (det) {
+    const int64_t G = (32 / (N / 4)) * kBwdWarps;  // channels per block
+    const int64_t tiles = (dims.dim + G - 1) / G;
+    int64_t bln = 0, slice = 0;
+    if (!mul_ok(rows, N, &bln) || !mul_ok(bln, tiles, &slice))
+      return SSM_ERR_INVALID;
+    const size_t en = size_t(dims.dim) * N, be = size_t(dims.batch) *
+                                                   dims.dim;
+    det_parts[1] = size_t(slice);
+    det_parts[2] = 2 * size_t(slice);
+    det_parts[3] = det_parts[2] + size_t(dims.batch) * en;
+    det_parts[4] = det_parts[3] + be;
+    const size_t need = (det_parts[4] + be) * sizeof(float);
+    if (need > h->det_bytes) {
+      if (h->det) cudaFreeAsync(h->det, s);
+      h->det = nullptr;
+      h->det_bytes = 0;
+      if (cudaMallocAsync(reinterpret_cast<void **>(&h->det), need, s) !=
+          cudaSuccess) {
+        cudaGetLastError();
+        return SSM_ERR_NOMEM;
+      }
+      h->det_bytes = need;
+    }
+  }
   const size_t bcn = size_t(rows) * N * sizeof(float);
-  if (cudaMemsetAsync(dB, 0, bcn, s) != cudaSuccess ||
+  if (!det && (cudaMemsetAsync(dB, 0, bcn, s) != cudaSuccess ||
       cudaMemsetAsync(dC, 0, bcn, s) != cudaSuccess ||
       cudaMemsetAsync(dA_log, 0, size_t(dims.dim) * N * sizeof(float), s) !=
           cudaSuccess ||
@@ -880,7 +943,7 @@ int ssm_scan_bwd(ssm_scan_t h, const void *x, const void *delta,
                  cudaSuccess) ||
       (ddelta_bias &&
        cudaMemsetAsync(ddelta_bias, 0, size_t(dims.dim) * sizeof(float), s) !=
-           cudaSuccess))
+           cudaSuccess)))
     return SSM_ERR_CUDA;
 
   ssm::ScanParams fp{};
@@ -897,6 +960,13 @@ int ssm_scan_bwd(ssm_scan_t h, const void *x, const void *delta,
   bp.x = x; bp.delta = delta; bp.z = z; bp.dy = dy; bp.B = B; bp.C = C;
   bp.A_log = A_log; bp.D = D; bp.delta_bias = delta_bias; bp.h0 = h0;
   bp.dh_last = dh_last; bp.ckpt = h->ckpt;
+  if (det) {
+    bp.part_dB = h->det + det_parts[0];
+    bp.part_dC = h->det + det_parts[1];
+    bp.part_dA = h->det + det_parts[2];
+    bp.part_dD = h->det + det_parts[3];
+    bp.part_db = h->det + det_parts[4];
+  }
   bp.dx = dx; bp.ddelta = ddelta; bp.dz = z ? dz : nullptr;
   bp.dB = dB; bp.dC = dC; bp.dA_log = dA_log;
   bp.dD = D ? dD : nullptr; bp.ddelta_bias = delta_bias ? ddelta_bias : nullptr;

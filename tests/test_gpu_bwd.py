@@ -210,3 +210,75 @@ def test_bwd_argument_errors(scan):
     # dB and dC take 16-byte atomic adds: rejected before any launch
     assert call(dB=dB.data_ptr() + 4) == S.SSM_ERR_ALIGN
     torch.cuda.synchronize()
+
+
+DET_CASES = {
+    "layer_bf16_whole": (3, dict(batch=2, seqlen=256, dim=64, a_jitter=0.5)),
+    "layer_bf16_ragged": (3, dict(batch=2, seqlen=203, dim=40, with_h0=True)),
+    "classifier_f32": (1, dict(batch=2, seqlen=203, dim=72, a_jitter=0.5)),
+    "n8_bf16": (2, dict(batch=2, seqlen=150, dim=48, dstate=8)),
+    "n4_f32_ragged": (0, dict(batch=2, seqlen=100, dim=36, dstate=4)),
+}
+
+
+@pytest.mark.parametrize("zoh", [False, True], ids=["dtBx", "zoh"])
+@pytest.mark.parametrize("name", sorted(DET_CASES))
+def test_bwd_deterministic(scan, name, zoh):
+    """SSM_DETERMINISTIC: every gradient, the channel and step sums
+    included, is the same bit for bit on every run; the gradients match the
+    oracle at the parity bar, and the per-element ones equal the atomic
+    path's bit for bit."""
+    idx, size = DET_CASES[name]
+    wl = W.make(idx, **size)
+    t = to_device(wl)
+    b, L, E, N = wl.batch, wl.seqlen, wl.dim, wl.dstate
+    dy_dev, dy_val, dh = _grads(wl.dtype, ((b, L, E), (b, E, N)), 31)
+    dyt, dht = _dev(dy_dev), torch.from_numpy(dh).cuda()
+
+    def run(det):
+        g = scan.backward(t["x"], t["delta"], t["A_log"], t["B"], t["C"],
+                          dyt, D=t["D"], z=t["z"], delta_bias=t["delta_bias"],
+                          h0=t["h0"], dh_last=dht, write_zoh=zoh,
+                          deterministic=det)
+        torch.cuda.synchronize()
+        return {k: v.float().cpu().numpy() for k, v in g.items()
+                if v is not None}
+
+    runs = [run(True) for _ in range(3)]
+    for k in runs[0]:
+        for r in runs[1:]:
+            assert np.array_equal(r[k], runs[0][k]), k
+    inp = oracle_inputs(wl)
+    ref = oracle.scan_bwd(inp["x"], inp["delta"], inp["A_log"], inp["B"],
+                          inp["C"], dy_val, D=inp["D"], z=inp["z"],
+                          delta_bias=inp["delta_bias"], h0=inp["h0"],
+                          dh_last=dh, write_zoh=zoh)
+    for k, v in runs[0].items():
+        assert rel_err(v, ref[k]) <= TOL[wl.dtype], k
+    atomic = run(False)
+    for k, v in runs[0].items():
+        if k in ("dB", "dC", "dA_log", "dD", "ddelta_bias"):
+            assert rel_err(v, atomic[k]) <= 1e-5, k
+        else:
+            assert np.array_equal(v, atomic[k]), k
+
+
+def test_bwd_deterministic_many_tiles(scan):
+    """64 channel tiles per sum: the deterministic sums repeat bit for bit
+    and agree with the atomic ones to 1e-5."""
+    wl = W.make(3, batch=2, seqlen=2048, dim=1024, a_jitter=0.5)
+    t = to_device(wl)
+    b, L, E, N = wl.batch, wl.seqlen, wl.dim, wl.dstate
+    dy_dev, _, dh = _grads(wl.dtype, ((b, L, E), (b, E, N)), 3)
+    dyt, dht = _dev(dy_dev), torch.from_numpy(dh).cuda()
+    runs = []
+    for det in (True, True, False):
+        g = scan.backward(t["x"], t["delta"], t["A_log"], t["B"], t["C"],
+                          dyt, D=t["D"], z=t["z"], delta_bias=t["delta_bias"],
+                          h0=t["h0"], dh_last=dht, deterministic=det)
+        torch.cuda.synchronize()
+        runs.append({k: v.float().cpu().numpy() for k, v in g.items()
+                     if v is not None})
+    for k in runs[0]:
+        assert np.array_equal(runs[1][k], runs[0][k]), k
+        assert rel_err(runs[0][k], runs[2][k]) <= 1e-5, k

@@ -107,6 +107,19 @@ def test_train_pair(scan, name, zoh):
         assert rel_err(v, ref[k]) <= TOL[wl.dtype], k
     # the backward with its own checkpointing forward gives the same
     _same_gradients(g, _host(_bwd(scan, t, dyt, dht, zoh, reuse=False)))
+    # and with deterministic sums, every gradient is the same bit for bit
+    own = _host(scan.backward(t["x"], t["delta"], t["A_log"], t["B"],
+                              t["C"], dyt, D=t["D"], z=t["z"],
+                              delta_bias=t["delta_bias"], h0=t["h0"],
+                              dh_last=dht, write_zoh=zoh, deterministic=True))
+    _fwd(scan, t, zoh, save=True)
+    reused = _host(scan.backward(t["x"], t["delta"], t["A_log"], t["B"],
+                                 t["C"], dyt, D=t["D"], z=t["z"],
+                                 delta_bias=t["delta_bias"], h0=t["h0"],
+                                 dh_last=dht, write_zoh=zoh,
+                                 reuse_checkpoints=True, deterministic=True))
+    for k in own:
+        assert np.array_equal(reused[k], own[k]), k
 
 
 def test_train_pair_full_size(scan):
