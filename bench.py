@@ -84,13 +84,15 @@ CONV_WIDTH = 4
 # the hash of the kernel sources that capture was taken from. A figure whose
 # sources have changed since is stale: the line then reports null.
 NCU_TRAFFIC = {
-    ("scan", 3): (1.030579456e9 + 0.316773120e9, "8eeadd9c24a3577c"),
-    ("step", 3): (0.409518848e9 + 0.330304512e9, "25f3d5fb59a178e8"),
-    ("conv", 3): (1.029994e9 + 0.317378816e9, "8eeadd9c24a3577c"),
-    # the reverse sweep, the dominant kernel of both (mean of 7 launches)
-    ("bwd", 3): (2.826236635e9 + 0.994677357e9, "f30039c1609bc49d"),
-    ("train", 3): (2.826236635e9 + 0.994677357e9, "f30039c1609bc49d"),
+    ("scan", 3): (1.030875648e9 + 0.317080320e9, "d217f8fde5b3f924"),
+    ("conv", 3): (1.030206720e9 + 0.316482304e9, "d217f8fde5b3f924"),
+    ("step", 3): (0.409519360e9 + 0.329945344e9, "66d2e73009442199"),
+    # the reverse sweep, the dominant kernel of both (mean of 2 launches of
+    # the training step's capture)
+    ("bwd", 3): (2.826098688e9 + 0.994444800e9, "89d2a316a4af5942"),
+    ("train", 3): (2.826098688e9 + 0.994444800e9, "89d2a316a4af5942"),
 }
+
 KERNEL_SOURCES = {
     "scan": ("kernel_chunked.cuh", "device_math.cuh", "scan_params.cuh",
              "ssm_scan_abi.cu"),
