@@ -91,3 +91,37 @@ def test_create_without_a_gpu_fails_cleanly(lib):
     rc = lib.ssm_scan_create(ctypes.byref(h), 0)
     assert rc in (S.SSM_ERR_CUDA, S.SSM_ERR_INVALID)
     assert not h.value
+
+
+def declared_enums():
+    """Every `SSM_NAME = value` enumerator of include/*.h (values written as
+    integers, negative integers or `1u << k`)."""
+    out = {}
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        for body in re.findall(r"enum\s*\{([^}]*)\}", text):
+            body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+            for name, val in re.findall(r"(SSM_\w+)\s*=\s*([^,]+)", body):
+                val = val.strip()
+                m = re.fullmatch(r"1u\s*<<\s*(\d+)", val)
+                out[name] = (1 << int(m.group(1))) if m else int(val)
+    return out
+
+
+def test_binding_constants_match_the_header():
+    """The binding's flag, dtype, status and variant constants carry the
+    header's values, so a flag added to one side cannot drift."""
+    enums = declared_enums()
+    for name in ("SSM_DELTA_SOFTPLUS", "SSM_WRITE_ZOH", "SSM_SAVE_CHECKPOINTS",
+                 "SSM_REUSE_CHECKPOINTS", "SSM_DETERMINISTIC", "SSM_F32",
+                 "SSM_BF16", "SSM_OK", "SSM_ERR_INVALID", "SSM_ERR_TIMEOUT",
+                 "SSM_VARIANT_CHUNKED"):
+        assert name in enums, name
+    for name, val in enums.items():
+        if hasattr(S, name):
+            assert getattr(S, name) == val, name
+    flags = [enums[n] for n in ("SSM_DELTA_SOFTPLUS", "SSM_WRITE_ZOH",
+                                "SSM_SAVE_CHECKPOINTS",
+                                "SSM_REUSE_CHECKPOINTS", "SSM_DETERMINISTIC")]
+    assert len(set(flags)) == len(flags)           # distinct bits
+    assert all(f & (f - 1) == 0 for f in flags)    # one bit each
