@@ -387,7 +387,8 @@ class ScanOp:
         from selective_state_space_51_b200 import workloads as W
         self.name = args.op
         self.launches_per_step = 1
-        self.wl = wl = W.make(plan["shape"], seed=plan["seed"])
+        extra = {"dim": args.dim} if getattr(args, "dim", None) else {}
+        self.wl = wl = W.make(plan["shape"], seed=plan["seed"], **extra)
         self.t = _to_device(wl.dev, dev)
         self.conv = None
         if args.op == "conv":
@@ -719,7 +720,9 @@ def _finish(args, op, world, rank, local, dev, dist, scan, clocks, total_ms,
         "dtype": "f32", "io_dtype": wl.dtype, "data": "synthetic",
         "config": dict(workload_config(wl, op.name, world, args.shape),
                        **({"deterministic_sums": True}
-                          if getattr(op, "det", False) else {})),
+                          if getattr(op, "det", False) else {}),
+                       **({"grid_study_dim": args.dim}
+                          if getattr(args, "dim", None) else {})),
         "l2": l2,
         "gb_per_s": gbps,
         "roofline": roof,
@@ -783,6 +786,10 @@ def main(argv=None):
                          "backward pass, or a training step (forward "
                          "keeping checkpoints + backward from them)")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--dim", type=int, default=None,
+                    help="--op scan / conv: another channel count E for the "
+                         "shape (for studies of the grid; not a bench line "
+                         "of the stated workloads)")
     ap.add_argument("--deterministic", action="store_true",
                     help="--op bwd / train: bitwise reproducible summed "
                          "gradients (SSM_DETERMINISTIC)")
