@@ -222,7 +222,8 @@ enum { kWalkMain = 0, kWalkCorrect = 1 };
 // SAVE: the specialised path's forward that also writes those checkpoints
 // (y and all), for a backward that reuses them.
 template <class Cfg, bool SPLIT, bool ZOH = false, bool CONV = false,
-          bool FAST = false, bool CKPT = false, bool SAVE = false>
+          bool FAST = false, bool CKPT = false, bool SAVE = false,
+          bool DYN = false>
 __global__ void __launch_bounds__(Cfg::THREADS)
 scan_chunked_kernel(const ScanParams p) {
   static_assert(!ZOH || Cfg::TB == 1,
@@ -235,6 +236,8 @@ scan_chunked_kernel(const ScanParams p) {
                 "checkpoints are written by the unsplit one-time-block scan");
   static_assert(!SAVE || (FAST && !CKPT && !CONV),
                 "SAVE is the specialised forward that keeps its checkpoints");
+  static_assert(!DYN || (FAST && !SPLIT && !CKPT),
+                "DYN is the specialised scan run by persistent blocks");
   using T = typename Cfg::T;
   constexpr int NG = Cfg::NG, TB = Cfg::TB, K = Cfg::K, TW = Cfg::TW;
   constexpr int CW = Cfg::CW, G = Cfg::G, N = Cfg::N, ESZ = Cfg::ESZ;
@@ -260,14 +263,24 @@ scan_chunked_kernel(const ScanParams p) {
   const int64_t L = p.seqlen, E = p.dim;
   const int64_t tiles = (E + G - 1) / G;
 
+  // DYN: the blocks are persistent workers, as many as leave every
+  // scheduler the same number of warps. Each pass takes the next unit (a
+  // chunk of seg_len steps of one batch row and channel tile) in ticket
+  // order, chunks of all tiles before the next chunk of any, waits until
+  // the previous chunk of its tile has published its end state, starts
+  // from that state and publishes its own. The state carried is exact, so
+  // no chunk is replayed, and the load stays even at chunk granularity.
+  for (;;) {
   // ---- which (piece, batch row, channel tile) this block scans
   int64_t unit = blockIdx.x;
-  if constexpr (SPLIT) {
+  if constexpr (SPLIT || DYN) {
     if (tid == 0) s_word = atomicAdd(p.ticket, 1u);
     __syncthreads();
     unit = s_word;
     __syncthreads();
   }
+  if constexpr (DYN)
+    if (unit >= int64_t(p.segments) * p.batch * tiles) break;
   const int64_t seg = unit / (p.batch * tiles);
   const int64_t rem = unit - seg * p.batch * tiles;
   const int64_t b = rem / tiles;
@@ -275,8 +288,8 @@ scan_chunked_kernel(const ScanParams p) {
   const int64_t e0 = tile * G;
   const int64_t e = e0 + cl;
   const bool ch_ok = FAST || e < E;
-  const int64_t t_begin = SPLIT ? seg * p.seg_len : 0;
-  const int64_t t_end = SPLIT ? min(L, t_begin + p.seg_len) : L;
+  const int64_t t_begin = (SPLIT || DYN) ? seg * p.seg_len : 0;
+  const int64_t t_end = (SPLIT || DYN) ? min(L, t_begin + p.seg_len) : L;
 
   const T *gx = static_cast<const T *>(p.x);
   const T *gdl = static_cast<const T *>(p.delta);
@@ -306,6 +319,36 @@ scan_chunked_kernel(const ScanParams p) {
       const float *hp = p.h0 + (b * E + e) * N + 4 * g;
       h01 = make_float2(hp[0], hp[1]);
       h23 = make_float2(hp[2], hp[3]);
+    }
+  }
+  if constexpr (DYN) {
+    if (seg > 0) {
+      // the previous chunk's end state, once it is published (bounded wait;
+      // on timeout the status word says so and the chunk starts from zero)
+      const unsigned *flag =
+          p.flags + (b * p.segments + seg - 1) * tiles + tile;
+      if (tid == 0) {
+        const unsigned want = (p.epoch << 2) | kFlagInclusive;
+        bool ok = false;
+        for (unsigned spin = 0; spin < p.spin_limit; ++spin) {
+          if (ld_acquire(flag) == want) {
+            ok = true;
+            break;
+          }
+          __nanosleep(64);
+        }
+        s_word = ok ? 1u : 0u;
+        if (!ok) atomicExch(p.status, kStatusTimeout);
+      }
+      __syncthreads();
+      const bool got = s_word != 0;
+      __syncthreads();
+      float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      if (got)
+        v = __ldcg(reinterpret_cast<const float4 *>(
+            p.incl_state + ((b * p.segments + seg - 1) * E + e) * N + 4 * g));
+      h01 = make_float2(v.x, v.y);
+      h23 = make_float2(v.z, v.w);
     }
   }
   const float bias = (ch_ok && p.delta_bias) ? p.delta_bias[e] : 0.0f;
@@ -858,6 +901,21 @@ scan_chunked_kernel(const ScanParams p) {
   walk(std::integral_constant<int, kWalkMain>(), w_begin, w_end);
 
   float2 H01 = h01, H23 = h23;  // true end state of this piece
+  if constexpr (DYN) {
+    // (the publication test hook: the first chunk of each tile stays
+    // unpublished, so its successor's bounded wait runs out)
+    const bool suppress = (p.debug & kDebugNoPublish) && seg == 0;
+    if (seg + 1 < p.segments && !suppress) {  // the next chunk starts here
+      __stcg(reinterpret_cast<float4 *>(
+                 p.incl_state + ((b * p.segments + seg) * E + e) * N + 4 * g),
+             make_float4(h01.x, h01.y, h23.x, h23.y));
+      __threadfence();
+      __syncthreads();
+      if (tid == 0)
+        st_release(p.flags + (b * p.segments + seg) * tiles + tile,
+                   (p.epoch << 2) | kFlagInclusive);
+    }
+  }
   if constexpr (SPLIT) {
     const int64_t S = p.segments;
     const int64_t slot = ((b * S + seg) * E + e) * N + 4 * g;
@@ -951,6 +1009,8 @@ scan_chunked_kernel(const ScanParams p) {
     hp[2] = H23.x;
     hp[3] = H23.y;
   }
+  if constexpr (!DYN) break;
+  }  // the DYN pass loop
 }
 
 }  // namespace ssm

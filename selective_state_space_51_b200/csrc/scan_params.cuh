@@ -63,6 +63,17 @@ enum { kFlagNone = 0, kFlagAggregate = 1, kFlagInclusive = 2 };
 // Test hooks: the first piece of every sequence never publishes, so its
 // successor's bounded wait must run out and report kStatusTimeout; the
 // decode step uses its per-thread-load kernel instead of the bulk-copy one.
-enum { kDebugNoPublish = 1u << 0, kDebugStepPerThread = 1u << 1 };
+enum {
+  kDebugNoPublish = 1u << 0,
+  kDebugStepPerThread = 1u << 1,
+  // the specialised scan runs on persistent blocks wherever it can, in
+  // chunks of kDynTestChunk steps (tests of the chunk hand-over on small
+  // shapes); kDebugNoDyn: never
+  kDebugForceDyn = 1u << 2,
+  kDebugNoDyn = 1u << 3
+};
+// Steps per chunk of the persistent-block scan, and in its forced test mode.
+constexpr int64_t kDynChunk = 1024;
+constexpr int64_t kDynTestChunk = 64;
 
 }  // namespace ssm

@@ -217,10 +217,11 @@ int64_t auto_segments(const ssm::ScanParams &p, int sm_count) {
 }
 
 template <class Cfg, bool SPLIT, bool ZOH, bool CONV, bool FAST = false,
-          bool CKPT = false, bool SAVE = false>
+          bool CKPT = false, bool SAVE = false, bool DYN = false>
 int launch_kernel(const ssm::ScanParams &p, int64_t blocks, cudaStream_t s) {
   if (blocks > 0x7fffffff) return SSM_ERR_UNSUPPORTED;
-  auto kern = ssm::scan_chunked_kernel<Cfg, SPLIT, ZOH, CONV, FAST, CKPT, SAVE>;
+  auto kern =
+      ssm::scan_chunked_kernel<Cfg, SPLIT, ZOH, CONV, FAST, CKPT, SAVE, DYN>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Cfg::SMEM_BYTES) != cudaSuccess) {
     cudaGetLastError();
@@ -228,6 +229,33 @@ int launch_kernel(const ssm::ScanParams &p, int64_t blocks, cudaStream_t s) {
   }
   kern<<<(unsigned)blocks, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+// Whether the specialised scan of these arguments runs on persistent blocks:
+// when its tiles do not divide evenly over the schedulers (16 warps per SM),
+// blocks take chunks of them in ticket order, so that every scheduler
+// carries the same work, where one block per tile would leave some of them
+// a fifth warp to the end. On yes, sets the chunking in p, grows and clears
+// the hand-over workspace and returns the worker count in *workers (else 0).
+template <class Cfg>
+int plan_dyn(ssm_scan_s *h, ssm::ScanParams &p, int64_t tiles,
+             cudaStream_t s, int64_t *workers) {
+  *workers = 0;
+  const int64_t w = int64_t(h->sm_count) * (16 / Cfg::NW);
+  const int64_t units = p.batch * tiles;
+  const bool force = (h->debug & ssm::kDebugForceDyn) != 0;
+  const int64_t chunk = force ? ssm::kDynTestChunk : ssm::kDynChunk;
+  if (h->segments > 0 || (h->debug & ssm::kDebugNoDyn) ||
+      chunk % Cfg::TW != 0 || p.seqlen <= chunk ||
+      !(force || (units > w && units % w != 0)))
+    return SSM_OK;
+  const int64_t C = (p.seqlen + chunk - 1) / chunk;
+  p.segments = int(C);
+  p.seg_len = chunk;
+  const int rc = ensure_workspace(h, p, tiles, C, s);
+  if (rc != SSM_OK) return rc;
+  *workers = std::min(w, units * C);
+  return SSM_OK;
 }
 
 template <class Cfg, bool ZOH = false, bool CONV = false>
@@ -250,9 +278,16 @@ int launch_chunked(ssm_scan_s *h, ssm::ScanParams &p, int64_t segs_req,
     // whole tiles and windows, gated, softplus, no checkpoints: the
     // specialised kernel tests none of these at run time
     if (segs <= 1 && p.z && p.softplus && !p.ckpt && p.y &&
-        p.dim % Cfg::G == 0 && p.seqlen % Cfg::TW == 0)
+        p.dim % Cfg::G == 0 && p.seqlen % Cfg::TW == 0) {
+      int64_t workers = 0;
+      const int rc = plan_dyn<Cfg>(h, p, tiles, s, &workers);
+      if (rc != SSM_OK) return rc;
+      if (workers > 0)
+        return launch_kernel<Cfg, false, false, CONV, true, false, false,
+                             true>(p, workers, s);
       return launch_kernel<Cfg, false, false, CONV, true>(
           p, p.batch * tiles, s);
+    }
   }
   if (segs <= 1)
     return launch_kernel<Cfg, false, ZOH, CONV>(p, p.batch * tiles, s);
@@ -327,9 +362,17 @@ int launch_save(ssm_scan_s *h, ssm::ScanParams &p, cudaStream_t s) {
   h->last_segments = 1;
   if (p.write_zoh) return launch_kernel<Cfg, false, true, false>(p, blocks, s);
   if (p.z && p.softplus && p.y && p.dim % Cfg::G == 0 &&
-      p.seqlen % Cfg::TW == 0)
+      p.seqlen % Cfg::TW == 0) {
+    int64_t workers = 0;
+    const int rc =
+        plan_dyn<Cfg>(h, p, (p.dim + Cfg::G - 1) / Cfg::G, s, &workers);
+    if (rc != SSM_OK) return rc;
+    if (workers > 0)
+      return launch_kernel<Cfg, false, false, false, true, false, true, true>(
+          p, workers, s);
     return launch_kernel<Cfg, false, false, false, true, false, true>(
         p, blocks, s);
+  }
   return launch_kernel<Cfg, false, false, false>(p, blocks, s);
 }
 

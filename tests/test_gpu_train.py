@@ -44,11 +44,11 @@ def _fwd(scan, t, zoh, save):
     return y, hl
 
 
-def _bwd(scan, t, dyt, dht, zoh, reuse):
+def _bwd(scan, t, dyt, dht, zoh, reuse, det=False):
     return scan.backward(t["x"], t["delta"], t["A_log"], t["B"], t["C"], dyt,
                          D=t["D"], z=t["z"], delta_bias=t["delta_bias"],
                          h0=t["h0"], dh_last=dht, write_zoh=zoh,
-                         reuse_checkpoints=reuse)
+                         reuse_checkpoints=reuse, deterministic=det)
 
 
 def _host(g):
@@ -124,19 +124,24 @@ def test_train_pair(scan, name, zoh):
 
 def test_train_pair_full_size(scan):
     """The Mamba-2.8B layer as the bench runs it: the reused backward equals
-    the self-contained one, and the forward's y equals the plain forward's
-    bit for bit (same kernel arithmetic, checkpoints on the side)."""
+    the self-contained one bit for bit, every gradient (with deterministic
+    sums: at this size the atomic sums of 320 channel tiles spread by about
+    1e-5 run to run), and the forward's y equals the plain forward's bit for
+    bit (same kernel arithmetic, checkpoints on the side)."""
     wl = W.make(3)
     t = to_device(wl)
     dyt, _, dh = _incoming(wl, 23)
     dht = torch.from_numpy(dh).cuda()
     y0, h0 = _fwd(scan, t, False, save=False)
     y0, h0 = y0.clone(), h0.clone()
-    own = _host(_bwd(scan, t, dyt, dht, False, reuse=False))
+    own = _host(_bwd(scan, t, dyt, dht, False, reuse=False, det=True))
     y1, h1 = _fwd(scan, t, False, save=True)
     torch.cuda.synchronize()
     assert torch.equal(y1, y0) and torch.equal(h1, h0)
-    _same_gradients(own, _host(_bwd(scan, t, dyt, dht, False, reuse=True)))
+    reused = _host(_bwd(scan, t, dyt, dht, False, reuse=True, det=True))
+    assert own.keys() == reused.keys()
+    for k in own:
+        assert np.array_equal(reused[k], own[k]), k
 
 
 def test_reuse_needs_matching_checkpoints(scan):
