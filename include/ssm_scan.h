@@ -46,12 +46,16 @@
  *     before anything is launched. A failed launch returns SSM_ERR_CUDA.
  *   - Thread safety: a handle may be used by one host thread at a time, and
  *     carries at most one in-flight call on any stream at a time when it
- *     needs workspace (long sequences with few channels, and the backward
- *     pass's checkpoints). Different handles are independent.
+ *     needs workspace (long sequences with few channels; shapes whose
+ *     channel tiles do not divide evenly over the SMs, which run on
+ *     persistent blocks handing chunks over; the backward pass's
+ *     checkpoints). Different handles are independent.
  *   - CUDA graphs: ssm_scan_step, ssm_scan_fwd and ssm_scan_fwd_conv only
  *     enqueue memsets and kernels once their workspace exists, so their
  *     calls can be captured into a graph and replayed, split sequences
- *     included (each call clears its own publication flags on the stream).
+ *     included (each call clears its own publication flags on the stream),
+ *     and so can the persistent-block scan (it clears its ticket and
+ *     hand-over flags the same way).
  *     Calls that grow a workspace do so on their first use with that shape:
  *     make that call before capturing.
  */
