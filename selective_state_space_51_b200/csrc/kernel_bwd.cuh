@@ -50,6 +50,19 @@ struct BwdParams {
   // part_dB, part_dC [tiles][b, L, N]; part_dA [b][E, N]; part_dD, part_db
   // [b][E] (written only with D / delta_bias)
   float *part_dB, *part_dC, *part_dA, *part_dD, *part_db;
+  // persistent blocks (DYN): units of (chunk, batch row, tile) taken from
+  // *dyn_ticket; chunk k covers windows [nwin - (k + 1) W, nwin - k W)
+  // (W = dyn_chunk_windows), chunks from the end of the sequence. A chunk
+  // hands lam, the dA sums and the dD / bias partials of each thread to the
+  // next (earlier) chunk through dyn_carry [b * tiles][threads][12] (10
+  // used; rows 16-byte aligned), and
+  // sets dyn_flags [b][dyn_chunks][tiles] (cleared before the launch).
+  unsigned *dyn_ticket, *dyn_flags;
+  float *dyn_carry;
+  int dyn_chunks, dyn_chunk_windows;
+  int *status;          // device status word (kStatusTimeout)
+  unsigned spin_limit;  // polls of a hand-over wait
+  unsigned debug;       // kDebugNoPublish: chunk 0 keeps its hand-over back
   void *dx, *ddelta, *dz;  // [b, L, E] activation dtype (dz: with z only)
   float *dB, *dC;          // [b, L, N], summed into (zero before the launch)
   float *dA_log;           // [E, N], summed into
@@ -100,14 +113,19 @@ struct BwdCfg {
 // windows (L a multiple of TW), a gate and the softplus step, so none of
 // those is tested at run time.
 // Held to 18 warps per SM (9 two-warp blocks: the shared-memory limit), so
-// that the Mamba-2.8B layer's 1280 blocks are resident in one wave.
+// that the Mamba-2.8B layer's 1280 blocks are resident in one wave; the
+// persistent variant to the 16 warps per SM it runs.
 // DET: the summed gradients go to per-block partial slices (see BwdParams)
 // instead of float32 atomics, so that a fixed-order reduction makes them
 // bitwise reproducible; the NW warps of a block combine their channel sums
 // through shared memory first, in warp order.
+// DYN (with FAST): persistent blocks over (chunk, batch row, tile) units,
+// the sweep's state handed from chunk to chunk (see BwdParams), so that
+// every scheduler carries the same work where the tiles do not divide
+// evenly over the SMs.
 template <typename T, int NG, int NW, bool ZOH, bool FAST = false,
-          bool DET = false>
-__global__ void __launch_bounds__(32 * NW, 18 / NW)
+          bool DET = false, bool DYN = false>
+__global__ void __launch_bounds__(32 * NW, (DYN ? 16 : 18) / NW)
     scan_bwd_kernel(const BwdParams p) {
   using Cfg = BwdCfg<T, NG, NW>;
   constexpr int N = Cfg::N, CW = Cfg::CW, G = Cfg::G, TW = Cfg::TW;
@@ -121,14 +139,34 @@ __global__ void __launch_bounds__(32 * NW, 18 / NW)
   const int c = lane / NG;
   const int cl = warp * CW + c;  // channel within the tile
 
+  static_assert(!DYN || FAST, "persistent blocks run the specialised sweep");
   const int64_t L = p.seqlen, E = p.dim;
   const int64_t tiles = (E + G - 1) / G;
-  const int64_t b = blockIdx.x / tiles;
-  const int64_t e0 = (blockIdx.x - b * tiles) * G;
-  const int64_t e = e0 + cl;
-  const bool ch_ok = FAST || e < E;
   const int64_t nwin = (L + TW - 1) / TW;
   const int64_t nck = (L + kCkptSteps - 1) / kCkptSteps;  // checkpoints
+  __shared__ unsigned s_unit;
+  (void)s_unit;
+
+  for (;;) {  // DYN: one unit per pass; else one pass
+  int64_t unit = blockIdx.x, chunk = 0;
+  if constexpr (DYN) {
+    if (tid == 0) s_unit = atomicAdd(p.dyn_ticket, 1u);
+    __syncthreads();
+    unit = s_unit;
+    __syncthreads();
+    if (unit >= int64_t(p.dyn_chunks) * p.batch * tiles) break;
+    chunk = unit / (p.batch * tiles);
+    unit -= chunk * p.batch * tiles;
+  }
+  const int64_t b = unit / tiles;
+  const int64_t tile = unit - b * tiles;
+  const int64_t e0 = tile * G;
+  const int64_t e = e0 + cl;
+  const bool ch_ok = FAST || e < E;
+  // this unit's windows [w_lo, w_hi)
+  const int64_t w_hi = DYN ? nwin - chunk * p.dyn_chunk_windows : nwin;
+  const int64_t w_lo =
+      DYN ? (w_hi > p.dyn_chunk_windows ? w_hi - p.dyn_chunk_windows : 0) : 0;
 
   float *const sS = reinterpret_cast<float *>(smem + 2 * Cfg::STAGE);
   float *const sX = sS + TW * SP;
@@ -189,7 +227,6 @@ __global__ void __launch_bounds__(32 * NW, 18 / NW)
   // add a lane's sum for history row pr of the half at rb into dst [b, L, N]
   // (DET: the block's sum into its slice of the partial array `part`; slot
   // 0 or 1 picks the exchange buffer of the pass)
-  const int64_t tile = blockIdx.x - b * tiles;
   float4 *const sRed = reinterpret_cast<float4 *>(smem + Cfg::SMEM_BYTES);
   (void)tile;
   (void)sRed;
@@ -271,17 +308,52 @@ __global__ void __launch_bounds__(32 * NW, 18 / NW)
     }
   };
 
-  const int64_t w_last = nwin - 1;
+  const int64_t w_last = w_hi - 1;
   stage(w_last, 0);
   cp_async_commit();
   load_ckpts(w_last);
-  for (int64_t w = w_last; w >= 0; --w) {
+  if constexpr (DYN) {
+    if (chunk > 0) {
+      // the later chunk's hand-over, once published (bounded wait; on
+      // timeout the status word says so and this chunk starts from zero)
+      const unsigned *flag =
+          p.dyn_flags + (b * p.dyn_chunks + chunk - 1) * tiles + tile;
+      if (tid == 0) {
+        bool ok = false;
+        for (unsigned spin = 0; spin < p.spin_limit; ++spin) {
+          if (ld_acquire(flag) != 0u) {
+            ok = true;
+            break;
+          }
+          __nanosleep(64);
+        }
+        s_unit = ok ? 1u : 0u;
+        if (!ok) atomicExch(p.status, kStatusTimeout);
+      }
+      __syncthreads();
+      const bool got = s_unit != 0u;
+      __syncthreads();
+      const float *cv =
+          p.dyn_carry + ((b * tiles + tile) * THREADS + tid) * 12;
+      const float4 u0 = got ? __ldcg(reinterpret_cast<const float4 *>(cv))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 u1 = got ? __ldcg(reinterpret_cast<const float4 *>(cv + 4))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float2 u2 = got ? __ldcg(reinterpret_cast<const float2 *>(cv + 8))
+                            : make_float2(0.f, 0.f);
+      lam[0] = u0.x; lam[1] = u0.y; lam[2] = u0.z; lam[3] = u0.w;
+      dA[0] = u1.x; dA[1] = u1.y; dA[2] = u1.z; dA[3] = u1.w;
+      sum_dD = u2.x;
+      sum_db = u2.y;
+    }
+  }
+  for (int64_t w = w_last; w >= w_lo; --w) {
     const int par = int((w_last - w) & 1);
     // this window's tiles have landed, and every thread is done with the
     // previous window, whose buffer now takes the next window's tiles
     cp_async_wait<0>();
     __syncthreads();
-    if (w > 0) stage(w - 1, par ^ 1);
+    if (w > w_lo) stage(w - 1, par ^ 1);
     cp_async_commit();
 
     const int64_t t0 = w * TW;
@@ -340,7 +412,7 @@ __global__ void __launch_bounds__(32 * NW, 18 / NW)
     // (this window's checkpoints were loaded during the previous window)
     const float hck[4] = {ck_lo.x, ck_lo.y, ck_lo.z, ck_lo.w};
     const float hmid[4] = {ck_hi.x, ck_hi.y, ck_hi.z, ck_hi.w};
-    if (w > 0) load_ckpts(w - 1);
+    if (w > w_lo) load_ckpts(w - 1);
     // advance h over rows [r0, r0 + HALF); STORE: keep each state in sH
     // (row 1 + r - r0)
     auto recompute = [&](float (&h)[4], int r0, bool store) {
@@ -540,6 +612,23 @@ __global__ void __launch_bounds__(32 * NW, 18 / NW)
     }
   }
   cp_async_wait<0>();
+  if constexpr (DYN) {
+    if (w_lo > 0) {  // an earlier chunk goes on from here
+      float *const cv =
+          p.dyn_carry + ((b * tiles + tile) * THREADS + tid) * 12;
+      __stcg(reinterpret_cast<float4 *>(cv),
+             make_float4(lam[0], lam[1], lam[2], lam[3]));
+      __stcg(reinterpret_cast<float4 *>(cv + 4),
+             make_float4(dA[0], dA[1], dA[2], dA[3]));
+      __stcg(reinterpret_cast<float2 *>(cv + 8), make_float2(sum_dD, sum_db));
+      __threadfence();
+      __syncthreads();
+      if (tid == 0 && !((p.debug & kDebugNoPublish) && chunk == 0))
+        st_release(p.dyn_flags + (b * p.dyn_chunks + chunk) * tiles + tile,
+                   1u);
+      continue;
+    }
+  }
   // every lane of a channel finished some of its steps: sum the partials
 #pragma unroll
   for (int m = 1; m < NG; m <<= 1) {
@@ -569,6 +658,8 @@ __global__ void __launch_bounds__(32 * NW, 18 / NW)
       }
     }
   }
+  if constexpr (!DYN) break;
+  }  // the DYN pass loop
 }
 
 // out[i] = sum over k = 0 .. slices-1, in that order, of part[k n + i]; n a

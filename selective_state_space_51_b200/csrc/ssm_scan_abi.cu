@@ -41,6 +41,9 @@ struct ssm_scan_s {
   // deterministic backward: the per-block partial sums
   float *det = nullptr;
   size_t det_bytes = 0;
+  // persistent-block backward: hand-over flags and carried sums
+  void *bdyn = nullptr;
+  size_t bdyn_bytes = 0;
   ssm_scan_dims ckpt_dims{};
   int ckpt_dtype = 0;
   uint32_t ckpt_flags = 0;
@@ -592,7 +595,7 @@ int sum_slices(const float *part, int64_t slices, int64_t n, float *out,
 constexpr int kBwdWarps = 2;
 
 template <typename T, int NG, bool ZOH>
-int launch_bwd(const ssm::BwdParams &p, cudaStream_t s) {
+int launch_bwd(ssm_scan_s *h, ssm::BwdParams &p, cudaStream_t s) {
   using Cfg = ssm::BwdCfg<T, NG, kBwdWarps>;
   const int64_t tiles = (p.dim + Cfg::G - 1) / Cfg::G;
   const int64_t blocks = p.batch * tiles;
@@ -602,8 +605,62 @@ int launch_bwd(const ssm::BwdParams &p, cudaStream_t s) {
   const bool fast = p.dim % Cfg::G == 0 && p.seqlen % Cfg::TW == 0 && p.z &&
                     p.softplus;
   const bool det = p.part_dB != nullptr;
+  // persistent blocks where the tiles do not divide evenly over 16 warps per
+  // SM (as in the forward): chunks of the sweep hand their state over
+  int64_t grid = blocks;
+  bool dyn = false;
+  if (fast && !(h->debug & ssm::kDebugNoDyn)) {
+    const bool force = (h->debug & ssm::kDebugForceDyn) != 0;
+    const int64_t wc = (force ? ssm::kDynTestChunk : ssm::kDynChunk) / Cfg::TW;
+    const int64_t nwin = p.seqlen / Cfg::TW;
+    const int64_t workers = int64_t(h->sm_count) * (16 / kBwdWarps);
+    if (wc > 0 && nwin > wc &&
+        (force || (blocks > workers && blocks % workers != 0))) {
+      const int64_t C = (nwin + wc - 1) / wc;
+      const size_t nflags = size_t(p.batch) * C * tiles;
+      const size_t off = align256(nflags * sizeof(unsigned));
+      const size_t need =
+          off + size_t(blocks) * Cfg::THREADS * 12 * sizeof(float);
+      int rc = ensure_ctl(h, s);
+      if (rc != SSM_OK) return rc;
+      if (need > h->bdyn_bytes) {
+        if (h->bdyn) cudaFreeAsync(h->bdyn, s);
+        h->bdyn = nullptr;
+        h->bdyn_bytes = 0;
+        if (cudaMallocAsync(&h->bdyn, need, s) != cudaSuccess) {
+          cudaGetLastError();
+          return SSM_ERR_NOMEM;
+        }
+        h->bdyn_bytes = need;
+      }
+      unsigned char *base = static_cast<unsigned char *>(h->bdyn);
+      p.dyn_flags = reinterpret_cast<unsigned *>(base);
+      p.dyn_carry = reinterpret_cast<float *>(base + off);
+      p.dyn_ticket = reinterpret_cast<unsigned *>(h->ctl + 1);
+      p.dyn_chunks = int(C);
+      p.dyn_chunk_windows = int(wc);
+      p.status = h->ctl;
+      p.spin_limit = h->spin_limit;
+      p.debug = h->debug;
+      // the ticket restarts and the hand-over flags are cleared on the
+      // stream before every launch (graph replays included)
+      if (cudaMemsetAsync(p.dyn_ticket, 0, sizeof(unsigned), s) !=
+              cudaSuccess ||
+          cudaMemsetAsync(p.dyn_flags, 0, nflags * sizeof(unsigned), s) !=
+              cudaSuccess) {
+        cudaGetLastError();
+        return SSM_ERR_CUDA;
+      }
+      dyn = true;
+      grid = std::min<int64_t>(workers, blocks * C);
+    }
+  }
   auto kern =
-      det ? (fast ? ssm::scan_bwd_kernel<T, NG, kBwdWarps, ZOH, true, true>
+      dyn ? (det ? ssm::scan_bwd_kernel<T, NG, kBwdWarps, ZOH, true, true, true>
+                 : ssm::scan_bwd_kernel<T, NG, kBwdWarps, ZOH, true, false,
+                                        true>)
+      : det
+          ? (fast ? ssm::scan_bwd_kernel<T, NG, kBwdWarps, ZOH, true, true>
                   : ssm::scan_bwd_kernel<T, NG, kBwdWarps, ZOH, false, true>)
           : (fast ? ssm::scan_bwd_kernel<T, NG, kBwdWarps, ZOH, true, false>
                   : ssm::scan_bwd_kernel<T, NG, kBwdWarps, ZOH, false, false>);
@@ -614,7 +671,7 @@ int launch_bwd(const ssm::BwdParams &p, cudaStream_t s) {
     cudaGetLastError();
     return SSM_ERR_CUDA;
   }
-  kern<<<unsigned(blocks), Cfg::THREADS, smem, s>>>(p);
+  kern<<<unsigned(grid), Cfg::THREADS, smem, s>>>(p);
   if (cudaGetLastError() != cudaSuccess) return SSM_ERR_CUDA;
   if (!det) return SSM_OK;
   const int64_t bln = p.batch * p.seqlen * p.dstate;
@@ -634,11 +691,11 @@ int launch_bwd(const ssm::BwdParams &p, cudaStream_t s) {
 // reverse sweep alone, from the checkpoints a SSM_SAVE_CHECKPOINTS forward
 // left.
 template <class Cf, typename T, int NG>
-int run_bwd(ssm::ScanParams &fp, const ssm::BwdParams &bp, bool reuse,
-            cudaStream_t s) {
+int run_bwd(ssm_scan_s *h, ssm::ScanParams &fp, ssm::BwdParams &bp,
+            bool reuse, cudaStream_t s) {
   if (reuse)  // the training forward left the checkpoints
-    return fp.write_zoh ? launch_bwd<T, NG, true>(bp, s)
-                        : launch_bwd<T, NG, false>(bp, s);
+    return fp.write_zoh ? launch_bwd<T, NG, true>(h, bp, s)
+                        : launch_bwd<T, NG, false>(h, bp, s);
   const int64_t tiles = (fp.dim + Cf::G - 1) / Cf::G;
   const int64_t blocks = fp.batch * tiles;
   // the checkpoint-only forward: no readout, C and z not read; with whole
@@ -654,8 +711,8 @@ int run_bwd(ssm::ScanParams &fp, const ssm::BwdParams &bp, bool reuse,
                : launch_kernel<Cf, false, false, false, false, true>(fp, blocks,
                                                                     s);
   if (rc != SSM_OK) return rc;
-  return fp.write_zoh ? launch_bwd<T, NG, true>(bp, s)
-                      : launch_bwd<T, NG, false>(bp, s);
+  return fp.write_zoh ? launch_bwd<T, NG, true>(h, bp, s)
+                      : launch_bwd<T, NG, false>(h, bp, s);
 }
 
 }  // namespace
@@ -774,7 +831,7 @@ int ssm_scan_create(ssm_scan_t *out, int device) {
 int ssm_scan_destroy(ssm_scan_t h) {
   if (!h) return SSM_OK;
   int rc = SSM_OK;
-  if (h->ws || h->ctl || h->ckpt || h->det) {
+  if (h->ws || h->ctl || h->ckpt || h->det || h->bdyn) {
     int prev = 0;
     cudaGetDevice(&prev);
     cudaSetDevice(h->device);
@@ -782,6 +839,7 @@ int ssm_scan_destroy(ssm_scan_t h) {
     if (h->ctl && cudaFree(h->ctl) != cudaSuccess) rc = SSM_ERR_CUDA;
     if (h->ckpt && cudaFree(h->ckpt) != cudaSuccess) rc = SSM_ERR_CUDA;
     if (h->det && cudaFree(h->det) != cudaSuccess) rc = SSM_ERR_CUDA;
+    if (h->bdyn && cudaFree(h->bdyn) != cudaSuccess) rc = SSM_ERR_CUDA;
     cudaSetDevice(prev);
   }
   delete h;
@@ -1018,12 +1076,12 @@ int ssm_scan_bwd(ssm_scan_t h, const void *x, const void *delta,
   bp.dstate = int(N); bp.softplus = fp.softplus;
 
   if (dtype == SSM_BF16) {
-    if (N == 16) return run_bwd<C16b1, __nv_bfloat16, 4>(fp, bp, reuse, s);
-    return run_bwd<C8b1, __nv_bfloat16, 2>(fp, bp, reuse, s);
+    if (N == 16) return run_bwd<C16b1, __nv_bfloat16, 4>(h, fp, bp, reuse, s);
+    return run_bwd<C8b1, __nv_bfloat16, 2>(h, fp, bp, reuse, s);
   }
-  if (N == 16) return run_bwd<C16f1, float, 4>(fp, bp, reuse, s);
-  if (N == 8) return run_bwd<C8f1, float, 2>(fp, bp, reuse, s);
-  return run_bwd<C4f1, float, 1>(fp, bp, reuse, s);
+  if (N == 16) return run_bwd<C16f1, float, 4>(h, fp, bp, reuse, s);
+  if (N == 8) return run_bwd<C8f1, float, 2>(h, fp, bp, reuse, s);
+  return run_bwd<C4f1, float, 1>(h, fp, bp, reuse, s);
 }
 
 }  // extern "C"

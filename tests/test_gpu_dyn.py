@@ -211,3 +211,94 @@ def test_forced_chunks_keep_the_training_checkpoints(scan):
     torch.cuda.synchronize()
     for k, v in own.items():
         assert torch.equal(g[k], v), k
+
+
+BWD_CASES = {
+    "bf16_L256": (3, dict(batch=2, seqlen=256, dim=64, a_jitter=0.5)),
+    "f32_L160_h0": (1, dict(batch=2, seqlen=160, dim=64, with_h0=True)),
+    "bf16_n8_L192": (2, dict(batch=2, seqlen=192, dim=64, dstate=8)),
+}
+
+
+def _bwd_all(scan, t, dy, dh, flags, zoh=False, det=True):
+    _debug(scan, flags)
+    try:
+        g = scan.backward(t["x"], t["delta"], t["A_log"], t["B"], t["C"], dy,
+                          D=t["D"], z=t["z"], delta_bias=t["delta_bias"],
+                          h0=t["h0"], dh_last=dh, write_zoh=zoh,
+                          deterministic=det)
+        torch.cuda.synchronize()
+        assert scan.sync_status() == S.SSM_OK
+        return {k: v.clone() for k, v in g.items() if v is not None}
+    finally:
+        _debug(scan, 0)
+
+
+def _incoming(wl, seed):
+    rng = np.random.Generator(np.random.PCG64(seed))
+    dy = rng.standard_normal((wl.batch, wl.seqlen, wl.dim), dtype=np.float32)
+    dh = rng.standard_normal((wl.batch, wl.dim, wl.dstate), dtype=np.float32)
+    if wl.dtype == W.BF16:
+        bits = W.round_to_bf16_bits(dy)
+        return (torch.from_numpy(bits.view(np.int16)).cuda()
+                .view(torch.bfloat16), W.bf16_bits_to_f32(bits), dh)
+    return torch.from_numpy(dy).cuda(), dy, dh
+
+
+@pytest.mark.parametrize("zoh", [False, True], ids=["dtBx", "zoh"])
+@pytest.mark.parametrize("name", sorted(BWD_CASES))
+def test_backward_chunks_match_one_block_per_tile_and_oracle(scan, name, zoh):
+    """The reverse sweep on persistent blocks (forced 4-window chunks, the
+    sweep's adjoint and sums handed from each chunk to the earlier one):
+    every gradient equal bit for bit to one block per tile (deterministic
+    sums in both), and the oracle at the parity bar."""
+    idx, size = BWD_CASES[name]
+    wl = W.make(idx, **size)
+    t = to_device(wl)
+    dy, dy_val, dh = _incoming(wl, 41)
+    dht = torch.from_numpy(dh).cuda()
+    ref_gpu = _bwd_all(scan, t, dy, dht, NO_DYN, zoh)
+    got = _bwd_all(scan, t, dy, dht, FORCE_DYN, zoh)
+    assert got.keys() == ref_gpu.keys()
+    for k in got:
+        assert torch.equal(got[k], ref_gpu[k]), k
+    inp = oracle_inputs(wl)
+    ref = oracle.scan_bwd(inp["x"], inp["delta"], inp["A_log"], inp["B"],
+                          inp["C"], dy_val, D=inp["D"], z=inp["z"],
+                          delta_bias=inp["delta_bias"], h0=inp["h0"],
+                          dh_last=dh, write_zoh=zoh)
+    for k, v in got.items():
+        assert rel_err(v.float().cpu().numpy(), ref[k]) <= TOL[wl.dtype], k
+
+
+def test_backward_uneven_tiles_take_the_persistent_path(scan):
+    """1200 tiles for 148 x 8 workers, 1024-step chunks: bit for bit the
+    gradients of one block per tile (deterministic sums)."""
+    wl = W.make(3, batch=8, seqlen=2048, dim=2400, a_jitter=0.5)
+    t = to_device(wl)
+    dy, _, dh = _incoming(wl, 43)
+    dht = torch.from_numpy(dh).cuda()
+    ref_gpu = _bwd_all(scan, t, dy, dht, NO_DYN)
+    got = _bwd_all(scan, t, dy, dht, 0)
+    for k in got:
+        assert torch.equal(got[k], ref_gpu[k]), k
+
+
+def test_backward_unpublished_chunk_times_out_and_recovers(scan):
+    wl = W.make(3, batch=2, seqlen=256, dim=32)
+    t = to_device(wl)
+    dy, _, dh = _incoming(wl, 47)
+    dht = torch.from_numpy(dh).cuda()
+    ok = _bwd_all(scan, t, dy, dht, NO_DYN)
+    _debug(scan, FORCE_DYN | NO_PUBLISH, 2000)
+    try:
+        scan.backward(t["x"], t["delta"], t["A_log"], t["B"], t["C"], dy,
+                      D=t["D"], z=t["z"], delta_bias=t["delta_bias"],
+                      dh_last=dht, deterministic=True)
+        torch.cuda.synchronize()
+        assert scan.sync_status() == S.SSM_ERR_TIMEOUT
+    finally:
+        _debug(scan, 0)
+    again = _bwd_all(scan, t, dy, dht, FORCE_DYN)
+    for k in ok:
+        assert torch.equal(again[k], ok[k]), k
