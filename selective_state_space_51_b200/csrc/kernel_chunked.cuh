@@ -236,7 +236,7 @@ scan_chunked_kernel(const ScanParams p) {
                 "checkpoints are written by the unsplit one-time-block scan");
   static_assert(!SAVE || (FAST && !CKPT && !CONV),
                 "SAVE is the specialised forward that keeps its checkpoints");
-  static_assert(!DYN || (FAST && !SPLIT && !CKPT),
+  static_assert(!DYN || (FAST && !SPLIT),
                 "DYN is the specialised scan run by persistent blocks");
   using T = typename Cfg::T;
   constexpr int NG = Cfg::NG, TB = Cfg::TB, K = Cfg::K, TW = Cfg::TW;

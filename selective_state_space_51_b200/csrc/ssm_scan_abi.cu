@@ -702,14 +702,19 @@ int run_bwd(ssm_scan_s *h, ssm::ScanParams &fp, ssm::BwdParams &bp,
   // tiles and windows and the softplus step, the specialised instantiation
   const bool fast = !fp.write_zoh && fp.softplus && fp.dim % Cf::G == 0 &&
                     fp.seqlen % Cf::TW == 0;
-  int rc = fp.write_zoh
-               ? launch_kernel<Cf, false, true, false, false, true>(fp, blocks,
-                                                                   s)
-           : fast
-               ? launch_kernel<Cf, false, false, false, true, true>(fp, blocks,
-                                                                   s)
-               : launch_kernel<Cf, false, false, false, false, true>(fp, blocks,
-                                                                    s);
+  int64_t workers = 0;
+  int rc = SSM_OK;
+  if (fast) rc = plan_dyn<Cf>(h, fp, tiles, s, &workers);
+  if (rc != SSM_OK) return rc;
+  rc = fp.write_zoh
+           ? launch_kernel<Cf, false, true, false, false, true>(fp, blocks, s)
+       : workers > 0
+           ? launch_kernel<Cf, false, false, false, true, true, false, true>(
+                 fp, workers, s)
+       : fast
+           ? launch_kernel<Cf, false, false, false, true, true>(fp, blocks, s)
+           : launch_kernel<Cf, false, false, false, false, true>(fp, blocks,
+                                                                s);
   if (rc != SSM_OK) return rc;
   return fp.write_zoh ? launch_bwd<T, NG, true>(h, bp, s)
                       : launch_bwd<T, NG, false>(h, bp, s);
