@@ -84,14 +84,15 @@ CONV_WIDTH = 4
 # the hash of the kernel sources that capture was taken from. A figure whose
 # sources have changed since is stale: the line then reports null.
 NCU_TRAFFIC = {
-    ("scan", 3): (1.030875648e9 + 0.317080320e9, "d217f8fde5b3f924"),
-    ("conv", 3): (1.030206720e9 + 0.316482304e9, "d217f8fde5b3f924"),
-    ("step", 3): (0.409519360e9 + 0.329945344e9, "66d2e73009442199"),
+    ("scan", 3): (1.084032768e9 + 0.328505088e9, "716d66fa5be1b7fd"),
+    ("conv", 3): (1.041672960e9 + 0.327872512e9, "716d66fa5be1b7fd"),
+    ("step", 3): (0.409533184e9 + 0.330125056e9, "5ea473594a5cc7eb"),
     # the reverse sweep, the dominant kernel of both (mean of 2 launches of
     # the training step's capture)
-    ("bwd", 3): (2.826098688e9 + 0.994444800e9, "89d2a316a4af5942"),
-    ("train", 3): (2.826098688e9 + 0.994444800e9, "89d2a316a4af5942"),
+    ("bwd", 3): (2.799154560e9 + 1.014581632e9, "ea513157fd3e3039"),
+    ("train", 3): (2.799154560e9 + 1.014581632e9, "ea513157fd3e3039"),
 }
+
 
 KERNEL_SOURCES = {
     "scan": ("kernel_chunked.cuh", "device_math.cuh", "scan_params.cuh",
