@@ -73,7 +73,7 @@ enum {
   kDebugNoDyn = 1u << 3
 };
 // Steps per chunk of the persistent-block scan, and in its forced test mode.
-constexpr int64_t kDynChunk = 1024;
+constexpr int64_t kDynChunk = 512;
 constexpr int64_t kDynTestChunk = 64;
 
 }  // namespace ssm

@@ -73,7 +73,7 @@ def test_forced_chunks_match_one_block_per_tile_and_oracle(scan, name):
 
 def test_uneven_tiles_take_the_persistent_path(scan):
     """8 sequences x 150 tiles = 1200 units for 148 x 8 two-warp workers:
-    the shape the path is for, with 1024-step chunks. Bitwise equal to one
+    the shape the path is for, with its default chunks. Bitwise equal to one
     block per tile, and to the oracle on sampled channels."""
     wl = W.make(3, batch=8, seqlen=2048, dim=2400, a_jitter=0.5)
     t = to_device(wl)
@@ -272,7 +272,7 @@ def test_backward_chunks_match_one_block_per_tile_and_oracle(scan, name, zoh):
 
 
 def test_backward_uneven_tiles_take_the_persistent_path(scan):
-    """1200 tiles for 148 x 8 workers, 1024-step chunks: bit for bit the
+    """1200 tiles for 148 x 8 workers, default chunks: bit for bit the
     gradients of one block per tile (deterministic sums)."""
     wl = W.make(3, batch=8, seqlen=2048, dim=2400, a_jitter=0.5)
     t = to_device(wl)
